@@ -1,0 +1,463 @@
+#!/usr/bin/env python
+"""Throughput of the quantized linear layer on a CogVideoX-2B-shaped block.
+
+One step = one DMPQ transformer-block pass of the hot path at M = 17776
+tokens (13x30x45 video latents + 226 text tokens, hidden 1920):
+  * the router: Gamma = |out - in|_1 / |in|_1 over the block's input/output
+    pair [17776, 1920] and the INT8/NVFP4 decision at threshold 0.05;
+  * four linears -- QKV 1920->5760, out-proj 1920->1920, FFN-up 1920->7680,
+    FFN-down 7680->1920 -- each as tensor amax (block-128 Hadamard), fused
+    Hadamard + NVFP4 quantization, and the tcgen05 W4A4 GEMM with bf16 out.
+The synthetic block is a stable one (Gamma below the threshold), so every
+linear runs on the NVFP4 route; weights are packed offline, before timing.
+
+Metric: TFLOP/s of the whole step (2*M*N*K summed over the four linears).
+Each rank runs its own independent block (weak scaling, no collective on
+the data path); `value` is the sum over ranks / the slowest rank's time.
+
+--impl reference times the CPU oracle (numpy, the machine's host cores) on a
+bounded row/column sample of the same four linears per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_quantized_linear_block_b200 import synthetic as S  # noqa: E402
+
+METRIC = "W4A4 qlinear TFLOPS at CogVideoX-2B FFN shape (% of B200 FP4 peak); quant GB/s"
+UNIT = "TFLOP/s"
+THRESHOLD = 0.05
+M_TOKENS = S.M_COGVIDEOX
+BLOCK_SIGMA = 0.01          # stable block: Gamma ~ 0.01 < 0.05 -> NVFP4 route
+FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
+NVFP4_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # bf16 in, E2M1 out, E4M3 per 16
+# DRAM bytes per launch of the W4A4 GEMM from an ncu capture, valid only for
+# the kernel source it was taken on (sha256 of the GEMM sources).
+GEMM_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (barrier + max-over-ranks timing only)
+# ---------------------------------------------------------------------------
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def dist_done(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], [], set()
+        for line in out.strip().splitlines():
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, v in zip(self.NAMES, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def gemm_source_sha() -> str:
+    h = hashlib.sha256()
+    for name in ("gemm_w4a4.cu", "gemm_common.cuh", "ql_common.cuh"):
+        with open(os.path.join(ROOT, "bit_quantized_linear_block_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------
+def make_inputs(seed_offset: int):
+    """Host (CPU, bf16) inputs of one block: 4 linear inputs, 4 weights and
+    the router's input/output pair."""
+    lins = []
+    for lin in S.COGVIDEOX_2B:
+        x, w = S.cogvideox2b_linear(lin, m=M_TOKENS, seed=1 + seed_offset)
+        lins.append((lin, x, w))
+    rng = np.random.default_rng([1 + seed_offset, 900])
+    bin_ = lins[0][1]
+    noise = rng.standard_normal(size=tuple(bin_.shape), dtype=np.float32) * np.float32(BLOCK_SIGMA)
+    bout = S.to_bf16(bin_.float().numpy() + noise)
+    return lins, bin_, bout
+
+
+def step_flops(lins) -> float:
+    return float(sum(2.0 * M_TOKENS * lin.n * lin.k for lin, _, _ in lins))
+
+
+def run_ours(args, rank, world, local):
+    from bit_quantized_linear_block_b200 import qlinear as ql
+    dev = torch.device("cuda", local)
+    lins, bin_h, bout_h = make_inputs(seed_offset=100 * rank)
+    flops = step_flops(lins)
+    xs = [x.to(dev) for _, x, _ in lins]
+    pws = [ql.qlinear_prepare_weights(w.to(dev), ql.QL_W_NVFP4, hadamard=True) for _, _, w in lins]
+    bin_d, bout_d = bin_h.to(dev), bout_h.to(dev)
+    ys = [torch.empty((M_TOKENS, lin.n), dtype=torch.bfloat16, device=dev) for lin, _, _ in lins]
+    amax = [torch.zeros(1, dtype=torch.float32, device=dev) for _ in lins]
+    amax_ws = [torch.zeros(ql.lib.qlinear_quantize_ws_bytes(M_TOKENS, lin.k, ql.QL_ROUTE_NVFP4),
+                           dtype=torch.uint8, device=dev) for lin, _, _ in lins]
+    qbufs = [ql.qlinear_quantize_act(x, ql.QL_ROUTE_NVFP4, hadamard=True, rowmajor_scales=False)
+             for x in xs]
+    route_pinned = torch.zeros(1, dtype=torch.int32, pin_memory=True)
+    gamma0, route0 = ql.qlinear_route(bin_d, bout_d, THRESHOLD)
+    torch.cuda.synchronize()
+    host_route = int(route0.item())
+    assert host_route == ql.QL_ROUTE_NVFP4, "the benchmark block must be a stable (NVFP4) block"
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        # Gamma of this block; the decision is read one step later (Gamma_{t-1})
+        if ev is not None:
+            ev["route"][0].record(stream)
+        g, r = ql.qlinear_route(bin_d, bout_d, THRESHOLD)
+        route_pinned.copy_(r, non_blocking=True)
+        if ev is not None:
+            ev["route"][1].record(stream)
+        for i, (lin, _, _) in enumerate(lins):
+            if ev is not None:
+                ev["amax"][i][0].record(stream)
+            ql.qlinear_tensor_amax(xs[i], True, out=amax[i], ws=amax_ws[i])
+            if ev is not None:
+                ev["quant"][i][0].record(stream)
+            ql.qlinear_quantize_act(xs[i], host_route, True, amax_in=amax[i], out=qbufs[i])
+            if ev is not None:
+                ev["gemm"][i][0].record(stream)
+            ql.qlinear_gemm(host_route, qbufs[i], M_TOKENS, pws[i], Y=ys[i])
+            if ev is not None:
+                ev["gemm"][i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+
+    def pair():
+        return (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+
+    evs = [{"route": pair(), "amax": [pair() for _ in lins], "quant": [pair() for _ in lins],
+            "gemm": [pair() for _ in lins]} for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)     # let the sampler start before the timed region
+    t0, t1 = pair()
+    t0.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    dist_barrier(world)
+    assert ql.qlinear_device_status() == 0
+    ms = t0.elapsed_time(t1)
+    ms_max = dist_max(ms, world)
+
+    def tot(key, i=None):
+        s = 0.0
+        for e in evs:
+            if key == "route":
+                s += e["route"][0].elapsed_time(e["route"][1])
+            elif key == "amax":
+                s += e["amax"][i][0].elapsed_time(e["quant"][i][0])
+            elif key == "quant":
+                s += e["quant"][i][0].elapsed_time(e["gemm"][i][0])
+            else:
+                s += e["gemm"][i][0].elapsed_time(e["gemm"][i][1])
+        return s / len(evs)
+
+    per = {}
+    for i, (lin, _, _) in enumerate(lins):
+        per[lin.name] = {"amax_us": 1e3 * tot("amax", i), "quant_us": 1e3 * tot("quant", i),
+                         "gemm_us": 1e3 * tot("gemm", i),
+                         "gemm_tflops": 2.0 * M_TOKENS * lin.n * lin.k / (tot("gemm", i) * 1e-3) / 1e12}
+    route_us = 1e3 * tot("route")
+    gemm_ms = sum(tot("gemm", i) for i in range(len(lins)))
+    quant_ms = sum(tot("quant", i) for i in range(len(lins)))
+    amax_ms = sum(tot("amax", i) for i in range(len(lins)))
+    elems = sum(M_TOKENS * lin.k for lin, _, _ in lins)
+    peaks, peak_kind = measured_peaks()
+    peak_fp4 = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+    sha = gemm_source_sha()
+    traffic = GEMM_TRAFFIC.get(sha)
+    result = {
+        "metric": METRIC, "value": None, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": "cogvideox2b_block_linears", "M": M_TOKENS,
+                   "linears": {lin.name: [lin.k, lin.n] for lin, _, _ in lins},
+                   "route": "nvfp4 (block Gamma < 0.05)", "hadamard": 128,
+                   "l2": "no flush: each step reads 477 MB of activations (> 126 MB L2)",
+                   "parallelism": f"dp{world} (independent blocks per rank)"},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": peak_fp4, "unit": "TFLOP/s",
+                     "frac": gemm_tflops / peak_fp4, "traffic": traffic,
+                     "kernel": "k_gemm_w4a4 (all four linears)",
+                     "peak_note": f"{peak_kind} bf16 sustained x {FP4_PER_BF16:g} (nominal FP4/BF16)"},
+        "quant": {"kernel": "k_quant_nvfp4", "gbs": elems * NVFP4_BYTES_PER_ELEM / (quant_ms * 1e-3) / 1e9,
+                  "hbm_frac": elems * NVFP4_BYTES_PER_ELEM / (quant_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                  "bytes_per_elem": NVFP4_BYTES_PER_ELEM},
+        "amax": {"kernel": "k_amax", "gbs": elems * 2.0 / (amax_ms * 1e-3) / 1e9},
+        "route_kernel": {"kernel": "k_gamma_route", "us": route_us,
+                         "gbs": 4.0 * M_TOKENS * 1920 / (route_us * 1e-6) / 1e9},
+        "per_linear": per,
+        "gpu_launches": args.steps * (1 + 3 * len(lins)),
+        "clocks": clocks,
+        "gemm_source_sha": sha,
+    }
+    result["value"] = world * flops / (ms_max * 1e-3 / args.steps) / 1e12
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, ql, lins, pws, bin_h, bout_h, dev, flops, world)
+    return result
+
+
+def run_e2e(args, ql, lins, pws, bin_h, bout_h, dev, flops, world):
+    """Same step through the public forward call with HOST buffers: pinned
+    host -> device copies of every input, device -> host copies of every
+    output, inside the timed region."""
+    xh = [x.pin_memory() for _, x, _ in lins]
+    bih, boh = bin_h.pin_memory(), bout_h.pin_memory()
+    yh = [torch.empty((M_TOKENS, lin.n), dtype=torch.bfloat16).pin_memory() for lin, _, _ in lins]
+    xd = [torch.empty_like(x, device=dev) for x in xh]
+    bid, bod = torch.empty_like(bih, device=dev), torch.empty_like(boh, device=dev)
+    yd = [torch.empty((M_TOKENS, lin.n), dtype=torch.bfloat16, device=dev) for lin, _, _ in lins]
+    plans = [ql.ForwardPlan(M_TOKENS, pw, ql.QL_ROUTE_NVFP4, dev) for pw in pws]
+    for p in plans:
+        p.ws.zero_()
+    route_h = torch.zeros(1, dtype=torch.int32).pin_memory()
+
+    def step():
+        bid.copy_(bih, non_blocking=True)
+        bod.copy_(boh, non_blocking=True)
+        _, r = ql.qlinear_route(bid, bod, THRESHOLD)
+        route_h.copy_(r, non_blocking=True)
+        for i in range(len(lins)):
+            xd[i].copy_(xh[i], non_blocking=True)
+            ql.qlinear_forward(xd[i], pws[i], ql.QL_ROUTE_NVFP4, Y=yd[i], plan=plans[i])
+            yh[i].copy_(yd[i], non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    a.record(s)
+    for _ in range(args.e2e_steps):
+        step()
+    b.record(s)
+    torch.cuda.synchronize()
+    ms = dist_max(a.elapsed_time(b), world) / args.e2e_steps
+    h2d = sum(x.numel() * 2 for x in xh) + bih.numel() * 2 + boh.numel() * 2
+    d2h = sum(y.numel() * 2 for y in yh) + 4
+    return {"value": world * flops / (ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+class OracleSampler:
+    """The oracle's forward on a bounded sample of each linear: `rows`
+    activation rows x `cols` weight rows (output columns).  Weight packing
+    of the sampled weight rows happens once, outside the timing."""
+
+    def __init__(self, lins, rows: int, cols: int):
+        from oracle import qlinear_oracle as O
+        self.O = O
+        self.items = []
+        for lin, x, w in lins:
+            xb = S.bf16_bits(x)[:rows]
+            wq = O.prepare_weights_nvfp4(S.bf16_bits(w)[:cols])
+            self.items.append((lin, xb, wq))
+        self.flops = float(sum(2.0 * rows * min(cols, lin.n) * lin.k for lin, _, _ in lins))
+
+    def step(self):
+        for lin, xb, wq in self.items:
+            self.O.forward(xb, wq, self.O.ROUTE_NVFP4)
+
+
+def cpu_baseline(lins, budget_s: float = 12.0):
+    rows, cols = 128, 512
+    samp = OracleSampler(lins, rows, cols)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        samp.step()
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": samp.flops * n / dt / 1e12, "unit": UNIT, "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{n} x oracle forward (Hadamard + NVFP4 quantize + fp64 GEMM) of {rows} token rows "
+                      f"x {cols} output columns of each of the 4 linears (weights packed beforehand); "
+                      f"elementwise numpy on 1 core, BLAS on the listed threads"}
+
+
+def run_reference(args, rank, world):
+    lins, _, _ = make_inputs(seed_offset=0)
+    budget = 150.0 / max(1, args.steps + args.warmup)     # keep the whole run to a few minutes
+    rows, cols = 16, 64
+    samp = OracleSampler(lins, rows, cols)
+    t = time.perf_counter()
+    samp.step()
+    one = time.perf_counter() - t
+    scale = max(1, int(budget / max(one, 1e-6)))
+    rows = min(M_TOKENS, rows * int(np.sqrt(scale)) if scale > 1 else rows)
+    samp = OracleSampler(lins, rows, cols)
+    for _ in range(args.warmup):
+        samp.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        samp.step()
+    dt = time.perf_counter() - t0
+    value = samp.flops * args.steps / dt / 1e12
+    sample = (f"per step: oracle forward of {rows} token rows x {cols} output columns of each "
+              f"CogVideoX-2B block linear (QKV, out, FFN-up, FFN-down), K as in the workload")
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": "cogvideox2b_block_linears", "M": M_TOKENS,
+                       "linears": {lin.name: [lin.k, lin.n] for lin, _, _ in lins}},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_init()
+    try:
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps(run_reference(args, rank, world)), flush=True)
+            return
+        res = run_ours(args, rank, world, local)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                lins, _, _ = make_inputs(seed_offset=0)
+                res["cpu_baseline"] = cpu_baseline(lins)
+            print(json.dumps(res), flush=True)
+    finally:
+        dist_done(world)
+
+
+if __name__ == "__main__":
+    main()

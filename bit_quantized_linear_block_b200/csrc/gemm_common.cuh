@@ -1,0 +1,170 @@
+// Pieces shared by the tcgen05 GEMM kernels: arguments, tile order, bounded
+// teardown, the bf16 epilogue and host-side tensor-map creation.
+#pragma once
+
+#include <algorithm>
+#include "ql_common.cuh"
+
+namespace ql {
+
+constexpr int kEpiChunkCols = 64;                        // bf16 columns per TMA store
+constexpr int kEpiChunkBytes = 128 * kEpiChunkCols * 2;  // 16 KB staging tile
+constexpr long long kDrainLimit = 4000000000ll;          // cycles for teardown waits
+
+struct GemmArgs {
+  int32_t M, N, K;
+  int32_t tiles_m, tiles_n, num_tiles;
+  int32_t num_kst;      // K stages of the main loop
+  int32_t k_atoms;      // NVFP4: K / 64 (4-scale groups per row)
+  int32_t sfb_atoms;    // NVFP4: 128-row scale atoms of the weights
+  int32_t group_m;      // tile raster: m-blocks per group
+  const uint8_t* sfa;   // NVFP4 activation scales (MMA layout)
+  const uint8_t* sfb;   // NVFP4 weight scales (MMA layout)
+  const float* g_a;     // activation tensor scale (NVFP4 / per-tensor INT8)
+  const float* g_w;     // weight tensor scale (NVFP4)
+  const float* row_scale;  // per-token activation scales (INT8 route)
+  const float* col_scale0; // Q-ARVD s_norm
+  const float* col_scale1; // Q-ARVD s_out
+  const int32_t* kinfo;    // Q-ARVD class sizes
+  float alpha_mul;
+  long long wait_limit;
+  int* status;             // device status word
+};
+
+__device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
+  const uint32_t a = smem_u32(p);
+  return p + (((a + 1023u) & ~1023u) - a);
+}
+
+// Tile t -> (m-block, n-block).  Groups of `group_m` m-blocks sweep all
+// n-blocks together so that concurrently running CTAs share A and B tiles
+// in L2.
+__device__ __forceinline__ void tile_coords(int t, const GemmArgs& p, int& mb, int& nb) {
+  const int per_group = p.group_m * p.tiles_n;
+  const int g = t / per_group;
+  const int first_m = g * p.group_m;
+  const int gm = min(p.group_m, p.tiles_m - first_m);
+  const int r = t - g * per_group;
+  mb = first_m + r % gm;
+  nb = r / gm;
+}
+
+__device__ __forceinline__ void fail_timeout(int* status, volatile int* abort_flag) {
+  record_error(status, QL_ERR_TIMEOUT);
+  *abort_flag = 1;
+}
+
+// Accumulator-ready wait of the 128 epilogue threads with ONE decision for
+// all of them: thread 128 does the bounded wait and publishes the outcome
+// through shared memory behind a named barrier, so no epilogue thread can
+// leave the tile loop while another one waits at a later named barrier.
+// The flag slot sits right after the abort flag.
+__device__ __forceinline__ bool epilogue_wait_uniform(uint64_t* bar, uint32_t parity, long long limit,
+                                                      volatile int* abort_flag, int* status) {
+  volatile int* slot = abort_flag + 1;
+  if (threadIdx.x == 128) {
+    const bool ok = (*abort_flag == 0) && mbar_wait(bar, parity, limit);
+    if (!ok) fail_timeout(status, abort_flag);
+    *slot = ok ? 1 : 0;
+  }
+  named_bar_sync(1, 128);
+  return *slot != 0;
+}
+
+// Wait for the last (up to) `stages` loads this producer issued, so that no
+// copy is still writing shared memory when the CTA retires.
+__device__ __forceinline__ void drain_loads(uint64_t* full, int issued, int stages, int* status) {
+  for (int j = max(0, issued - stages); j < issued; ++j) {
+    if (!mbar_wait(&full[j % stages], (j / stages) & 1, kDrainLimit))
+      record_error(status, QL_ERR_TIMEOUT);
+  }
+}
+
+// Wait until every tcgen05 operation issued by this thread has completed.
+__device__ __forceinline__ void drain_mma(uint64_t* bar, int* status) {
+  tc_commit(bar);
+  if (!mbar_wait(bar, 0, kDrainLimit)) record_error(status, QL_ERR_TIMEOUT);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+struct EpilogueState {
+  uint32_t buf;
+};
+
+// Store one 64-column chunk (this thread's row `row`, values v[0..63]) via
+// the swizzled staging buffer and a TMA store.  Called by all 128 epilogue
+// threads (warps 4-7); thread 128 issues the bulk operations.
+__device__ __forceinline__ void epilogue_store_chunk(const uint32_t (&packed)[32], uint8_t* sC,
+                                                     const CUtensorMap* tm_y, int c0, int r0,
+                                                     EpilogueState& es) {
+  const int row = threadIdx.x & 127;
+  const bool leader = threadIdx.x == 128;
+  if (leader) bulk_wait_read<1>();
+  named_bar_sync(1, 128);
+  uint8_t* dst = sC + es.buf * kEpiChunkBytes + row * 128;
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *reinterpret_cast<uint4*>(dst + ((q ^ (row & 7)) << 4)) =
+        make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+  fence_proxy_async_smem();
+  named_bar_sync(1, 128);
+  if (leader) {
+    tma_store_2d(tm_y, sC + es.buf * kEpiChunkBytes, c0, r0);
+    bulk_commit();
+  }
+  es.buf ^= 1;
+}
+
+// bf16 epilogue of one BM x BN fp32 accumulator: y = alpha * acc.  Frees
+// the accumulator (arrive on `tempty`) as soon as the last columns are in
+// registers.
+template <int BN>
+__device__ __forceinline__ void epilogue_tile(uint32_t acc_tmem, uint64_t* tempty, uint8_t* sC,
+                                              const CUtensorMap* tm_y, int m0, int n0, int N,
+                                              float alpha, EpilogueState& es) {
+  const int ew = (threadIdx.x >> 5) & 3;
+  const int lane = threadIdx.x & 31;
+  constexpr int CH = BN / kEpiChunkCols;
+#pragma unroll 1
+  for (int c = 0; c < CH; ++c) {
+    uint32_t r0[32], r1[32];
+    const uint32_t taddr = acc_tmem + (static_cast<uint32_t>(ew * 32) << 16) + c * kEpiChunkCols;
+    tmem_ld32(taddr, r0);
+    tmem_ld32(taddr + 32, r1);
+    tmem_ld_wait();
+    if (c == CH - 1) {
+      tc_fence_before();
+      if (lane == 0) mbar_arrive(tempty);
+    }
+    if (n0 + c * kEpiChunkCols >= N) continue;   // same for all 128 threads
+    uint32_t packed[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      packed[j] = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r0[2 * j])),
+                              __fmul_rn(alpha, __uint_as_float(r0[2 * j + 1])));
+      packed[16 + j] = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r1[2 * j])),
+                                   __fmul_rn(alpha, __uint_as_float(r1[2 * j + 1])));
+    }
+    epilogue_store_chunk(packed, sC, tm_y, n0 + c * kEpiChunkCols, m0, es);
+  }
+}
+
+__device__ __forceinline__ void epilogue_finish(EpilogueState&) {
+  if (threadIdx.x == 128) bulk_wait_all();
+}
+
+// ---------------------------------------------------------------------------
+// Host helpers (defined in capi.cu)
+// ---------------------------------------------------------------------------
+bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t inner,
+                  int64_t outer, int64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
+                  CUtensorMapSwizzle swizzle);
+int num_sms();
+bool set_smem_attr(const void* kernel, int bytes);
+void fill_gemm_args(GemmArgs& p, int64_t M, int N, int K, int BN, int* status);
+
+}  // namespace ql

@@ -1,0 +1,47 @@
+// Host-side launch functions of the kernels, one translation unit each,
+// called by the C-ABI layer (capi.cu).
+#pragma once
+
+#include <algorithm>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/qlinear.h"
+
+namespace ql {
+
+constexpr int kHbmCtasPerSm = 4;                 // 256-thread CTAs per SM for streaming kernels
+constexpr int kMaxPartials = 4096;               // upper bound of any streaming grid
+constexpr size_t kAmaxPartialBytes = kMaxPartials * sizeof(float);
+constexpr size_t kAmaxWsBytes = kAmaxPartialBytes + 256;   // partials + ticket
+constexpr size_t kRoutePartialBytes = 2 * kMaxPartials * sizeof(double);
+
+int num_sms();
+bool set_smem_attr(const void* kernel, int bytes);
+int hbm_grid(int64_t work_items, int per_cta);
+int qarvd_slices(int32_t N);
+
+// Tensor amax (rotated when hadamard != 0) into *amax_out; ws needs
+// kAmaxWsBytes (partials + ticket).
+ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* amax_out, void* ws,
+                      cudaStream_t st);
+ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, const float* amax_in,
+                             void* codes, void* sf_mma, void* sf_rm, float* g_out, cudaStream_t st);
+ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadamard, void* codes,
+                                  float* scales, cudaStream_t st);
+ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int32_t Kp,
+                                        const int32_t* gather, const float* amax_in, void* codes,
+                                        float* scale_out, cudaStream_t st);
+ql_status launch_gamma_route(const void* in, const void* out, int64_t numel, float threshold,
+                             double* gamma, int32_t* route, void* ws, cudaStream_t st);
+ql_status launch_qarvd_prepare(const void* W, int32_t N, int32_t K, float tau, float alpha,
+                               const ql_weights* w, void* ws, cudaStream_t st);
+
+ql_status launch_gemm_w4a4(const void* a_codes, const uint8_t* a_sf, const float* g_a, int64_t M,
+                           const ql_weights* w, void* Y, cudaStream_t st, int* status);
+ql_status launch_gemm_w4a8(const void* a_codes, const float* a_scales, int64_t M,
+                           const ql_weights* w, void* Y, cudaStream_t st, int* status);
+ql_status launch_gemm_qarvd(const void* a_codes, const float* s_x, int64_t M, const ql_weights* w,
+                            void* Y, cudaStream_t st, int* status);
+
+}  // namespace ql

@@ -1,0 +1,219 @@
+/*
+ * qlinear.h -- C ABI of the B200 (sm_100a) quantized linear layer.
+ *
+ * The layer follows two web pages on video-diffusion-transformer
+ * quantization:
+ *   "6Bit-Diffusion" (gist.science 2603.18742), Methodology B.1 (DMPQ):
+ *     an online block Hadamard transform on the activations, activations
+ *     routed per transformer block to INT8 (sensitive blocks) or NVFP4
+ *     (stable blocks) by the block's input/output relative L1 distance
+ *     Gamma, and all weights quantized offline to NVFP4;
+ *   "Q-ARVD: Autoregressive Video Diffusion Models의 양자화", Methodology
+ *     and Formula/operation flow: outlier input channels found from the
+ *     channel L2 norms by a median/MAD modified z-score with threshold tau
+ *     and minimum magnitude alpha, separate per-output-channel scales for
+ *     the outlier and normal channel classes, per-tensor INT8 activations.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device,
+ *     allocated and owned by the caller.  The library never allocates device
+ *     memory; scratch space is a caller-provided workspace whose size the
+ *     matching *_ws_bytes() query returns.  Pointers must be 16-byte aligned
+ *     (256-byte for workspaces and weight buffers).
+ *   - A workspace must be zero-filled before its first use.  Kernels that
+ *     count finished CTAs in it put the counter back to zero, so a workspace
+ *     stays usable for later calls on the same stream; two calls in flight
+ *     at once need two workspaces.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *     Calls enqueue work and return; they never synchronize, except where a
+ *     comment says so.
+ *   - Calls return a ql_status and never throw or abort.  Shape and pointer
+ *     checks run on the host before anything is enqueued; a failed check
+ *     enqueues nothing.
+ *   - Matrices are row-major.  X is [M, K] (tokens x in-features), W is
+ *     [N, K] (nn.Linear layout), Y = X W^T is [M, N], all bf16.
+ *   - K must be a multiple of 128 (the Hadamard block) and N a multiple of
+ *     16.  M may be any value >= 0.
+ *   - Non-finite inputs give unspecified (but memory-safe) results.
+ *
+ * Data layouts:
+ *   NVFP4 codes   uint8 [rows, K/2]; byte j holds element 2j in its low
+ *                 nibble and 2j+1 in its high nibble; E2M1 code = sign bit 3,
+ *                 magnitude bits 0-2 indexing {0,.5,1,1.5,2,3,4,6}.
+ *   NVFP4 scales  one E4M3 byte per 16 elements along K.  "MMA layout":
+ *                 rows padded to a multiple of 128 (padding scales are 0);
+ *                 512-byte atoms, atom (r/128, j/4) at byte offset
+ *                 ((r/128) * (K/64) + j/4) * 512; inside an atom, scale j of
+ *                 row r sits at (r%32)*16 + ((r/32)%4)*4 + j%4.
+ *                 "Row-major": uint8 [rows, K/16].
+ *   Tensor scale  fp32 g = amax(rotated tensor) / 2688 (1 if amax is 0);
+ *                 dequantized value = e2m1 * e4m3 * g.
+ *   INT8 token    int8 [M, K] and fp32 [M] scales s_m = amax_m / 127.
+ */
+#ifndef QLINEAR_H
+#define QLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define QLINEAR_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define QL_API __attribute__((visibility("default")))
+#else
+#define QL_API
+#endif
+
+typedef enum {
+  QL_OK = 0,
+  QL_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, negative size      */
+  QL_ERR_UNSUPPORTED_SHAPE = 2, /* K % 128, N % 16, or a size beyond limits   */
+  QL_ERR_ALIGNMENT = 3,         /* pointer not aligned as required            */
+  QL_ERR_CUDA = 4,              /* a CUDA runtime call failed                 */
+  QL_ERR_TIMEOUT = 5,           /* a device-side wait hit its limit           */
+  QL_ERR_WORKSPACE = 6,         /* workspace or buffer smaller than required  */
+  QL_ERR_NO_DEVICE = 7          /* no usable sm_100 device                    */
+} ql_status;
+
+/* Weight formats. */
+typedef enum {
+  QL_W_NVFP4 = 0,       /* NVFP4 (E2M1 + E4M3/16 + fp32), optional Hadamard  */
+  QL_W_QARVD_INT4 = 2   /* Q-ARVD dual-scale signed INT4, K permuted         */
+} ql_weight_format;
+
+/* Activation routes / formats. */
+typedef enum {
+  QL_ROUTE_NVFP4 = 0,       /* W4A4: NVFP4 activations                       */
+  QL_ROUTE_INT8 = 1,        /* W4A8: per-token INT8 activations              */
+  QL_ACT_INT8_TENSOR = 2    /* Q-ARVD: per-tensor INT8, permuted K           */
+} ql_act_format;
+
+typedef struct {
+  int32_t fmt;       /* ql_weight_format                                       */
+  int32_t hadamard;  /* NVFP4: 1 = rotate K by blockdiag(H_128) (must match the
+                        activations' setting); Q-ARVD: must be 0              */
+  float tau;         /* Q-ARVD modified z-score threshold (3.5)                */
+  float alpha;       /* Q-ARVD minimum magnitude factor (2.0)                  */
+} ql_weight_cfg;
+
+/* Packed weights.  Filled by qlinear_prepare_weights(); every pointer points
+   into the caller's weight buffer.  Treat as read-only. */
+typedef struct {
+  int32_t fmt, N, K, hadamard;
+  int32_t Kp;            /* Q-ARVD: padded permuted K of codes/activations     */
+  int32_t reserved0;
+  void* codes;           /* NVFP4 [N, K/2]; Q-ARVD INT4 nibbles [N, Kp/2]       */
+  void* sf;              /* NVFP4 block scales, MMA layout                      */
+  float* gscale;         /* NVFP4 fp32 tensor scale g_w (1 value)               */
+  uint8_t* outlier_mask; /* Q-ARVD [K], 1 = outlier channel                     */
+  int32_t* perm;         /* Q-ARVD [K] channels in class order                  */
+  int32_t* gather;       /* Q-ARVD [Kp] source channel of each slot, -1 = pad   */
+  int32_t* kinfo;        /* Q-ARVD [4] k_norm, k_norm_pad, n_out, k_out_pad     */
+  float* s_norm;         /* Q-ARVD [N] scale of the normal channels             */
+  float* s_out;          /* Q-ARVD [N] scale of the outlier channels            */
+  double* norms;         /* Q-ARVD [K] input-channel L2 norms                   */
+} ql_weights;
+
+/* ---- library ------------------------------------------------------------ */
+
+QL_API int qlinear_abi_version(void);
+QL_API const char* qlinear_status_string(int status);
+
+/* Reads and clears the device status word of the current device, which the
+   kernels set when a bounded wait times out (QL_ERR_TIMEOUT) .  Synchronizes
+   `stream` first.  *status_out receives QL_OK or the first error recorded. */
+QL_API ql_status qlinear_device_status(void* stream, int32_t* status_out);
+
+/* Test hook: the cycle budget of every pipeline wait in the GEMM kernels
+   (default about one second).  0 makes the first wait that is not already
+   satisfied time out, so a test can exercise the timeout path; the kernel
+   then drains its in-flight copies with a separate, generous budget and
+   returns.  Negative restores the default.  Host-global, not thread-safe. */
+QL_API void qlinear_debug_set_wait_limit(long long cycles);
+
+/* ---- sizes ---------------------------------------------------------------- */
+
+/* Bytes of NVFP4 block scales in the MMA layout for a [rows, K] tensor. */
+QL_API size_t qlinear_sf_bytes(int64_t rows, int32_t K);
+
+/* ---- weights: offline preparation ----------------------------------------
+   NVFP4 (6Bit-Diffusion, Methodology B.1): W -> (Hadamard) -> NVFP4 with a
+   tensor scale from amax of the rotated W.
+   Q-ARVD (Q-ARVD, Methodology / Formula and operation flow): channel norms,
+   median/MAD z-score mask, class-ordered permutation, per-row dual INT4
+   scales, INT4 codes.  The weight buffer (qlinear_weights_bytes) holds every
+   output; `ws` is scratch (qlinear_prepare_ws_bytes).  Asynchronous. */
+QL_API size_t qlinear_weights_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg);
+QL_API size_t qlinear_prepare_ws_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg);
+QL_API ql_status qlinear_prepare_weights(const void* W_bf16, int32_t N, int32_t K,
+                                  const ql_weight_cfg* cfg,
+                                  void* wbuf, size_t wbuf_bytes, ql_weights* out,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* ---- DMPQ router (6Bit-Diffusion, Methodology A.1 and B.1) ----------------
+   Gamma = sum|out - in| / sum|in| over `numel` bf16 elements (fp32
+   differences, fp64 sums); *route_dev = 1 (INT8) if Gamma > threshold else
+   0 (NVFP4); Gamma = +inf (route INT8) when sum|in| is 0.  gamma_dev and
+   route_dev are device pointers. */
+QL_API size_t qlinear_route_ws_bytes(int64_t numel);
+QL_API ql_status qlinear_route(const void* in_bf16, const void* out_bf16, int64_t numel,
+                        float threshold, double* gamma_dev, int32_t* route_dev,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* ---- tensor amax ------------------------------------------------------------
+   *amax_out (device fp32) = max |H x| over the whole [M, K] tensor (|x| when
+   hadamard is 0): the input of the dynamic NVFP4 tensor scale
+   g = amax / (6 * 448) and of the per-tensor INT8 scale amax / 127.  One
+   launch; ws needs qlinear_quantize_ws_bytes(M, K, QL_ROUTE_NVFP4) bytes. */
+QL_API ql_status qlinear_tensor_amax(const void* X_bf16, int64_t M, int32_t K, int32_t hadamard,
+                                     float* amax_out, void* ws, size_t ws_bytes, void* stream);
+
+/* ---- activation quantization (inspection entry point) ---------------------
+   QL_ROUTE_NVFP4:     codes uint8 [M, K/2]; sf_mma (MMA layout, required);
+                       sf_rowmajor [M, K/16] (optional, may be NULL);
+                       scales = fp32[1] tensor scale g_x.
+   QL_ROUTE_INT8:      codes int8 [M, K]; scales = fp32 [M]; sf_* unused.
+   QL_ACT_INT8_TENSOR: needs Q-ARVD weights `w`; codes int8 [M, w->Kp] in the
+                       weights' channel order with zero padding; scales =
+                       fp32[1]; hadamard must be 0.
+   `hadamard` = 1 rotates each 128-block of K first (NVFP4 / INT8 routes).
+   amax_in: optional device fp32 tensor amax (NVFP4 and per-tensor INT8),
+   e.g. from qlinear_tensor_amax or a calibrated static value; NULL makes the
+   call compute the dynamic amax itself (one extra launch). */
+QL_API size_t qlinear_quantize_ws_bytes(int64_t M, int32_t K, int32_t act_fmt);
+QL_API ql_status qlinear_quantize_act(const void* X_bf16, int64_t M, int32_t K,
+                                      int32_t act_fmt, int32_t hadamard, const ql_weights* w,
+                                      const float* amax_in, void* codes, void* sf_mma,
+                                      void* sf_rowmajor, float* scales,
+                                      void* ws, size_t ws_bytes, void* stream);
+
+/* ---- GEMM on quantized activations ----------------------------------------
+   Y[m, n] = bf16(alpha_m * sum_k a[m,k] w[n,k]) with fp32 accumulation:
+   QL_ROUTE_NVFP4:     tcgen05 block-scaled FP4 MMA; alpha = g_x g_w / 128 if
+                       the weights are rotated, else g_x g_w.
+   QL_ROUTE_INT8:      INT8 x NVFP4 weights expanded on chip to bf16;
+                       alpha_m = s_m g_w (/128 if rotated).
+   QL_ACT_INT8_TENSOR: INT8 x INT4 integer MMA, two class accumulators;
+                       y = s_x (s_norm[n] acc_normal + s_out[n] acc_outlier).
+   Operands are the outputs of qlinear_quantize_act for the same format. */
+QL_API ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf,
+                       const float* a_scales, int64_t M, const ql_weights* w,
+                       void* Y_bf16, void* stream);
+
+/* ---- forward: quantize + GEMM ----------------------------------------------
+   route: QL_ROUTE_NVFP4 or QL_ROUTE_INT8 for NVFP4 weights (the activation
+   rotation follows w->hadamard); ignored for Q-ARVD weights (per-tensor
+   INT8).  Scratch for the quantized activations lives in `ws`. */
+QL_API size_t qlinear_forward_ws_bytes(int64_t M, const ql_weights* w, int32_t route);
+QL_API ql_status qlinear_forward(const void* X_bf16, int64_t M, const ql_weights* w,
+                          int32_t route, void* Y_bf16,
+                          void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLINEAR_H */

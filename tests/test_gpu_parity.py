@@ -1,0 +1,205 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on
+identical seeded bf16 inputs.  Quantized codes, scales, masks and routes
+must match bit for bit; GEMM outputs within the stated tolerances."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import qlinear_oracle as O
+from bit_quantized_linear_block_b200 import synthetic as S
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ql():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from bit_quantized_linear_block_b200 import qlinear
+    return qlinear
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _x(m, k, seed, outliers=8, scale=50.0):
+    return S.activations_fixed_outliers(m, k, outliers, scale, seed, 1)
+
+
+def normwise_err(y, r):
+    return float(np.abs(y - r).max() / max(np.abs(r).max(), 1e-30))
+
+
+def excess_err(y, r):
+    """Error beyond the bf16 rounding of the output (2^-9 relative)."""
+    ex = np.maximum(0.0, np.abs(y - r) - 2.0 ** -9 * np.maximum(np.abs(y), np.abs(r)))
+    return float(ex.max() / max(np.abs(r).max(), 1e-30))
+
+
+# ---------------------------------------------------------------- quantizers
+
+SHAPES = [(1, 128), (77, 384), (256, 1920), (300, 640), (129, 1024)]
+
+
+@pytest.mark.parametrize("m,k", SHAPES)
+@pytest.mark.parametrize("hadamard", [True, False])
+def test_nvfp4_quantize_bit_exact(ql, m, k, hadamard):
+    x = _x(m, k, seed=m + k)
+    xb = S.bf16_bits(x)
+    h = O.block_hadamard(O.bf16_bits_to_f32(xb)) if hadamard else O.bf16_bits_to_f32(xb)
+    packed, sb, g = O.nvfp4_quantize(h)
+    q = ql.qlinear_quantize_act(x.cuda(), ql.QL_ROUTE_NVFP4, hadamard=hadamard)
+    torch.cuda.synchronize()
+    assert _np(q["scales"])[0] == g
+    assert np.array_equal(_np(q["sf_rowmajor"]), sb)
+    assert np.array_equal(_np(ql.sf_mma_to_rowmajor(q["sf_mma"], m, k)), sb)
+    mpad = (m + 127) // 128 * 128
+    assert not _np(ql.sf_mma_to_rowmajor(q["sf_mma"], mpad, k))[m:].any()   # padding rows
+    assert np.array_equal(_np(q["codes"]), packed)
+
+
+def test_nvfp4_quantize_zero_and_tiny_blocks(ql):
+    x = np.zeros((130, 256), np.float32)
+    x[0, 0] = 3000.0
+    x[5, 16:32] = 1e-3          # subnormal E4M3 block scale
+    x[7, 32:48] = -1e-6         # scale rounds to 0 -> all +0 codes
+    x[9, 64:80] = -0.0
+    xt = S.to_bf16(x)
+    packed, sb, g = O.nvfp4_quantize(O.bf16_bits_to_f32(S.bf16_bits(xt)))
+    q = ql.qlinear_quantize_act(xt.cuda(), ql.QL_ROUTE_NVFP4, hadamard=False)
+    torch.cuda.synchronize()
+    assert _np(q["scales"])[0] == g
+    assert np.array_equal(_np(q["sf_rowmajor"]), sb)
+    assert np.array_equal(_np(q["codes"]), packed)
+
+
+@pytest.mark.parametrize("m,k", SHAPES)
+@pytest.mark.parametrize("hadamard", [True, False])
+def test_int8_token_quantize_bit_exact(ql, m, k, hadamard):
+    x = _x(m, k, seed=3 * m + k)
+    xb = S.bf16_bits(x)
+    h = O.block_hadamard(O.bf16_bits_to_f32(xb)) if hadamard else O.bf16_bits_to_f32(xb)
+    qo, so = O.int8_per_token(h)
+    q = ql.qlinear_quantize_act(x.cuda(), ql.QL_ROUTE_INT8, hadamard=hadamard)
+    torch.cuda.synchronize()
+    assert np.array_equal(_np(q["scales"])[:m], so)
+    assert np.array_equal(_np(q["codes"]), qo)
+
+
+def test_int8_token_zero_row(ql):
+    x = np.zeros((3, 128), np.float32)
+    x[1] = np.arange(128) - 64
+    xt = S.to_bf16(x)
+    qo, so = O.int8_per_token(O.block_hadamard(O.bf16_bits_to_f32(S.bf16_bits(xt))))
+    q = ql.qlinear_quantize_act(xt.cuda(), ql.QL_ROUTE_INT8, hadamard=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(_np(q["scales"]), so) and np.array_equal(_np(q["codes"]), qo)
+
+
+# ---------------------------------------------------------------- router
+
+@pytest.mark.parametrize("numel", [0, 5, 1920, 256 * 1920 + 3])
+def test_route_gamma(ql, numel):
+    rng = np.random.default_rng(numel)
+    x = rng.standard_normal(numel).astype(np.float32)
+    y = x + rng.standard_normal(numel).astype(np.float32) * 0.04
+    xt, yt = S.to_bf16(x), S.to_bf16(y)
+    g_ref = O.dmpq_gamma(S.bf16_bits(xt), S.bf16_bits(yt))
+    g, r = ql.qlinear_route(xt.cuda(), yt.cuda(), 0.05)
+    torch.cuda.synchronize()
+    g, r = float(_np(g)[0]), int(_np(r)[0])
+    if numel == 0:
+        assert g == float("inf") and r == 1
+    else:
+        assert g == pytest.approx(g_ref, rel=1e-12)
+        assert r == O.dmpq_route(g_ref, 0.05)
+
+
+def test_route_closed_forms(ql):
+    rng = np.random.default_rng(9)
+    x = rng.integers(-15, 16, size=4096).astype(np.float32) / 16
+    xt = S.to_bf16(x)
+    for y, want in [(x, 0.0), (x * np.float32(1.125), 0.125), (-x, 2.0)]:
+        g, r = ql.qlinear_route(xt.cuda(), S.to_bf16(y).cuda(), 0.125)
+        torch.cuda.synchronize()
+        assert float(_np(g)[0]) == want
+        assert int(_np(r)[0]) == (1 if want > 0.125 else 0)
+
+
+def test_route_sweep_blocks_match_oracle(ql):
+    """The routing sweep's blocks at a reduced token count: identical routes."""
+    for b in range(30):
+        x, y, sigma = S.dmpq_block_pair(b, m=512)
+        g_ref = O.dmpq_gamma(S.bf16_bits(x), S.bf16_bits(y))
+        assert abs(g_ref - 0.05) / 0.05 > 1e-9
+        g, r = ql.qlinear_route(x.cuda(), y.cuda(), 0.05)
+        torch.cuda.synchronize()
+        assert float(_np(g)[0]) == pytest.approx(g_ref, rel=1e-12)
+        assert int(_np(r)[0]) == O.dmpq_route(g_ref, 0.05)
+
+
+# ---------------------------------------------------------------- weights
+
+@pytest.mark.parametrize("n,k", [(1920, 1920), (640, 384), (16, 128)])
+def test_prepare_weights_nvfp4_bit_exact(ql, n, k):
+    w = S.weights(n, k, 0.02, 5, n + k)
+    ref = O.prepare_weights_nvfp4(S.bf16_bits(w), hadamard=True)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True)
+    torch.cuda.synchronize()
+    codes = _np(pw.view("codes", torch.uint8, n * k // 2)).reshape(n, k // 2)
+    sf = pw.view("sf", torch.uint8, ql.lib.qlinear_sf_bytes(n, k))
+    assert _np(pw.view("gscale", torch.float32, 1))[0] == ref["g"]
+    assert np.array_equal(_np(ql.sf_mma_to_rowmajor(sf, n, k)), ref["sb"])
+    assert np.array_equal(codes, ref["packed"])
+
+
+# ---------------------------------------------------------------- W4A4 GEMM
+
+W4A4_CASES = [
+    (256, 1920, 1920),   # the single-linear workload
+    (300, 384, 640),     # ragged M, two 192-wide tiles, half-full last K stage
+    (129, 640, 384),     # N not a multiple of 192 -> 128-wide tiles
+    (1, 192, 128),
+    (1000, 5760, 1920),  # many tiles per CTA (persistent loop, both accumulators)
+]
+
+
+@pytest.mark.parametrize("m,n,k", W4A4_CASES)
+def test_forward_w4a4_parity(ql, m, n, k):
+    x = _x(m, k, seed=m * 7 + n)
+    w = S.weights(n, k, 0.02, 6, m + n + k)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    wq = O.prepare_weights_nvfp4(wb)
+    rows = np.arange(m) if m <= 512 else np.unique(np.r_[np.random.default_rng(0).choice(m, 256, replace=False), m - 1])
+    ref = O.forward(xb, wq, O.ROUTE_NVFP4, rows=rows)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True)
+    y = ql.qlinear_forward(x.cuda(), pw, ql.QL_ROUTE_NVFP4)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    yn = _np(y.float())[rows].astype(np.float64)
+    assert np.isfinite(yn).all()
+    assert normwise_err(yn, ref) <= 1e-2
+
+
+def test_gemm_timeout_path_reports_and_recovers(ql):
+    """A zero wait budget makes the GEMM's first unsatisfied wait time out:
+    the kernel records QL_ERR_TIMEOUT, drains and returns; the context stays
+    usable and the next call with the default budget is correct."""
+    m, n, k = 256, 384, 1920
+    x = _x(m, k, seed=11)
+    w = S.weights(n, k, 0.02, 6, 11)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True)
+    xc = x.cuda()
+    assert ql.qlinear_device_status() == 0
+    ql.qlinear_debug_set_wait_limit(0)
+    try:
+        ql.qlinear_forward(xc, pw, ql.QL_ROUTE_NVFP4)
+        st = ql.qlinear_device_status()
+    finally:
+        ql.qlinear_debug_set_wait_limit(-1)
+    assert st == 5
+    y = ql.qlinear_forward(xc, pw, ql.QL_ROUTE_NVFP4)
+    assert ql.qlinear_device_status() == 0
+    ref = O.forward(S.bf16_bits(x), O.prepare_weights_nvfp4(S.bf16_bits(w)), O.ROUTE_NVFP4)
+    assert normwise_err(_np(y.float()).astype(np.float64), ref) <= 1e-2
