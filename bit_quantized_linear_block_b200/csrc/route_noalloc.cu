@@ -1,0 +1,149 @@
+// Allocation-free DMPQ router.
+//
+// Same Gamma / route computation as qlinear_route, but its scratch (per-CTA
+// fp64 partial sums and a finished-CTA counter) lives in a file-scope device
+// array instead of a caller-provided workspace, so a caller that cannot
+// allocate device memory can still run the router.  The array is sized for
+// kNoAllocMaxCtas CTAs; every device that loads the library keeps it until
+// the process exits.
+#include <mutex>
+
+#include "ql_common.cuh"
+#include "launchers.h"
+
+namespace {
+
+constexpr int kNoAllocMaxCtas = 1024;
+constexpr size_t kTicketOffset = kNoAllocMaxCtas * 2 * sizeof(double);   // after the partials
+constexpr size_t kNoAllocScratchBytes = kTicketOffset + 256;              // 16640 bytes
+constexpr int kMaxDev = 64;
+
+// In host code this name is only a stand-in for the device array; the host
+// passes the address that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
+
+std::mutex g_setup_mu;
+void* g_scratch_addr[kMaxDev] = {nullptr};
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Gamma = sum|out - in| / sum|in| (fp32 differences, fp64 sums) with the
+// scratch at `scratch`: partials [2 * gridDim.x] doubles, then the counter.
+__global__ void __launch_bounds__(ql::kThreadsHbm)
+    k_gamma_route_static(const uint4* __restrict__ in, const uint4* __restrict__ out, int64_t numel,
+                         unsigned char* __restrict__ scratch, float threshold,
+                         double* __restrict__ gamma_out, int32_t* __restrict__ route_out) {
+  double* partials = reinterpret_cast<double*>(scratch);
+  unsigned int* ticket = reinterpret_cast<unsigned int*>(scratch + kTicketOffset);
+  double s1 = 0.0, s0 = 0.0;
+  const int64_t nvec = numel >> 3;
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthr = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = tid; i < nvec; i += nthr) {
+    const uint4 a = __ldcs(in + i);
+    const uint4 b = __ldcs(out + i);
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float x0 = ql::bf16_lo(wa[k]), x1 = ql::bf16_hi(wa[k]);
+      const float y0 = ql::bf16_lo(wb[k]), y1 = ql::bf16_hi(wb[k]);
+      s1 += static_cast<double>(fabsf(__fsub_rn(y0, x0)));
+      s1 += static_cast<double>(fabsf(__fsub_rn(y1, x1)));
+      s0 += static_cast<double>(fabsf(x0));
+      s0 += static_cast<double>(fabsf(x1));
+    }
+  }
+  if (tid < (numel & 7)) {
+    const unsigned short* ia = reinterpret_cast<const unsigned short*>(in) + (nvec << 3) + tid;
+    const unsigned short* ib = reinterpret_cast<const unsigned short*>(out) + (nvec << 3) + tid;
+    const float x = __uint_as_float(static_cast<uint32_t>(*ia) << 16);
+    const float y = __uint_as_float(static_cast<uint32_t>(*ib) << 16);
+    s1 += static_cast<double>(fabsf(__fsub_rn(y, x)));
+    s0 += static_cast<double>(fabsf(x));
+  }
+  s1 = warp_sum(s1);
+  s0 = warp_sum(s0);
+  __shared__ double red[2][ql::kThreadsHbm / 32];
+  __shared__ bool s_last;
+  if ((threadIdx.x & 31) == 0) {
+    red[0][threadIdx.x >> 5] = s1;
+    red[1][threadIdx.x >> 5] = s0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double a = 0.0, b = 0.0;
+    for (int i = 0; i < ql::kThreadsHbm / 32; ++i) {
+      a += red[0][i];
+      b += red[1][i];
+    }
+    partials[2 * blockIdx.x] = a;
+    partials[2 * blockIdx.x + 1] = b;
+    __threadfence();
+    s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (s_last && threadIdx.x == 0) {
+    __threadfence();
+    double a = 0.0, b = 0.0;
+    const volatile double* p = partials;
+    for (unsigned int i = 0; i < gridDim.x; ++i) {
+      a += p[2 * i];
+      b += p[2 * i + 1];
+    }
+    const double gamma = (b == 0.0) ? __longlong_as_double(0x7ff0000000000000ll) : a / b;
+    *gamma_out = gamma;
+    *route_out = (gamma > static_cast<double>(threshold)) ? 1 : 0;
+    *ticket = 0u;
+  }
+}
+
+bool is_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+extern "C" ql_status qlinear_route_noalloc(const void* in, const void* out, int64_t numel,
+                                           float threshold, double* gamma_dev, int32_t* route_dev,
+                                           void* stream) {
+  if (numel < 0 || gamma_dev == nullptr || route_dev == nullptr) return QL_ERR_INVALID_ARG;
+  if (numel > 0 && (in == nullptr || out == nullptr)) return QL_ERR_INVALID_ARG;
+  if (!(threshold == threshold)) return QL_ERR_INVALID_ARG;
+  if (!is_aligned(in, 16) || !is_aligned(out, 16) || !is_aligned(gamma_dev, 8) ||
+      !is_aligned(route_dev, 4))
+    return QL_ERR_ALIGNMENT;
+  int dev = -1, major = 0, minor = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return QL_ERR_NO_DEVICE;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return QL_ERR_NO_DEVICE;
+  if (major != 10 || minor != 0) return QL_ERR_NO_DEVICE;
+  // Set-up, once per device with that device current: the device address of
+  // the scratch array.
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_setup_mu);
+    if (g_scratch_addr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || p == nullptr) return QL_ERR_CUDA;
+      g_scratch_addr[dev] = p;
+    }
+    scratch = g_scratch_addr[dev];
+  }
+  const int64_t want = (numel / 8 + ql::kThreadsHbm - 1) / ql::kThreadsHbm;
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(sms) * ql::kHbmCtasPerSm));
+  if (grid > kNoAllocMaxCtas) return QL_ERR_UNSUPPORTED_SHAPE;   // would overrun the scratch array
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The array keeps the previous call's contents: the counter must start at 0.
+  if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + kTicketOffset, 0, sizeof(unsigned int), st) !=
+      cudaSuccess)
+    return QL_ERR_CUDA;
+  k_gamma_route_static<<<static_cast<unsigned int>(grid), ql::kThreadsHbm, 0, st>>>(
+      static_cast<const uint4*>(in), static_cast<const uint4*>(out), numel,
+      static_cast<unsigned char*>(scratch), threshold, gamma_dev, route_dev);
+  return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}

@@ -164,6 +164,27 @@ QL_API ql_status qlinear_route(const void* in_bf16, const void* out_bf16, int64_
                         float threshold, double* gamma_dev, int32_t* route_dev,
                         void* ws, size_t ws_bytes, void* stream);
 
+/* ---- router without a workspace (no counterpart on the pages) --------------
+   Same Gamma and route as qlinear_route, for callers that cannot allocate
+   device memory or hand over a workspace: code that runs where another
+   component owns every device allocation (an inference engine or plugin host
+   with its own memory pool and budget), or a latency-critical loop that must
+   not call cudaMalloc, which can block and synchronize the device.  The
+   caller still passes the inputs and the two outputs.
+   Scratch: a file-scope device array of 16640 bytes (fp64 partial sums of
+   up to 1024 CTAs plus a finished-CTA counter); every GPU that loads this
+   library holds it until the process exits.  The first call on a device
+   looks up the array's device address with cudaGetSymbolAddress and caches
+   it, so make that first call before any stream capture.  All calls share
+   the one array and it keeps the last call's contents; each call zeroes the
+   counter before its kernel runs.  Calls that overlap on the GPU (two
+   streams, two host threads) race on the array: serialize them.  A call
+   that would need more than 1024 CTAs of scratch returns
+   QL_ERR_UNSUPPORTED_SHAPE (on a 148-SM B200 the grid is at most 592). */
+QL_API ql_status qlinear_route_noalloc(const void* in_bf16, const void* out_bf16, int64_t numel,
+                                       float threshold, double* gamma_dev, int32_t* route_dev,
+                                       void* stream);
+
 /* ---- tensor amax ------------------------------------------------------------
    *amax_out (device fp32) = max |H x| over the whole [M, K] tensor (|x| when
    hadamard is 0): the input of the dynamic NVFP4 tensor scale
