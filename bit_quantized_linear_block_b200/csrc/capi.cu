@@ -138,6 +138,11 @@ ql_status check_m(int64_t M) {
   if (M > (int64_t(1) << 31) - 128) return QL_ERR_UNSUPPORTED_SHAPE;
   return QL_OK;
 }
+// Streaming kernels index 128-element blocks with 32-bit integers.
+ql_status check_mk(int64_t M, int64_t K) {
+  if ((M + 127) / 128 * 128 * (K / 128) >= (int64_t(1) << 32)) return QL_ERR_UNSUPPORTED_SHAPE;
+  return QL_OK;
+}
 ql_status check_w(const ql_weights* w) {
   if (w == nullptr || w->codes == nullptr) return QL_ERR_INVALID_ARG;
   if (w->fmt != QL_W_NVFP4 && w->fmt != QL_W_QARVD_INT4) return QL_ERR_INVALID_ARG;
@@ -245,6 +250,7 @@ ql_status qlinear_prepare_weights(const void* W, int32_t N, int32_t K, const ql_
   if (cfg->fmt != QL_W_NVFP4 && cfg->fmt != QL_W_QARVD_INT4) return QL_ERR_INVALID_ARG;
   QL_TRY(check_k(K));
   if (N <= 0 || N % 16 != 0 || N > (1 << 24)) return QL_ERR_UNSUPPORTED_SHAPE;
+  QL_TRY(check_mk(N, K));
   if (cfg->fmt == QL_W_QARVD_INT4 && (cfg->hadamard != 0 || K > 16384 || !(cfg->tau > 0.f) ||
                                       !(cfg->alpha >= 0.f)))
     return QL_ERR_INVALID_ARG;
@@ -316,6 +322,7 @@ ql_status qlinear_tensor_amax(const void* X, int64_t M, int32_t K, int32_t hadam
                               void* ws, size_t ws_bytes, void* stream) {
   QL_TRY(check_m(M));
   QL_TRY(check_k(K));
+  QL_TRY(check_mk(M, K));
   if (amax_out == nullptr || ws == nullptr || (M > 0 && X == nullptr)) return QL_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(amax_out, 4) || !aligned(ws, 256)) return QL_ERR_ALIGNMENT;
   if (ws_bytes < qlinear_quantize_ws_bytes(M, K, QL_ROUTE_NVFP4)) return QL_ERR_WORKSPACE;
@@ -329,6 +336,7 @@ ql_status qlinear_quantize_act(const void* X, int64_t M, int32_t K, int32_t act_
                                void* stream) {
   QL_TRY(check_m(M));
   QL_TRY(check_k(K));
+  QL_TRY(check_mk(M, K));
   if (codes == nullptr || scales == nullptr || ws == nullptr || (M > 0 && X == nullptr))
     return QL_ERR_INVALID_ARG;
   if (act_fmt == QL_ROUTE_NVFP4) {
@@ -396,6 +404,7 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
                           void* ws, size_t ws_bytes, void* stream) {
   QL_TRY(check_m(M));
   QL_TRY(check_w(w));
+  QL_TRY(check_mk(M, w->K));
   if (ws == nullptr || (M > 0 && (X == nullptr || Y == nullptr))) return QL_ERR_INVALID_ARG;
   const int32_t fmt = (w->fmt == QL_W_QARVD_INT4) ? int32_t(QL_ACT_INT8_TENSOR) : route;
   if (fmt != QL_ROUTE_NVFP4 && fmt != QL_ROUTE_INT8 && fmt != QL_ACT_INT8_TENSOR) return QL_ERR_INVALID_ARG;

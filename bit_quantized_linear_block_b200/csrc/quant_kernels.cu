@@ -66,40 +66,169 @@ __device__ __forceinline__ float warp_max(float m) {
 }
 
 // ---------------------------------------------------------------------------
+// Streaming front end shared by the amax and NVFP4 kernels: half a Hadamard
+// block (64 bf16 = 128 bytes) per lane, the two halves of a block in lanes
+// 2i and 2i+1.
+//
+// A warp walks the flat tensor in chunks of 16 blocks (4 KB) with a
+// kRing-deep cp.async ring of 4 KB slots in shared memory.  Loads are 16-byte
+// cp.async copies in which lane l takes bytes 16*(l + 32 i) of the chunk, so
+// one instruction moves 512 contiguous bytes.  Each lane's 128 bytes land in
+// their own 128-byte region with 16-byte slot s stored at s ^ (lane % 8);
+// the read-back, where every lane reads its own region slot by slot, is then
+// free of bank conflicts.
+// ---------------------------------------------------------------------------
+constexpr int kRing = 3;                         // stages per warp
+constexpr int kLaneBytes = 128;                  // 64 bf16
+constexpr int kChunkBytes = 32 * kLaneBytes;     // 16 blocks of 128 bf16
+constexpr int kWarpsPerCta = kThreadsHbm / 32;                         // amax: 2 CTAs/SM
+constexpr int kRingBytesPerCta = kWarpsPerCta * kRing * kChunkBytes;   // 96 KB
+constexpr int kRingCtasPerSm = 2;
+constexpr int kQuantThreads = 384;                                     // NVFP4: 1 CTA/SM
+constexpr int kQuantWarps = kQuantThreads / 32;
+constexpr int kQuantRingBytes = kQuantWarps * kRing * kChunkBytes;     // 144 KB
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Issue the copies of chunk `c` (past the end: zero-size copies that read
+// nothing) into ring slot `slot`.
+__device__ __forceinline__ void issue_chunk(uint32_t ring, int slot, const uint8_t* base,
+                                            int64_t total_bytes, int64_t c) {
+  const uint32_t lane = lane_id();
+  const int64_t cbase = c * kChunkBytes;
+  const uint32_t sbase = ring + slot * kChunkBytes;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t o = 16u * (lane + 32u * i);
+    const uint32_t owner = o >> 7, s16 = (o >> 4) & 7u;
+    const uint32_t dst = sbase + owner * kLaneBytes + ((s16 ^ (owner & 7u)) << 4);
+    const bool ok = cbase + o < total_bytes;
+    cp_async16(dst, ok ? static_cast<const void*>(base + cbase + o) : static_cast<const void*>(base),
+               ok ? 16u : 0u);
+  }
+}
+
+// This lane's 64 elements of a landed slot, in pair registers
+// P[j] = (x_j, x_{j+32}), j = 0..31 (indices within the lane's half block).
+__device__ __forceinline__ void read_half(const uint8_t* slot_ptr, float2 (&P)[32]) {
+  const uint32_t lane = lane_id();
+  const uint8_t* my = slot_ptr + lane * kLaneBytes;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint4 a = *reinterpret_cast<const uint4*>(my + ((s ^ (lane & 7u)) << 4));        // x_{8s..8s+7}
+    const uint4 b = *reinterpret_cast<const uint4*>(my + (((s + 4) ^ (lane & 7u)) << 4));  // x_{32+8s..}
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      P[8 * s + 2 * i] = make_float2(bf16_lo(wa[i]), bf16_lo(wb[i]));
+      P[8 * s + 2 * i + 1] = make_float2(bf16_hi(wa[i]), bf16_hi(wb[i]));
+    }
+  }
+}
+
+// Block-128 FWHT with the block split over lanes 2i (elements 0..63) and 2i+1
+// (64..127).  Distances 1..16 are butterflies between pairs (packed f32x2),
+// 32 is inside each pair, 64 goes across the lane pair.  Each butterfly
+// (a, b) -> (RN(a + b), RN(a - b)); a - b is computed as fma(b, -1, a),
+// which rounds the same exact value once.  All lanes must call this.
+__device__ __forceinline__ void fwht128_half(float2 (&P)[32]) {
+  const float2 m1 = make_float2(-1.f, -1.f);
+#pragma unroll
+  for (int s = 1; s < 32; s <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if ((j & s) == 0) {
+        const float2 a = P[j], b = P[j + s];
+        P[j] = __fadd2_rn(a, b);
+        P[j + s] = __ffma2_rn(b, m1, a);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const float a = P[j].x, b = P[j].y;
+    P[j] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
+  const float sg = (lane_id() & 1u) ? -1.f : 1.f;
+  const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    float2 p;
+    p.x = __shfl_xor_sync(0xffffffffu, P[j].x, 1);
+    p.y = __shfl_xor_sync(0xffffffffu, P[j].y, 1);
+    P[j] = __ffma2_rn(P[j], sg2, p);   // lower half: x + p, upper half: p - x
+  }
+}
+
+// Per-warp ring driver: calls body(P, half_index) for each half block this
+// lane owns (half_index = 2 * block + (lane & 1)).
+template <int WARPS, class Body>
+__device__ __forceinline__ void stream_blocks(const uint8_t* x, int64_t total_bytes, int hadamard,
+                                              uint8_t* ring_all, Body body) {
+  const int wid = threadIdx.x >> 5;
+  uint8_t* ring_g = ring_all + wid * kRing * kChunkBytes;
+  const uint32_t ring = smem_u32(ring_g);
+  const int64_t nchunks = (total_bytes + kChunkBytes - 1) / kChunkBytes;
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * WARPS + wid;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * WARPS;
+  const int64_t mine = (gw < nchunks) ? (nchunks - gw + nw - 1) / nw : 0;
+#pragma unroll
+  for (int i = 0; i < kRing - 1; ++i) {
+    issue_chunk(ring, i, x, total_bytes, gw + i * nw);
+    cp_async_commit();
+  }
+  for (int64_t k = 0; k < mine; ++k) {
+    issue_chunk(ring, static_cast<int>((k + kRing - 1) % kRing), x, total_bytes, gw + (k + kRing - 1) * nw);
+    cp_async_commit();
+    cp_async_wait<kRing - 1>();
+    __syncwarp();
+    float2 P[32];
+    read_half(ring_g + (k % kRing) * kChunkBytes, P);
+    __syncwarp();
+    if (hadamard) fwht128_half(P);
+    body(P, (gw + k * nw) * 32 + lane_id());
+  }
+  cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
 // amax of |H x| (or |x| when hadamard == 0) over a contiguous tensor whose
 // element count is a multiple of 128.  Each CTA writes its partial max; the
 // last CTA to finish (atomic ticket) folds them into *amax_out and resets
 // the ticket.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreadsHbm)
-    k_amax(const uint4* __restrict__ x, int64_t units, int hadamard, float* __restrict__ partials,
-           unsigned int* __restrict__ ticket, float* __restrict__ amax_out) {
+__global__ void __launch_bounds__(kThreadsHbm, kRingCtasPerSm)
+    k_amax(const uint8_t* __restrict__ x, int64_t total_bytes, int hadamard,
+           float* __restrict__ partials, unsigned int* __restrict__ ticket, float* __restrict__ amax_out) {
+  extern __shared__ __align__(128) uint8_t ring_all[];
   const uint32_t lane = lane_id();
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t chunks = (units + 7) >> 3;
   float m = 0.f;
-  for (int64_t c = warp; c < chunks; c += nwarps) {
-    const int64_t u = c * 8 + (lane >> 2);
-    float v[32];
-    if (u < units) {
-      load32(x + (c * 1024 + lane * 32) / 8, v);
-    } else {
+  stream_blocks<kWarpsPerCta>(x, total_bytes, hadamard, ring_all, [&](float2 (&P)[32], int64_t) {
+    float2 mm = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = 0.f;
+    for (int j = 0; j < 32; ++j) {
+      mm.x = fmaxf(mm.x, fabsf(P[j].x));
+      mm.y = fmaxf(mm.y, fabsf(P[j].y));
     }
-    if (hadamard) fwht128(v, lane & 3);
-#pragma unroll
-    for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
-  }
+    m = fmaxf(m, fmaxf(mm.x, mm.y));   // blocks past the end hold zeros
+  });
   m = warp_max(m);
-  __shared__ float red[kThreadsHbm / 32];
+  __shared__ float red[kWarpsPerCta];
   __shared__ bool s_last;
   if (lane == 0) red[threadIdx.x >> 5] = m;
   __syncthreads();
   if (threadIdx.x == 0) {
     float r = red[0];
-    for (int i = 1; i < kThreadsHbm / 32; ++i) r = fmaxf(r, red[i]);
+    for (int i = 1; i < kWarpsPerCta; ++i) r = fmaxf(r, red[i]);
     partials[blockIdx.x] = r;
     __threadfence();
     s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
@@ -118,72 +247,95 @@ __global__ void __launch_bounds__(kThreadsHbm)
   }
 }
 
+// Eight E2M1 codes (hardware RN-even, saturating convert), element 0 in
+// bits 0-3 ... element 7 in bits 28-31.  Each convert packs its second
+// source operand in the low nibble and its first in the high nibble.
+__device__ __forceinline__ uint32_t e2m1x8(float a0, float a1, float a2, float a3, float a4, float a5,
+                                           float a6, float a7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+  return r;
+}
+
 // ---------------------------------------------------------------------------
 // NVFP4 quantizer.  g = amax / 2688 (1 if amax == 0) from the device amax.
 // Per 16-element block: sb = E4M3(RN(amax_b / RN(6 g))); if sb == 0 all
 // codes are +0, else code = E2M1(RN(h * RN(1 / RN(sb * g)))).
-// Rows M .. Mpad-1 (padding of the last 128-row atom) get zero scales.
+// In the pair layout each lane holds four 16-element blocks, two in the .x
+// and two in the .y halves of its registers, so two blocks are scaled by one
+// packed multiply.  Rows M .. Mpad-1 (padding of the last
+// 128-row atom) get zero scales.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreadsHbm)
-    k_quant_nvfp4(const uint4* __restrict__ x, int64_t M, int32_t K, int hadamard,
+__global__ void __launch_bounds__(kQuantThreads, 1)
+    k_quant_nvfp4(const uint8_t* __restrict__ x, int64_t M, int32_t K, int hadamard,
                   const float* __restrict__ amax_in, uint4* __restrict__ codes,
                   uint8_t* __restrict__ sf_mma, uint8_t* __restrict__ sf_rm,
                   float* __restrict__ g_out) {
-  const float amax = __ldg(amax_in);
-  const float g = (amax == 0.f) ? 1.f : __fdiv_rn(amax, 2688.f);
+  extern __shared__ __align__(128) uint8_t ring_all[];
+  const float amax_t = __ldg(amax_in);
+  const float g = (amax_t == 0.f) ? 1.f : __fdiv_rn(amax_t, 2688.f);
   if (blockIdx.x == 0 && threadIdx.x == 0 && g_out != nullptr) *g_out = g;
   const float d = __fmul_rn(6.f, g);
-
-  const uint32_t lane = lane_id();
-  const int32_t upr = K >> 7;                 // Hadamard blocks per row
-  const int32_t k_atoms = K >> 6;             // 4-scale groups per row
-  const int64_t mpad = (M + 127) & ~int64_t(127);
-  const int64_t units = M * upr, units_pad = mpad * upr;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const int64_t chunks = (units_pad + 7) >> 3;
-  const uint32_t q = lane & 3;
-
-  for (int64_t c = warp; c < chunks; c += nwarps) {
-    const int64_t u = c * 8 + (lane >> 2);
-    const bool real = u < units;
-    float v[32];
-    if (real) {
-      load32(x + (u * 128 + q * 32) / 8, v);
-    } else {
+  const uint32_t upr = static_cast<uint32_t>(K >> 7);
+  const int32_t k_atoms = K >> 6;
+  const int64_t units = M * upr;
+  const int64_t halves = 2 * units;
+  stream_blocks<kQuantWarps>(x, M * K * 2, hadamard, ring_all, [&](float2 (&P)[32], int64_t hu) {
+    if (hu >= halves) return;
+    // 16-element blocks of this half: b = 0, 1 in P[16b..16b+15].x, b = 2, 3
+    // in the .y halves of the same registers.
+    uint32_t sb[4];
+    uint32_t cw[8];   // codes of elements 8i .. 8i+7 of this half in cw[i]
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = 0.f;
-    }
-    if (hadamard) fwht128(v, q);
-    if (u >= units_pad) continue;
-    const int64_t row = u / upr;
-    const int32_t blk = static_cast<int32_t>(u - row * upr);
-    const int32_t j0 = blk * 8 + static_cast<int32_t>(q) * 2;    // first of this lane's 2 scales
-    uint32_t sb[2] = {0u, 0u};
-    uint32_t packed[4] = {0u, 0u, 0u, 0u};
-    if (real) {
+    for (int b = 0; b < 2; ++b) {
+      float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        float amax = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[16 * b + j]));
-        sb[b] = e4m3_code(__fdiv_rn(amax, d));
-        if (sb[b] != 0u) {
-          const float inv = __frcp_rn(__fmul_rn(e4m3_value(sb[b]), g));
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const uint32_t cd = e2m1_code(__fmul_rn(v[16 * b + j], inv));
-            packed[2 * b + j / 8] |= cd << (4 * (j % 8));
-          }
-        }
+      for (int t = 0; t < 16; ++t) {
+        a.x = fmaxf(a.x, fabsf(P[16 * b + t].x));
+        a.y = fmaxf(a.y, fabsf(P[16 * b + t].y));
       }
-      codes[(u * 128 + q * 32) / 32] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      if (sf_rm != nullptr)
-        *reinterpret_cast<uint16_t*>(sf_rm + row * (K >> 4) + j0) =
-            static_cast<uint16_t>(sb[0] | (sb[1] << 8));
+      sb[b] = e4m3_code(__fdiv_rn(a.x, d));
+      sb[b + 2] = e4m3_code(__fdiv_rn(a.y, d));
+      const float2 inv = make_float2(sb[b] ? __frcp_rn(__fmul_rn(e4m3_value(sb[b]), g)) : 0.f,
+                                     sb[b + 2] ? __frcp_rn(__fmul_rn(e4m3_value(sb[b + 2]), g)) : 0.f);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = 16 * b + 8 * h;
+        float2 y[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) y[t] = __fmul2_rn(P[j + t], inv);
+        const uint32_t lo = e2m1x8(y[0].x, y[1].x, y[2].x, y[3].x, y[4].x, y[5].x, y[6].x, y[7].x);
+        const uint32_t hi = e2m1x8(y[0].y, y[1].y, y[2].y, y[3].y, y[4].y, y[5].y, y[6].y, y[7].y);
+        cw[2 * b + h] = sb[b] ? lo : 0u;           // all-zero block -> +0 codes
+        cw[4 + 2 * b + h] = sb[b + 2] ? hi : 0u;
+      }
     }
-    *reinterpret_cast<uint16_t*>(sf_mma + sf_mma_offset(row, j0, k_atoms)) =
-        static_cast<uint16_t>(sb[0] | (sb[1] << 8));
+    uint4* dst = codes + hu * 2;
+    dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    // half index -> (row, first scale index); 32-bit division (units < 2^32)
+    const uint32_t u = static_cast<uint32_t>(hu >> 1);
+    const uint32_t row = u / upr;
+    const uint32_t j0 = (u - row * upr) * 8 + (static_cast<uint32_t>(hu) & 1u) * 4;
+    const uint32_t sw = sb[0] | (sb[1] << 8) | (sb[2] << 16) | (sb[3] << 24);
+    *reinterpret_cast<uint32_t*>(sf_mma + sf_mma_offset(row, j0, k_atoms)) = sw;
+    if (sf_rm != nullptr) *reinterpret_cast<uint32_t*>(sf_rm + static_cast<size_t>(row) * (K >> 4) + j0) = sw;
+  });
+  // zero scales of the padding rows of the last 128-row atom
+  const int64_t mpad = (M + 127) & ~int64_t(127);
+  const int64_t pad_words = (mpad - M) * (K >> 6);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < pad_words;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = M + i / (K >> 6);
+    const int32_t j0 = static_cast<int32_t>(i % (K >> 6)) * 4;
+    *reinterpret_cast<uint32_t*>(sf_mma + sf_mma_offset(row, j0, k_atoms)) = 0u;
   }
 }
 
@@ -303,24 +455,37 @@ int hbm_grid(int64_t work_items, int per_cta) {
   return static_cast<int>(std::max<int64_t>(1, std::min(want, cap)));
 }
 
+// Streaming kernels with the cp.async ring: 96 KB of shared memory and at
+// most 128 registers per thread, two resident CTAs per SM.
+static int ring_grid(int64_t nchunks) {
+  const int64_t want = (nchunks + kWarpsPerCta - 1) / kWarpsPerCta;
+  return static_cast<int>(
+      std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(num_sms()) * kRingCtasPerSm)));
+}
+
 ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* amax_out, void* ws,
                       cudaStream_t st) {
   const int64_t units = M * (K / 128);
-  const int grid = hbm_grid((units + 7) / 8, kThreadsHbm / 32);
+  if (units == 0) return cudaMemsetAsync(amax_out, 0, sizeof(float), st) == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  const int grid = ring_grid((units * 256 + kChunkBytes - 1) / kChunkBytes);
   float* partials = static_cast<float*>(ws);
   unsigned int* ticket = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + kAmaxPartialBytes);
-  k_amax<<<grid, kThreadsHbm, 0, st>>>(static_cast<const uint4*>(x), units, hadamard, partials, ticket,
-                                       amax_out);
+  if (!set_smem_attr(reinterpret_cast<const void*>(k_amax), kRingBytesPerCta)) return QL_ERR_CUDA;
+  k_amax<<<grid, kThreadsHbm, kRingBytesPerCta, st>>>(static_cast<const uint8_t*>(x), units * 256,
+                                                      hadamard, partials, ticket, amax_out);
   return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, const float* amax_in,
                              void* codes, void* sf_mma, void* sf_rm, float* g_out, cudaStream_t st) {
-  const int64_t mpad = (M + 127) / 128 * 128;
-  const int grid = hbm_grid((mpad * (K / 128) + 7) / 8, kThreadsHbm / 32);
-  k_quant_nvfp4<<<grid, kThreadsHbm, 0, st>>>(static_cast<const uint4*>(x), M, K, hadamard, amax_in,
-                                              static_cast<uint4*>(codes), static_cast<uint8_t*>(sf_mma),
-                                              static_cast<uint8_t*>(sf_rm), g_out);
+  if (M == 0) return QL_OK;
+  const int64_t nchunks = (M * K * 2 + kChunkBytes - 1) / kChunkBytes;
+  const int grid = static_cast<int>(std::max<int64_t>(
+      1, std::min<int64_t>((nchunks + kQuantWarps - 1) / kQuantWarps, num_sms())));
+  if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_nvfp4), kQuantRingBytes)) return QL_ERR_CUDA;
+  k_quant_nvfp4<<<grid, kQuantThreads, kQuantRingBytes, st>>>(
+      static_cast<const uint8_t*>(x), M, K, hadamard, amax_in, static_cast<uint4*>(codes),
+      static_cast<uint8_t*>(sf_mma), static_cast<uint8_t*>(sf_rm), g_out);
   return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
