@@ -78,9 +78,13 @@ bool set_smem_attr(const void* kernel, int bytes) {
   std::lock_guard<std::mutex> lk(g_mu);
   auto it = g_smem_set[d].find(kernel);
   if (it != g_smem_set[d].end() && it->second >= bytes) return true;
-  if (bytes > 48 * 1024 &&
-      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+  // Opt in whenever dynamic shared memory is used: static shared memory
+  // counts against the same 48 KB default.
+  if (bytes > 0 &&
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+    (void)cudaGetLastError();
     return false;
+  }
   g_smem_set[d][kernel] = bytes;
   return true;
 }

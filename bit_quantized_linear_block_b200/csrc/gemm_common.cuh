@@ -54,15 +54,16 @@ __device__ __forceinline__ void fail_timeout(int* status, volatile int* abort_fl
   *abort_flag = 1;
 }
 
-// Accumulator-ready wait of the 128 epilogue threads with ONE decision for
-// all of them: thread 128 does the bounded wait and publishes the outcome
+// Accumulator-ready wait of the 128 epilogue threads (one 128-aligned group
+// of four warps) with ONE decision for all of them: the group's first thread
+// does the bounded wait and publishes the outcome
 // through shared memory behind a named barrier, so no epilogue thread can
 // leave the tile loop while another one waits at a later named barrier.
 // The flag slot sits right after the abort flag.
 __device__ __forceinline__ bool epilogue_wait_uniform(uint64_t* bar, uint32_t parity, long long limit,
                                                       volatile int* abort_flag, int* status) {
   volatile int* slot = abort_flag + 1;
-  if (threadIdx.x == 128) {
+  if ((threadIdx.x & 127) == 0) {
     const bool ok = (*abort_flag == 0) && mbar_wait(bar, parity, limit);
     if (!ok) fail_timeout(status, abort_flag);
     *slot = ok ? 1 : 0;
@@ -97,12 +98,13 @@ struct EpilogueState {
 
 // Store one 64-column chunk (this thread's row `row`, values v[0..63]) via
 // the swizzled staging buffer and a TMA store.  Called by all 128 epilogue
-// threads (warps 4-7); thread 128 issues the bulk operations.
+// threads (a 128-aligned group of four warps); its first thread issues the
+// bulk operations.
 __device__ __forceinline__ void epilogue_store_chunk(const uint32_t (&packed)[32], uint8_t* sC,
                                                      const CUtensorMap* tm_y, int c0, int r0,
                                                      EpilogueState& es) {
   const int row = threadIdx.x & 127;
-  const bool leader = threadIdx.x == 128;
+  const bool leader = row == 0;
   if (leader) bulk_wait_read<1>();
   named_bar_sync(1, 128);
   uint8_t* dst = sC + es.buf * kEpiChunkBytes + row * 128;
@@ -119,16 +121,22 @@ __device__ __forceinline__ void epilogue_store_chunk(const uint32_t (&packed)[32
   es.buf ^= 1;
 }
 
-// bf16 epilogue of one BM x BN fp32 accumulator: y = alpha * acc.  Frees
-// the accumulator (arrive on `tempty`) as soon as the last columns are in
-// registers.
+// bf16 epilogue of one BM x BN fp32 accumulator: y = alpha * acc, with
+// alpha multiplied by row_scale[row] when row_scale is given (rows past
+// the end of the operand read no scale).  Frees the accumulator (arrive on
+// `tempty`) as soon as the last columns are in registers.
 template <int BN>
 __device__ __forceinline__ void epilogue_tile(uint32_t acc_tmem, uint64_t* tempty, uint8_t* sC,
                                               const CUtensorMap* tm_y, int m0, int n0, int N,
-                                              float alpha, EpilogueState& es) {
+                                              float alpha, EpilogueState& es,
+                                              const float* row_scale = nullptr, int M = 0) {
   const int ew = (threadIdx.x >> 5) & 3;
   const int lane = threadIdx.x & 31;
   constexpr int CH = BN / kEpiChunkCols;
+  if (row_scale != nullptr) {
+    const int m = m0 + (threadIdx.x & 127);
+    alpha = (m < M) ? __fmul_rn(alpha, __ldg(row_scale + m)) : 0.f;
+  }
 #pragma unroll 1
   for (int c = 0; c < CH; ++c) {
     uint32_t r0[32], r1[32];
@@ -154,7 +162,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t acc_tmem, uint64_t* tempt
 }
 
 __device__ __forceinline__ void epilogue_finish(EpilogueState&) {
-  if (threadIdx.x == 128) bulk_wait_all();
+  if ((threadIdx.x & 127) == 0) bulk_wait_all();
 }
 
 // ---------------------------------------------------------------------------

@@ -236,7 +236,7 @@ static ql_status launch_w4a4_cfg(const void* a_codes, const uint8_t* a_sf, const
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int grid = std::min(p.num_tiles, num_sms());
   kern<<<grid, 256, C::SMEM, st>>>(ta, tb, ty, p);
-  return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 ql_status launch_gemm_w4a4(const void* a_codes, const uint8_t* a_sf, const float* g_a, int64_t M,

@@ -473,7 +473,7 @@ ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* 
   if (!set_smem_attr(reinterpret_cast<const void*>(k_amax), kRingBytesPerCta)) return QL_ERR_CUDA;
   k_amax<<<grid, kThreadsHbm, kRingBytesPerCta, st>>>(static_cast<const uint8_t*>(x), units * 256,
                                                       hadamard, partials, ticket, amax_out);
-  return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, const float* amax_in,
@@ -486,7 +486,7 @@ ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, 
   k_quant_nvfp4<<<grid, kQuantThreads, kQuantRingBytes, st>>>(
       static_cast<const uint8_t*>(x), M, K, hadamard, amax_in, static_cast<uint4*>(codes),
       static_cast<uint8_t*>(sf_mma), static_cast<uint8_t*>(sf_rm), g_out);
-  return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadamard, void* codes,
@@ -495,7 +495,7 @@ ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadam
   const int grid = hbm_grid(M, kThreadsHbm / 32);
   k_quant_int8_token<<<grid, kThreadsHbm, 0, st>>>(static_cast<const uint4*>(x), M, K, hadamard,
                                                    static_cast<int8_t*>(codes), scales);
-  return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int32_t Kp,
@@ -508,7 +508,7 @@ ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int
   k_quant_int8_tensor_perm<<<grid, kThreadsHbm, smem, st>>>(
       static_cast<const __nv_bfloat16*>(x), M, K, Kp, gather, amax_in, static_cast<int8_t*>(codes),
       scale_out);
-  return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 }  // namespace ql

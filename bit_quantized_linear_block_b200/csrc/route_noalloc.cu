@@ -145,5 +145,5 @@ extern "C" ql_status qlinear_route_noalloc(const void* in, const void* out, int6
   k_gamma_route_static<<<static_cast<unsigned int>(grid), ql::kThreadsHbm, 0, st>>>(
       static_cast<const uint4*>(in), static_cast<const uint4*>(out), numel,
       static_cast<unsigned char*>(scratch), threshold, gamma_dev, route_dev);
-  return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }

@@ -286,7 +286,7 @@ ql_status launch_gamma_route(const void* in, const void* out, int64_t numel, flo
   k_gamma_route<<<grid, kThreadsHbm, 0, st>>>(static_cast<const uint4*>(in),
                                               static_cast<const uint4*>(out), numel, partials,
                                               ticket, threshold, gamma, route);
-  return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 int qarvd_slices(int32_t N) { return std::max(1, std::min(64, N / 64)); }
@@ -299,7 +299,7 @@ ql_status launch_qarvd_prepare(const void* W, int32_t N, int32_t K, float tau, f
   dim3 g1((K / 2 + kThreadsHbm - 1) / kThreadsHbm, slices);
   k_colnorm_partial<<<g1, kThreadsHbm, 0, st>>>(static_cast<const uint32_t*>(W), N, K,
                                                 rows_per_slice, partial);
-  if (cudaPeekAtLastError() != cudaSuccess) return QL_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return QL_ERR_CUDA;
   int npow2 = 1;
   while (npow2 < K) npow2 <<= 1;
   const size_t smem_sel = static_cast<size_t>(npow2) * sizeof(double) + static_cast<size_t>(K) * 4;
@@ -307,7 +307,7 @@ ql_status launch_qarvd_prepare(const void* W, int32_t N, int32_t K, float tau, f
     return QL_ERR_CUDA;
   k_qarvd_select<<<1, 1024, smem_sel, st>>>(partial, slices, K, npow2, tau, alpha, w->Kp, w->norms,
                                             w->outlier_mask, w->perm, w->gather, w->kinfo);
-  if (cudaPeekAtLastError() != cudaSuccess) return QL_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return QL_ERR_CUDA;
   const size_t smem_pack = static_cast<size_t>(w->Kp) * sizeof(int32_t);
   if (!set_smem_attr(reinterpret_cast<const void*>(k_qarvd_pack), static_cast<int>(smem_pack)))
     return QL_ERR_CUDA;
@@ -315,7 +315,7 @@ ql_status launch_qarvd_prepare(const void* W, int32_t N, int32_t K, float tau, f
   k_qarvd_pack<<<grid, kThreadsHbm, smem_pack, st>>>(
       static_cast<const __nv_bfloat16*>(W), N, K, w->Kp, w->outlier_mask, w->gather, w->kinfo,
       static_cast<uint8_t*>(w->codes), w->s_norm, w->s_out);
-  return cudaPeekAtLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 }  // namespace ql

@@ -32,8 +32,10 @@ def normwise_err(y, r):
 
 
 def excess_err(y, r):
-    """Error beyond the bf16 rounding of the output (2^-9 relative)."""
-    ex = np.maximum(0.0, np.abs(y - r) - 2.0 ** -9 * np.maximum(np.abs(y), np.abs(r)))
+    """Error beyond the round-to-nearest bf16 rounding of the output: bf16
+    keeps 8 significant bits, so that rounding alone moves a value by up to
+    2^-8 of its magnitude."""
+    ex = np.maximum(0.0, np.abs(y - r) - 2.0 ** -8 * np.maximum(np.abs(y), np.abs(r)))
     return float(ex.max() / max(np.abs(r).max(), 1e-30))
 
 
@@ -203,3 +205,84 @@ def test_gemm_timeout_path_reports_and_recovers(ql):
     assert ql.qlinear_device_status() == 0
     ref = O.forward(S.bf16_bits(x), O.prepare_weights_nvfp4(S.bf16_bits(w)), O.ROUTE_NVFP4)
     assert normwise_err(_np(y.float()).astype(np.float64), ref) <= 1e-2
+
+
+# ---------------------------------------------------------------- W4A8 (INT8 route)
+
+W4A8_CASES = [(256, 1920, 1920), (300, 384, 640), (129, 640, 384), (1000, 5760, 1920), (1, 192, 128)]
+
+
+@pytest.mark.parametrize("m,n,k", W4A8_CASES)
+def test_forward_w4a8_int8_route_parity(ql, m, n, k):
+    x = _x(m, k, seed=m * 3 + n)
+    w = S.weights(n, k, 0.02, 7, m + n + k)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    wq = O.prepare_weights_nvfp4(wb)
+    rows = np.arange(m) if m <= 512 else np.unique(np.r_[np.random.default_rng(1).choice(m, 256, replace=False), m - 1])
+    ref = O.forward(xb, wq, O.ROUTE_INT8, rows=rows)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True)
+    y = ql.qlinear_forward(x.cuda(), pw, ql.QL_ROUTE_INT8)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    yn = _np(y.float())[rows].astype(np.float64)
+    assert np.isfinite(yn).all()
+    assert excess_err(yn, ref) <= 1e-3
+
+
+# ---------------------------------------------------------------- Q-ARVD
+
+def _qarvd_weights(n, k, seed, frac=0.05, scale=20.0):
+    return S.weights(n, k, 0.02, seed, 77, outlier_frac=frac, outlier_scale=scale)
+
+
+def _assert_guard_band(pk, tau=3.5, alpha=2.0):
+    """Mask decisions are bit-exact only away from the boundaries."""
+    m = pk["zscore"][np.isfinite(pk["zscore"])]
+    assert np.all(np.abs(m - tau) > 1e-9 * tau)
+    assert np.all(np.abs(pk["norms"] - alpha * pk["median"]) > 1e-9 * max(pk["median"], 1e-30))
+
+
+@pytest.mark.parametrize("n,k,frac", [(384, 640, 0.05), (256, 3072, 0.02), (64, 128, 0.0), (160, 1024, 0.3)])
+def test_prepare_weights_qarvd_bit_exact(ql, n, k, frac):
+    w = _qarvd_weights(n, k, seed=n + k, frac=frac)
+    wb = S.bf16_bits(w)
+    pk = O.qarvd_pack(wb, 3.5, 2.0)
+    _assert_guard_band(pk)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_QARVD_INT4, hadamard=False, tau=3.5, alpha=2.0)
+    torch.cuda.synchronize()
+    kp = pw.desc.Kp
+    norms = _np(pw.view("norms", torch.float64, k))
+    assert np.allclose(norms, pk["norms"], rtol=1e-13, atol=0)
+    assert np.array_equal(_np(pw.view("outlier_mask", torch.uint8, k)).astype(bool), pk["mask"])
+    assert np.array_equal(_np(pw.view("perm", torch.int32, k)), pk["perm"])
+    kinfo = _np(pw.view("kinfo", torch.int32, 4)).tolist()
+    assert kinfo == [pk["k_norm"], pk["k_norm_pad"], pk["n_out"], pk["k_out_pad"]]
+    assert np.array_equal(_np(pw.view("s_norm", torch.float32, n)), pk["s_norm"])
+    assert np.array_equal(_np(pw.view("s_out", torch.float32, n)), pk["s_out"])
+    want = np.zeros((n, kp), np.int8)
+    want[:, :pk["codes"].shape[1]] = pk["codes"]
+    got = _np(pw.view("codes", torch.uint8, n * kp // 2)).reshape(n, kp // 2)
+    assert np.array_equal(got, O.pack_int4(want))
+
+
+@pytest.mark.parametrize("m,n,k", [(300, 384, 640), (256, 256, 3072), (77, 128, 128)])
+def test_qarvd_activation_quant_and_forward_parity(ql, m, n, k):
+    w = _qarvd_weights(n, k, seed=m + n)
+    pk = O.qarvd_pack(S.bf16_bits(w), 3.5, 2.0)
+    x = _x(m, k, seed=m + 5 * k)
+    xb = S.bf16_bits(x)
+    qx, sx = O.int8_per_tensor(O.bf16_bits_to_f32(xb))
+    qxp = O.qarvd_permute_activations(qx, pk["perm"], pk["k_norm"], pk["k_norm_pad"], pk["n_out"], pk["k_out_pad"])
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_QARVD_INT4, hadamard=False)
+    xc = x.cuda()
+    q = ql.qlinear_quantize_act(xc, ql.QL_ACT_INT8_TENSOR, hadamard=False, w=pw)
+    y = ql.qlinear_forward(xc, pw)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    kp = pw.desc.Kp
+    want = np.zeros((m, kp), np.int8)
+    want[:, :qxp.shape[1]] = qxp
+    assert _np(q["scales"])[0] == sx
+    assert np.array_equal(_np(q["codes"]), want)
+    ref = O.gemm_qarvd(qxp, sx, pk["codes"], pk["s_norm"], pk["s_out"], pk["k_norm_pad"])
+    assert excess_err(_np(y.float()).astype(np.float64), ref) <= 1e-3
