@@ -172,6 +172,12 @@ def gemm_source_sha() -> str:
 # ---------------------------------------------------------------------------
 # workload
 # ---------------------------------------------------------------------------
+def rank_seed_offset(rank: int) -> int:
+    """Seed offset of a rank's synthetic block (weak scaling: every rank
+    processes its own, independent block)."""
+    return 100 * rank
+
+
 def make_inputs(seed_offset: int):
     """Host (CPU, bf16) inputs of one block: 4 linear inputs, 4 weights and
     the router's input/output pair."""
@@ -193,7 +199,7 @@ def step_flops(lins) -> float:
 def run_ours(args, rank, world, local):
     from bit_quantized_linear_block_b200 import qlinear as ql
     dev = torch.device("cuda", local)
-    lins, bin_h, bout_h = make_inputs(seed_offset=100 * rank)
+    lins, bin_h, bout_h = make_inputs(seed_offset=rank_seed_offset(rank))
     flops = step_flops(lins)
     xs = [x.to(dev) for _, x, _ in lins]
     pws = [ql.qlinear_prepare_weights(w.to(dev), ql.QL_W_NVFP4, hadamard=True) for _, _, w in lins]

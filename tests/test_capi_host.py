@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads,
+exports every entry point include/qlinear.h declares, and rejects bad
+arguments before touching CUDA."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlinear.h")
+
+
+@pytest.fixture(scope="module")
+def ql():
+    from bit_quantized_linear_block_b200 import qlinear
+    return qlinear
+
+
+def declared_functions():
+    with open(HEADER) as f:
+        text = f.read()
+    return re.findall(r"QL_API\s+[\w\s\*]+?\b(qlinear_\w+)\s*\(", text)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for required in ("qlinear_prepare_weights", "qlinear_route", "qlinear_forward",
+                     "qlinear_quantize_act", "qlinear_gemm", "qlinear_tensor_amax",
+                     "qlinear_device_status", "qlinear_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(ql):
+    out = subprocess.run(["nm", "-D", "--defined-only", ql.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT\s+(qlinear_\w+)", out))
+    declared = set(declared_functions())
+    assert declared, "no declarations parsed"
+    assert declared <= exported, declared - exported
+    for name in declared:
+        getattr(ql.lib, name)              # resolvable through ctypes too
+
+
+def test_abi_version_and_status_strings(ql):
+    with open(HEADER) as f:
+        ver = int(re.search(r"#define QLINEAR_ABI_VERSION (\d+)", f.read()).group(1))
+    assert ql.lib.qlinear_abi_version() == ver
+    assert ql.lib.qlinear_status_string(0) == b"ok"
+    assert ql.lib.qlinear_status_string(5) == b"device wait timed out"
+    assert ql.lib.qlinear_status_string(99) == b"unknown status"
+
+
+def test_size_queries(ql):
+    assert ql.lib.qlinear_sf_bytes(17776, 1920) == 17792 * 120      # rows padded to 128
+    assert ql.lib.qlinear_sf_bytes(1, 128) == 128 * 8
+    assert ql.lib.qlinear_sf_bytes(-1, 128) == 0 and ql.lib.qlinear_sf_bytes(4, 100) == 0
+    cfg = ql.WeightCfg(ql.QL_W_NVFP4, 1, 3.5, 2.0)
+    assert ql.lib.qlinear_weights_bytes(1920, 1920, C.byref(cfg)) >= 1920 * 960 + 1920 * 120
+    assert ql.lib.qlinear_weights_bytes(1920, 1000, C.byref(cfg)) == 0          # K % 128
+    cq = ql.WeightCfg(ql.QL_W_QARVD_INT4, 0, 3.5, 2.0)
+    assert ql.lib.qlinear_weights_bytes(384, 640, C.byref(cq)) >= 384 * (640 + 64) // 2
+    assert ql.lib.qlinear_quantize_ws_bytes(10, 130, 0) == 0
+    assert ql.lib.qlinear_route_ws_bytes(-1) == 0 and ql.lib.qlinear_route_ws_bytes(10) > 0
+
+
+FAKE = 1 << 20        # a 256-aligned non-null address; never dereferenced
+
+
+def test_forward_rejects_bad_arguments_without_a_device(ql):
+    w = ql.Weights(fmt=ql.QL_W_NVFP4, N=1920, K=1920, hadamard=1, codes=FAKE, sf=FAKE, gscale=FAKE)
+    f = ql.lib.qlinear_forward
+    assert f(None, 10, C.byref(w), 0, FAKE, FAKE, 1 << 30, None) == 1             # null X
+    assert f(FAKE, -1, C.byref(w), 0, FAKE, FAKE, 1 << 30, None) == 1             # M < 0
+    assert f(FAKE + 8, 10, C.byref(w), 0, FAKE, FAKE, 1 << 30, None) == 3         # misaligned X
+    assert f(FAKE, 10, C.byref(w), 7, FAKE, FAKE, 1 << 30, None) == 1             # bad route
+    assert f(FAKE, 10, C.byref(w), 0, FAKE, FAKE, 16, None) == 6                  # workspace
+    bad = ql.Weights(fmt=ql.QL_W_NVFP4, N=1920, K=1000, hadamard=1, codes=FAKE, sf=FAKE, gscale=FAKE)
+    assert f(FAKE, 10, C.byref(bad), 0, FAKE, FAKE, 1 << 30, None) == 2           # K % 128
+    odd = ql.Weights(fmt=ql.QL_W_NVFP4, N=100, K=1920, hadamard=1, codes=FAKE, sf=FAKE, gscale=FAKE)
+    assert f(FAKE, 10, C.byref(odd), 0, FAKE, FAKE, 1 << 30, None) == 2           # N % 16
+
+
+def test_other_entry_points_reject_bad_arguments(ql):
+    L = ql.lib
+    assert L.qlinear_route(FAKE, FAKE, 100, 0.05, None, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.qlinear_route(FAKE + 4, FAKE, 100, 0.05, FAKE, FAKE, FAKE, 1 << 20, None) == 3
+    assert L.qlinear_route(FAKE, FAKE, 100, 0.05, FAKE, FAKE, FAKE, 8, None) == 6
+    assert L.qlinear_route(FAKE, FAKE, 100, float("nan"), FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    na = L.qlinear_route_noalloc
+    na.restype = C.c_int
+    na.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p]
+    assert na(FAKE, FAKE, -5, 0.05, FAKE, FAKE, None) == 1
+    assert na(FAKE, FAKE + 2, 5, 0.05, FAKE, FAKE, None) == 3
+    assert L.qlinear_tensor_amax(FAKE, 4, 96, 1, FAKE, FAKE, 1 << 20, None) == 2
+    assert L.qlinear_quantize_act(FAKE, 4, 128, 9, 1, None, None, FAKE, FAKE, None, FAKE, FAKE,
+                                  1 << 20, None) == 1
+    cfg = ql.WeightCfg(ql.QL_W_QARVD_INT4, 1, 3.5, 2.0)                          # Q-ARVD has no rotation
+    desc = ql.Weights()
+    assert L.qlinear_prepare_weights(FAKE, 256, 256, C.byref(cfg), FAKE, 1 << 30, C.byref(desc),
+                                     FAKE, 1 << 30, None) == 1
+    assert L.qlinear_gemm(0, FAKE, FAKE, FAKE, 10, None, FAKE, None) == 1
+
+
+def test_valid_call_without_a_device_reports_no_device(ql):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    w = ql.Weights(fmt=ql.QL_W_NVFP4, N=1920, K=1920, hadamard=1, codes=FAKE, sf=FAKE, gscale=FAKE)
+    assert ql.lib.qlinear_forward(FAKE, 10, C.byref(w), 0, FAKE, FAKE, 1 << 30, None) == 7
