@@ -46,7 +46,11 @@ FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PF
 NVFP4_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # bf16 in, E2M1 out, E4M3 per 16
 # DRAM bytes per launch of the W4A4 GEMM from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of the GEMM sources).
-GEMM_TRAFFIC = {}
+GEMM_TRAFFIC = {
+    # profiles/gemm_w4a4_cogvideox2b_dram_traffic.md: 562.4 MB over the 4 GEMM
+    # launches of one step
+    "0e74e78f2d6104a9": 562.4e6 / 4,
+}
 
 
 def parse():
@@ -58,7 +62,35 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-case", choices=["quant", "gemm"], default=None,
+                    help="run one small standalone case for an ncu capture (prints no JSON)")
     return ap.parse_args()
+
+
+def profile_case(which: str):
+    """Small cases for ncu captures: inputs larger than L2 but a few GB at
+    most, two launches of each kernel after one untimed call."""
+    from bit_quantized_linear_block_b200 import qlinear as ql
+    dev = torch.device("cuda", 0)
+    if which == "quant":     # amax + NVFP4 quantizer on [32768, 4096] (268 MB of bf16)
+        m, k = 32768, 4096
+        x = S.activations_with_outlier_channels(m, k, 0.01, 30.0, 1, 1).to(dev)
+        amax = ql.qlinear_tensor_amax(x, True)
+        q = ql.qlinear_quantize_act(x, ql.QL_ROUTE_NVFP4, True, rowmajor_scales=False, amax_in=amax)
+        for _ in range(2):
+            ql.qlinear_tensor_amax(x, True, out=amax)
+            ql.qlinear_quantize_act(x, ql.QL_ROUTE_NVFP4, True, amax_in=amax, out=q)
+    else:                    # W4A4 GEMM M=8192, N=7680, K=1920 (FFN-up shape, fewer tokens)
+        m, n, k = 8192, 7680, 1920
+        x = S.activations_with_outlier_channels(m, k, 0.01, 30.0, 1, 1).to(dev)
+        w = S.weights(n, k, 0.02, 1, 2).to(dev)
+        pw = ql.qlinear_prepare_weights(w, ql.QL_W_NVFP4, True)
+        q = ql.qlinear_quantize_act(x, ql.QL_ROUTE_NVFP4, True, rowmajor_scales=False)
+        y = ql.qlinear_gemm(ql.QL_ROUTE_NVFP4, q, m, pw)
+        for _ in range(2):
+            ql.qlinear_gemm(ql.QL_ROUTE_NVFP4, q, m, pw, Y=y)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
 
 
 # ---------------------------------------------------------------------------
@@ -449,6 +481,9 @@ def run_reference(args, rank, world):
 
 def main():
     args = parse()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     rank, world, local = dist_init()
     try:
         if args.impl == "reference":

@@ -88,7 +88,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
   return true;
 }
 
-// ---- TMA / bulk copies (no cluster multicast anywhere) ---------------------
+// ---- TMA / bulk copies (every CTA loads its own tiles into its own smem) ---
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t c0, int32_t c1) {
   asm volatile(
