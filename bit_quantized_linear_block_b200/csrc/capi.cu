@@ -112,6 +112,29 @@ bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t d0, int64_t d1,
+                  int64_t d2, int64_t stride1_bytes, int64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                  uint32_t b2) {
+  CUtensorMap dummy;
+  if (!make_tmap_2d(&dummy, dtype, base, d0, d1, stride1_bytes, b0, b1, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return false;   // also resolves the encoder
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d0), static_cast<cuuint64_t>(d1),
+                              static_cast<cuuint64_t>(d2)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(stride1_bytes), static_cast<cuuint64_t>(stride2_bytes)};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return g_encode(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_sf_tmap(CUtensorMap* map, const void* base, int64_t rows, int K, uint32_t box_k) {
+  const int64_t groups = (rows + 127) / 128;
+  const int64_t k_atoms = K / 64;
+  return make_tmap_3d(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, base, 128, k_atoms, groups, 512, k_atoms * 512, 128,
+                      box_k, 1);
+}
+
 void fill_gemm_args(GemmArgs& p, int64_t M, int N, int K, int BN, int* status) {
   p.M = static_cast<int32_t>(M);
   p.N = N;

@@ -166,11 +166,106 @@ __device__ __forceinline__ void epilogue_finish(EpilogueState&) {
 }
 
 // ---------------------------------------------------------------------------
+// Per-warp epilogue.  A warp reads 32 TMEM lanes (its lane quarter) of the
+// accumulator and owns those 32 output rows; it stores them in boxes of
+// 32 rows x 32 bf16 columns through its own staging buffers (2 KB each,
+// 64-byte swizzle) with TMA stores, so epilogue warps never wait for each
+// other.  The output tensor map has box {32, 32} and SWIZZLE_64B.
+// ---------------------------------------------------------------------------
+constexpr int kWarpBoxCols = 32;
+constexpr int kWarpBoxBytes = 32 * kWarpBoxCols * 2;   // 2 KB
+
+struct WarpStoreState {
+  int next;   // staging buffer for the next box
+};
+
+// Accumulator-ready wait of one warp: lane 0 does the bounded wait and the
+// outcome is broadcast, so the whole warp takes the same branch.
+__device__ __forceinline__ bool warp_wait_uniform(uint64_t* bar, uint32_t parity, long long limit,
+                                                  volatile int* abort_flag, int* status) {
+  int ok = 0;
+  if (lane_id() == 0) {
+    ok = (*abort_flag == 0) && mbar_wait(bar, parity, limit);
+    if (!ok) fail_timeout(status, abort_flag);
+  }
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// One warp's share of an accumulator tile: NCH boxes of 32 columns starting
+// at TMEM address `taddr` (lane quarter already folded in) and at output
+// column `col0`; output row of lane i = row0 + i.  y = bf16(alpha * acc),
+// alpha times row_scale[row] when row_scale is given.  After the TMEM reads
+// the warp arrives once on the mbarrier at `release` (a shared::cluster
+// address: this CTA's barrier or the pair leader's).  Boxes entirely past M
+// or N are skipped; TMA clips partial ones.
+template <int NCH, int NBUF>
+__device__ __forceinline__ void epilogue_warp_tile(uint32_t taddr, uint32_t release, uint8_t* stage,
+                                                   const CUtensorMap* tm_y, int row0, int col0, int M,
+                                                   int N, float alpha, WarpStoreState& ws,
+                                                   const float* row_scale = nullptr) {
+  const int lane = lane_id();
+  uint32_t r[NCH][32];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) tmem_ld32(taddr + kWarpBoxCols * c, r[c]);
+  tmem_ld_wait();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive_cluster(release);
+  if (row_scale != nullptr) {
+    const int row = row0 + lane;
+    alpha = (row < M) ? __fmul_rn(alpha, __ldg(row_scale + row)) : 0.f;
+  }
+  if (row0 >= M) return;   // warp-uniform
+  const uint32_t swz = (lane >> 1) & 3;
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const int col = col0 + kWarpBoxCols * c;
+    if (col >= N) break;   // warp-uniform
+    uint8_t* buf = stage + ws.next * kWarpBoxBytes;
+    if (lane == 0) bulk_wait_read<NBUF - 1>();
+    __syncwarp();
+    uint8_t* dst = buf + lane * 64;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 v;
+      v.x = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[c][8 * q + 0])),
+                        __fmul_rn(alpha, __uint_as_float(r[c][8 * q + 1])));
+      v.y = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[c][8 * q + 2])),
+                        __fmul_rn(alpha, __uint_as_float(r[c][8 * q + 3])));
+      v.z = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[c][8 * q + 4])),
+                        __fmul_rn(alpha, __uint_as_float(r[c][8 * q + 5])));
+      v.w = pack_bf16x2(__fmul_rn(alpha, __uint_as_float(r[c][8 * q + 6])),
+                        __fmul_rn(alpha, __uint_as_float(r[c][8 * q + 7])));
+      *reinterpret_cast<uint4*>(dst + ((q ^ swz) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tm_y, buf, col, row0);
+      bulk_commit();
+    }
+    ws.next = (ws.next + 1 == NBUF) ? 0 : ws.next + 1;
+  }
+}
+
+__device__ __forceinline__ void epilogue_warp_finish() {
+  if (lane_id() == 0) bulk_wait_all();
+  __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
 // Host helpers (defined in capi.cu)
 // ---------------------------------------------------------------------------
 bool make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t inner,
                   int64_t outer, int64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer,
                   CUtensorMapSwizzle swizzle);
+bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, int64_t d0, int64_t d1,
+                  int64_t d2, int64_t stride1_bytes, int64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                  uint32_t b2);
+// Block scales in the MMA layout as a 3-D tensor of 32-bit words
+// (128 words of a 512-byte atom, K/64 atoms of a 128-row group, row groups);
+// one box is box_k atoms (4 = one 256-value K stage) of one group.
+bool make_sf_tmap(CUtensorMap* map, const void* base, int64_t rows, int K, uint32_t box_k);
 int num_sms();
 bool set_smem_attr(const void* kernel, int bytes);
 void fill_gemm_args(GemmArgs& p, int64_t M, int N, int K, int BN, int* status);

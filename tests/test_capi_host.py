@@ -108,3 +108,4 @@ def test_valid_call_without_a_device_reports_no_device(ql):
         pytest.skip("a device is present")
     w = ql.Weights(fmt=ql.QL_W_NVFP4, N=1920, K=1920, hadamard=1, codes=FAKE, sf=FAKE, gscale=FAKE)
     assert ql.lib.qlinear_forward(FAKE, 10, C.byref(w), 0, FAKE, FAKE, 1 << 30, None) == 7
+
