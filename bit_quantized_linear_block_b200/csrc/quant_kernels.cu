@@ -215,11 +215,11 @@ __global__ void __launch_bounds__(kThreadsHbm, kRingCtasPerSm)
   stream_blocks<kWarpsPerCta>(x, total_bytes, hadamard, ring_all, [&](float2 (&P)[32], int64_t) {
     float2 mm = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      mm.x = fmaxf(mm.x, fabsf(P[j].x));
-      mm.y = fmaxf(mm.y, fabsf(P[j].y));
+    for (int j = 0; j < 32; j += 2) {
+      mm.x = fmax3(mm.x, fabsf(P[j].x), fabsf(P[j + 1].x));
+      mm.y = fmax3(mm.y, fabsf(P[j].y), fabsf(P[j + 1].y));
     }
-    m = fmaxf(m, fmaxf(mm.x, mm.y));   // blocks past the end hold zeros
+    m = fmax3(m, mm.x, mm.y);   // blocks past the end hold zeros
   });
   m = warp_max(m);
   __shared__ float red[kWarpsPerCta];
@@ -297,9 +297,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     for (int b = 0; b < 2; ++b) {
       float2 a = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        a.x = fmaxf(a.x, fabsf(P[16 * b + t].x));
-        a.y = fmaxf(a.y, fabsf(P[16 * b + t].y));
+      for (int t = 0; t < 16; t += 2) {
+        a.x = fmax3(a.x, fabsf(P[16 * b + t].x), fabsf(P[16 * b + t + 1].x));
+        a.y = fmax3(a.y, fabsf(P[16 * b + t].y), fabsf(P[16 * b + t + 1].y));
       }
       sb[b] = e4m3_code(__fdiv_rn(a.x, d));
       sb[b + 2] = e4m3_code(__fdiv_rn(a.y, d));

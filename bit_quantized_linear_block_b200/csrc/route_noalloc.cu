@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "ql_common.cuh"
+#include "route_common.cuh"
 #include "launchers.h"
 
 namespace {
@@ -25,12 +26,6 @@ static __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBy
 std::mutex g_setup_mu;
 void* g_scratch_addr[kMaxDev] = {nullptr};
 
-__device__ __forceinline__ double warp_sum(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 // Gamma = sum|out - in| / sum|in| (fp32 differences, fp64 sums) with the
 // scratch at `scratch`: partials [2 * gridDim.x] doubles, then the counter.
 __global__ void __launch_bounds__(ql::kThreadsHbm)
@@ -39,67 +34,9 @@ __global__ void __launch_bounds__(ql::kThreadsHbm)
                          double* __restrict__ gamma_out, int32_t* __restrict__ route_out) {
   double* partials = reinterpret_cast<double*>(scratch);
   unsigned int* ticket = reinterpret_cast<unsigned int*>(scratch + kTicketOffset);
-  double s1 = 0.0, s0 = 0.0;
-  const int64_t nvec = numel >> 3;
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nthr = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = tid; i < nvec; i += nthr) {
-    const uint4 a = __ldcs(in + i);
-    const uint4 b = __ldcs(out + i);
-    const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
-    const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float x0 = ql::bf16_lo(wa[k]), x1 = ql::bf16_hi(wa[k]);
-      const float y0 = ql::bf16_lo(wb[k]), y1 = ql::bf16_hi(wb[k]);
-      s1 += static_cast<double>(fabsf(__fsub_rn(y0, x0)));
-      s1 += static_cast<double>(fabsf(__fsub_rn(y1, x1)));
-      s0 += static_cast<double>(fabsf(x0));
-      s0 += static_cast<double>(fabsf(x1));
-    }
-  }
-  if (tid < (numel & 7)) {
-    const unsigned short* ia = reinterpret_cast<const unsigned short*>(in) + (nvec << 3) + tid;
-    const unsigned short* ib = reinterpret_cast<const unsigned short*>(out) + (nvec << 3) + tid;
-    const float x = __uint_as_float(static_cast<uint32_t>(*ia) << 16);
-    const float y = __uint_as_float(static_cast<uint32_t>(*ib) << 16);
-    s1 += static_cast<double>(fabsf(__fsub_rn(y, x)));
-    s0 += static_cast<double>(fabsf(x));
-  }
-  s1 = warp_sum(s1);
-  s0 = warp_sum(s0);
-  __shared__ double red[2][ql::kThreadsHbm / 32];
-  __shared__ bool s_last;
-  if ((threadIdx.x & 31) == 0) {
-    red[0][threadIdx.x >> 5] = s1;
-    red[1][threadIdx.x >> 5] = s0;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double a = 0.0, b = 0.0;
-    for (int i = 0; i < ql::kThreadsHbm / 32; ++i) {
-      a += red[0][i];
-      b += red[1][i];
-    }
-    partials[2 * blockIdx.x] = a;
-    partials[2 * blockIdx.x + 1] = b;
-    __threadfence();
-    s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
-  }
-  __syncthreads();
-  if (s_last && threadIdx.x == 0) {
-    __threadfence();
-    double a = 0.0, b = 0.0;
-    const volatile double* p = partials;
-    for (unsigned int i = 0; i < gridDim.x; ++i) {
-      a += p[2 * i];
-      b += p[2 * i + 1];
-    }
-    const double gamma = (b == 0.0) ? __longlong_as_double(0x7ff0000000000000ll) : a / b;
-    *gamma_out = gamma;
-    *route_out = (gamma > static_cast<double>(threshold)) ? 1 : 0;
-    *ticket = 0u;
-  }
+  double s1, s0;
+  ql::gamma_thread_sums(in, out, numel, s1, s0);
+  ql::gamma_finish(s1, s0, partials, ticket, threshold, gamma_out, route_out);
 }
 
 bool is_aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }

@@ -4,8 +4,8 @@
 // ||in||_1 of one transformer block; INT8 activations when Gamma exceeds
 // the threshold, NVFP4 otherwise.  One launch: grid-stride 16-byte loads of
 // both tensors, fp32 differences, fp64 per-thread sums, per-CTA partials,
-// and the last CTA to finish (atomic ticket) folds the partials in CTA order
-// and writes Gamma and the route.
+// and the last CTA to finish (atomic ticket) adds the partials and writes
+// Gamma and the route.
 //
 // Q-ARVD (Methodology / Formula and operation flow): input-channel L2 norms
 // of W, median and MAD, modified z-score M_k = (v_k - median)/MAD, outlier
@@ -13,15 +13,11 @@
 // channels, each class padded to 32; per output row one INT4 scale per
 // class.
 #include "ql_common.cuh"
+#include "route_common.cuh"
 #include "launchers.h"
 
 namespace ql {
 
-__device__ __forceinline__ double warp_sum_d(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 
 // ---------------------------------------------------------------------------
 // Gamma / route
@@ -30,69 +26,9 @@ __global__ void __launch_bounds__(kThreadsHbm)
     k_gamma_route(const uint4* __restrict__ in, const uint4* __restrict__ out, int64_t numel,
                   double* __restrict__ partials, unsigned int* __restrict__ ticket, float threshold,
                   double* __restrict__ gamma_out, int32_t* __restrict__ route_out) {
-  double s1 = 0.0, s0 = 0.0;
-  const int64_t nvec = numel >> 3;
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nthr = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = tid; i < nvec; i += nthr) {
-    const uint4 a = __ldcs(in + i);
-    const uint4 b = __ldcs(out + i);
-    const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
-    const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float x0 = bf16_lo(wa[k]), x1 = bf16_hi(wa[k]);
-      const float y0 = bf16_lo(wb[k]), y1 = bf16_hi(wb[k]);
-      s1 += static_cast<double>(fabsf(__fsub_rn(y0, x0)));
-      s1 += static_cast<double>(fabsf(__fsub_rn(y1, x1)));
-      s0 += static_cast<double>(fabsf(x0));
-      s0 += static_cast<double>(fabsf(x1));
-    }
-  }
-  if (tid < (numel & 7)) {  // ragged tail (< 8 elements)
-    const unsigned short* ia = reinterpret_cast<const unsigned short*>(in) + (nvec << 3) + tid;
-    const unsigned short* ib = reinterpret_cast<const unsigned short*>(out) + (nvec << 3) + tid;
-    const float x = __uint_as_float(static_cast<uint32_t>(*ia) << 16);
-    const float y = __uint_as_float(static_cast<uint32_t>(*ib) << 16);
-    s1 += static_cast<double>(fabsf(__fsub_rn(y, x)));
-    s0 += static_cast<double>(fabsf(x));
-  }
-  s1 = warp_sum_d(s1);
-  s0 = warp_sum_d(s0);
-  __shared__ double red[2][kThreadsHbm / 32];
-  __shared__ bool s_last;
-  const int w = threadIdx.x >> 5;
-  if (lane_id() == 0) {
-    red[0][w] = s1;
-    red[1][w] = s0;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double a = 0.0, b = 0.0;
-    for (int i = 0; i < kThreadsHbm / 32; ++i) {
-      a += red[0][i];
-      b += red[1][i];
-    }
-    partials[2 * blockIdx.x] = a;
-    partials[2 * blockIdx.x + 1] = b;
-    __threadfence();
-    const unsigned int t = atomicAdd(ticket, 1u);
-    s_last = (t == gridDim.x - 1);
-  }
-  __syncthreads();
-  if (s_last && threadIdx.x == 0) {
-    __threadfence();
-    double a = 0.0, b = 0.0;
-    const volatile double* p = partials;
-    for (unsigned int i = 0; i < gridDim.x; ++i) {
-      a += p[2 * i];
-      b += p[2 * i + 1];
-    }
-    const double gamma = (b == 0.0) ? __longlong_as_double(0x7ff0000000000000ll) : a / b;
-    *gamma_out = gamma;
-    *route_out = (gamma > static_cast<double>(threshold)) ? 1 : 0;
-    *ticket = 0u;  // the workspace is reusable by the next call on this stream
-  }
+  double s1, s0;
+  gamma_thread_sums(in, out, numel, s1, s0);
+  gamma_finish(s1, s0, partials, ticket, threshold, gamma_out, route_out);
 }
 
 // ---------------------------------------------------------------------------
