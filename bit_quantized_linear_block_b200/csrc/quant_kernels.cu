@@ -18,47 +18,6 @@
 
 namespace ql {
 
-// 32 bf16 -> fp32 from 64 contiguous bytes.
-__device__ __forceinline__ void load32(const uint4* __restrict__ src, float (&v)[32]) {
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uint4 u = __ldg(src + c);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[8 * c + 2 * i] = bf16_lo(w[i]);
-      v[8 * c + 2 * i + 1] = bf16_hi(w[i]);
-    }
-  }
-}
-
-// Fast Walsh-Hadamard transform of one 128-block spread over 4 lanes
-// (q = lane % 4 holds elements 32q .. 32q+31).  Stage distances 1, 2, ...,
-// 64 in that order; the pair (i, i+s) becomes (RN(a+b), RN(a-b)).  All 32
-// lanes of the warp must call this together.
-__device__ __forceinline__ void fwht128(float (&v)[32], uint32_t q) {
-#pragma unroll
-  for (int s = 1; s < 32; s <<= 1) {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if ((j & s) == 0) {
-        const float a = v[j], b = v[j + s];
-        v[j] = __fadd_rn(a, b);
-        v[j + s] = __fsub_rn(a, b);
-      }
-    }
-  }
-#pragma unroll
-  for (uint32_t t = 1; t <= 2; t <<= 1) {
-    const bool upper = (q & t) != 0;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float p = __shfl_xor_sync(0xffffffffu, v[j], t);
-      v[j] = upper ? __fsub_rn(p, v[j]) : __fadd_rn(v[j], p);
-    }
-  }
-}
-
 __device__ __forceinline__ float warp_max(float m) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -340,110 +299,163 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Per-token INT8: one warp per row.  Pass 1: amax_m of the rotated row.
-// Pass 2: recompute the rotation (the row is L1/L2 resident) and quantize
-// q = clamp(rint(RN(h * RN(127 / amax_m))), -127, 127); s_m = RN(amax_m/127).
+// Per-token INT8: one warp per row.  The bf16 row is copied into shared
+// memory with coalesced 16-byte cp.async (the next row's copy is in flight
+// while this one is quantized; 16-byte slots swizzled as in the streaming
+// ring), lane l takes half blocks 32 p + l (p = 0, 1, ...) with the same
+// half-block FWHT as the NVFP4 path.  amax_m = max |h| over the row,
+// q = clamp(rint(RN(h * RN(127 / amax_m))), -127, 127), s_m = RN(amax_m/127).
+// A row of at most 2048 elements is rotated once and stays in registers;
+// longer rows are rotated again, from shared memory, for the second pass.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv, int8_t* dst) {
+  uint32_t w[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {   // elements 4i..4i+3 (.x halves) and 32+4i.. (.y halves)
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int ql = max(-127, min(127, __float2int_rn(__fmul_rn(P[4 * i + b].x, inv))));
+      const int qh = max(-127, min(127, __float2int_rn(__fmul_rn(P[4 * i + b].y, inv))));
+      lo |= (static_cast<uint32_t>(ql) & 0xFFu) << (8 * b);
+      hi |= (static_cast<uint32_t>(qh) & 0xFFu) << (8 * b);
+    }
+    w[i] = lo;
+    w[8 + i] = hi;
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+}
+
 __global__ void __launch_bounds__(kThreadsHbm)
-    k_quant_int8_token(const uint4* __restrict__ x, int64_t M, int32_t K, int hadamard,
+    k_quant_int8_token(const uint8_t* __restrict__ x, int64_t M, int32_t K, int hadamard,
                        int8_t* __restrict__ codes, float* __restrict__ scales) {
+  extern __shared__ __align__(128) uint8_t s_rows[];
   const uint32_t lane = lane_id();
-  const uint32_t q = lane & 3;
-  const int32_t upr = K >> 7;
-  const int32_t passes = (upr + 7) >> 3;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  for (int64_t row = warp; row < M; row += nwarps) {
-    const uint4* xr = x + row * (K / 8);
+  const int wid = threadIdx.x >> 5;
+  const int32_t row_bytes = 2 * K;
+  const int32_t halves = K >> 6;                 // 64-element half blocks per row
+  const int32_t passes = (halves + 31) >> 5;
+  uint8_t* rows[2] = {s_rows + (2 * wid) * row_bytes, s_rows + (2 * wid + 1) * row_bytes};
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + wid;
+  const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
+  auto issue_row = [&](int64_t r, uint8_t* dst) {
+    const uint8_t* src = x + r * row_bytes;
+    const uint32_t d = smem_u32(dst);
+    for (int32_t o = 16 * static_cast<int32_t>(lane); o < row_bytes; o += 512) {
+      const uint32_t owner = static_cast<uint32_t>(o) >> 7, s16 = (static_cast<uint32_t>(o) >> 4) & 7u;
+      const bool ok = r < M;
+      cp_async16(d + owner * kLaneBytes + ((s16 ^ (owner & 7u)) << 4),
+                 ok ? static_cast<const void*>(src + o) : static_cast<const void*>(x), ok ? 16u : 0u);
+    }
+  };
+  auto load_half = [&](const uint8_t* row, int p, float2 (&P)[32]) {
+    if (32 * p + static_cast<int32_t>(lane) < halves) {
+      read_half(row + p * kChunkBytes, P);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) P[j] = make_float2(0.f, 0.f);
+    }
+    if (hadamard) fwht128_half(P);   // all lanes (pair shuffles)
+  };
+  issue_row(gw, rows[0]);
+  cp_async_commit();
+  int k = 0;
+  for (int64_t r = gw; r < M; r += nw, ++k) {
+    issue_row(r + nw, rows[(k + 1) & 1]);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncwarp();
+    const uint8_t* row = rows[k & 1];
+    float2 P[32];
     float m = 0.f;
     for (int p = 0; p < passes; ++p) {
-      const int32_t u = p * 8 + static_cast<int32_t>(lane >> 2);
-      float v[32];
-      if (u < upr) {
-        load32(xr + (u * 128 + q * 32) / 8, v);
-      } else {
+      load_half(row, p, P);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
-      }
-      if (hadamard) fwht128(v, q);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
+      for (int j = 0; j < 32; j += 2)
+        m = fmax3(m, fmax3(fabsf(P[j].x), fabsf(P[j].y), fabsf(P[j + 1].x)), fabsf(P[j + 1].y));
     }
     m = warp_max(m);
     const float inv = (m == 0.f) ? 0.f : __fdiv_rn(127.f, m);
-    if (lane == 0) scales[row] = (m == 0.f) ? 0.f : __fdiv_rn(m, 127.f);
+    if (lane == 0) scales[r] = (m == 0.f) ? 0.f : __fdiv_rn(m, 127.f);
+    int8_t* crow = codes + r * K;
     for (int p = 0; p < passes; ++p) {
-      const int32_t u = p * 8 + static_cast<int32_t>(lane >> 2);
-      float v[32];
-      if (u < upr) {
-        load32(xr + (u * 128 + q * 32) / 8, v);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = 0.f;
-      }
-      if (hadamard) fwht128(v, q);
-      if (u < upr) {
-        uint32_t w[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          uint32_t packed = 0;
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            int qi = __float2int_rn(__fmul_rn(v[4 * i + b], inv));
-            qi = max(-127, min(127, qi));
-            packed |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * b);
-          }
-          w[i] = packed;
-        }
-        uint4* dst = reinterpret_cast<uint4*>(codes + row * K + u * 128 + q * 32);
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-      }
+      if (passes > 1) load_half(row, p, P);    // one pass: P still holds the rotated half
+      const int32_t hb = 32 * p + static_cast<int32_t>(lane);
+      if (hb < halves) quant_int8_half(P, inv, crow + 64 * hb);
     }
+    __syncwarp();
   }
+  cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
 // Per-tensor INT8 in Q-ARVD channel order.  Output row = Kp bytes; slot j
 // takes input channel gather[j] (or 0 for a padding slot).  The scale comes
 // from the device amax of the un-rotated tensor.
+// One CTA per row at a time: the bf16 row is copied into shared memory with
+// coalesced 16-byte cp.async (the next row's copy is in flight while this
+// one is quantized); each thread takes 4 consecutive slots per step, reads
+// their channels through the gather table (int16 in shared memory) and
+// writes 4 codes as one word of a shared output row, which leaves with
+// 16-byte stores.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreadsHbm)
-    k_quant_int8_tensor_perm(const __nv_bfloat16* __restrict__ x, int64_t M, int32_t K, int32_t Kp,
+struct PermLayout {
+  int32_t gather_bytes, row_bytes, out_bytes, total;
+  __host__ __device__ PermLayout(int32_t K, int32_t Kp)
+      : gather_bytes((Kp * 2 + 15) / 16 * 16), row_bytes(K * 2), out_bytes((Kp + 15) / 16 * 16),
+        total((Kp * 2 + 15) / 16 * 16 + 2 * K * 2 + (Kp + 15) / 16 * 16) {}
+};
+constexpr int kPermThreads = 256;
+
+__global__ void __launch_bounds__(kPermThreads)
+    k_quant_int8_tensor_perm(const uint8_t* __restrict__ x, int64_t M, int32_t K, int32_t Kp,
                              const int32_t* __restrict__ gather, const float* __restrict__ amax_in,
                              int8_t* __restrict__ codes, float* __restrict__ scale_out) {
-  extern __shared__ int32_t s_gather[];
-  for (int i = threadIdx.x; i < Kp; i += blockDim.x) s_gather[i] = gather[i];
+  extern __shared__ __align__(16) uint8_t s_perm[];
+  const PermLayout L(K, Kp);
+  int16_t* s_gather = reinterpret_cast<int16_t*>(s_perm);
+  uint8_t* rows[2] = {s_perm + L.gather_bytes, s_perm + L.gather_bytes + L.row_bytes};
+  uint32_t* orow = reinterpret_cast<uint32_t*>(s_perm + L.gather_bytes + 2 * L.row_bytes);
+  for (int i = threadIdx.x; i < Kp; i += blockDim.x) s_gather[i] = static_cast<int16_t>(gather[i]);
   const float amax = __ldg(amax_in);
   const float inv = (amax == 0.f) ? 0.f : __fdiv_rn(127.f, amax);
   if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = (amax == 0.f) ? 0.f : __fdiv_rn(amax, 127.f);
-  __syncthreads();
-  const uint32_t lane = lane_id();
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const unsigned short* xs = reinterpret_cast<const unsigned short*>(x);
-  for (int64_t row = warp; row < M; row += nwarps) {
-    const unsigned short* xr = xs + row * K;
-    for (int32_t j0 = static_cast<int32_t>(lane) * 16; j0 < Kp; j0 += 32 * 16) {
-      uint32_t w[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint32_t packed = 0;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int32_t src = s_gather[j0 + 4 * i + b];
-          int qi = 0;
-          if (src >= 0) {
-            const float v = __uint_as_float(static_cast<uint32_t>(__ldg(xr + src)) << 16);
-            qi = max(-127, min(127, __float2int_rn(__fmul_rn(v, inv))));
-          }
-          packed |= (static_cast<uint32_t>(qi) & 0xFFu) << (8 * b);
-        }
-        w[i] = packed;
-      }
-      *reinterpret_cast<uint4*>(codes + row * Kp + j0) = make_uint4(w[0], w[1], w[2], w[3]);
+  auto issue_row = [&](int64_t r, uint8_t* dst) {
+    const uint8_t* src = x + r * L.row_bytes;
+    const uint32_t d = smem_u32(dst);
+    for (int32_t o = 16 * static_cast<int32_t>(threadIdx.x); o < L.row_bytes; o += 16 * kPermThreads) {
+      const bool ok = r < M;
+      cp_async16(d + o, ok ? static_cast<const void*>(src + o) : static_cast<const void*>(x), ok ? 16u : 0u);
     }
+  };
+  auto q8 = [&](const unsigned short* xr, int32_t src) -> uint32_t {
+    if (src < 0) return 0u;
+    const float v = __uint_as_float(static_cast<uint32_t>(xr[src]) << 16);
+    return static_cast<uint32_t>(max(-127, min(127, __float2int_rn(__fmul_rn(v, inv))))) & 0xFFu;
+  };
+  issue_row(blockIdx.x, rows[0]);
+  cp_async_commit();
+  int k = 0;
+  for (int64_t r = blockIdx.x; r < M; r += gridDim.x, ++k) {
+    issue_row(r + gridDim.x, rows[(k + 1) & 1]);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();   // this row landed (all threads' copies); gather table ready
+    const unsigned short* xr = reinterpret_cast<const unsigned short*>(rows[k & 1]);
+    for (int32_t w = threadIdx.x; 4 * w < Kp; w += kPermThreads) {
+      const uint2 gi = *reinterpret_cast<const uint2*>(s_gather + 4 * w);   // 4 int16 indices
+      const int32_t g0 = static_cast<int16_t>(gi.x & 0xFFFFu), g1 = static_cast<int16_t>(gi.x >> 16);
+      const int32_t g2 = static_cast<int16_t>(gi.y & 0xFFFFu), g3 = static_cast<int16_t>(gi.y >> 16);
+      orow[w] = q8(xr, g0) | (q8(xr, g1) << 8) | (q8(xr, g2) << 16) | (q8(xr, g3) << 24);
+    }
+    __syncthreads();   // output row complete; the row buffer may be refilled
+    int8_t* dst = codes + r * Kp;
+    for (int32_t o = 16 * static_cast<int32_t>(threadIdx.x); o < Kp; o += 16 * kPermThreads)
+      *reinterpret_cast<uint4*>(dst + o) = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(orow) + o);
   }
+  cp_async_wait<0>();
 }
 
 // --------------------------------------------------------------------------
@@ -492,22 +504,28 @@ ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, 
 ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadamard, void* codes,
                                   float* scales, cudaStream_t st) {
   if (M == 0) return QL_OK;
-  const int grid = hbm_grid(M, kThreadsHbm / 32);
-  k_quant_int8_token<<<grid, kThreadsHbm, 0, st>>>(static_cast<const uint4*>(x), M, K, hadamard,
-                                                   static_cast<int8_t*>(codes), scales);
+  const int64_t per_warp = 4 * static_cast<int64_t>(K);   // two bf16 row buffers
+  const int warps = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kThreadsHbm / 32, (200 * 1024) / per_warp)));
+  if (per_warp > 200 * 1024) return QL_ERR_UNSUPPORTED_SHAPE;
+  const size_t smem = static_cast<size_t>(warps) * per_warp;
+  const int64_t want = (M + warps - 1) / warps;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 2 * num_sms())));
+  if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_int8_token), static_cast<int>(smem))) return QL_ERR_CUDA;
+  k_quant_int8_token<<<grid, 32 * warps, smem, st>>>(static_cast<const uint8_t*>(x), M, K, hadamard,
+                                                     static_cast<int8_t*>(codes), scales);
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int32_t Kp,
                                         const int32_t* gather, const float* amax_in, void* codes,
                                         float* scale_out, cudaStream_t st) {
-  const int grid = M == 0 ? 1 : hbm_grid(M, kThreadsHbm / 32);
-  const size_t smem = static_cast<size_t>(Kp) * sizeof(int32_t);
-  if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_int8_tensor_perm), static_cast<int>(smem)))
-    return QL_ERR_CUDA;
-  k_quant_int8_tensor_perm<<<grid, kThreadsHbm, smem, st>>>(
-      static_cast<const __nv_bfloat16*>(x), M, K, Kp, gather, amax_in, static_cast<int8_t*>(codes),
-      scale_out);
+  const PermLayout L(K, Kp);
+  if (L.total > 200 * 1024) return QL_ERR_UNSUPPORTED_SHAPE;
+  const int per_sm = std::max(1, std::min(4, (220 * 1024) / L.total));
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(M, static_cast<int64_t>(per_sm) * num_sms())));
+  if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_int8_tensor_perm), L.total)) return QL_ERR_CUDA;
+  k_quant_int8_tensor_perm<<<grid, kPermThreads, L.total, st>>>(static_cast<const uint8_t*>(x), M, K, Kp, gather,
+                                                                amax_in, static_cast<int8_t*>(codes), scale_out);
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
