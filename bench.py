@@ -21,6 +21,7 @@ bounded row/column sample of the same four linears per step.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -56,12 +57,14 @@ GEMM_TRAFFIC = {
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--configs", action="store_true",
+                    help="time every kernel of the five workload configurations (one JSON line, not the contract line)")
     ap.add_argument("--profile-case", choices=["quant", "gemm"], default=None,
                     help="run one small standalone case for an ncu capture (prints no JSON)")
     return ap.parse_args()
@@ -138,7 +141,7 @@ def dist_done(world: int):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
     NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -151,12 +154,14 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.dev)],
+                 "-lms", "50", "-i", str(self.dev)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
 
-    def stop(self):
+    def stop(self, t_begin: float | None = None, t_end: float | None = None):
+        """Median SM clock and throttle reasons of the samples whose host
+        timestamp lies in [t_begin, t_end] (all samples when not given)."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -168,8 +173,15 @@ class ClockSampler:
         sm, mx, reasons = [], [], set()
         for line in out.strip().splitlines():
             f = [c.strip() for c in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            if t_begin is not None and ts is not None and not (t_begin <= ts <= t_end):
+                continue
+            f = f[1:]
             try:
                 sm.append(float(f[1]))
                 mx.append(float(f[2]))
@@ -243,79 +255,97 @@ def run_ours(args, rank, world, local):
     qbufs = [ql.qlinear_quantize_act(x, ql.QL_ROUTE_NVFP4, hadamard=True, rowmajor_scales=False)
              for x in xs]
     route_pinned = torch.zeros(1, dtype=torch.int32, pin_memory=True)
-    gamma0, route0 = ql.qlinear_route(bin_d, bout_d, THRESHOLD)
+    gamma_d = torch.empty(1, dtype=torch.float64, device=dev)
+    route_d = torch.empty(1, dtype=torch.int32, device=dev)
+    route_ws = torch.zeros(ql.lib.qlinear_route_ws_bytes(bin_d.numel()), dtype=torch.uint8, device=dev)
+    gamma0, route0 = ql.qlinear_route(bin_d, bout_d, THRESHOLD, gamma=gamma_d, route=route_d, ws=route_ws)
     torch.cuda.synchronize()
     host_route = int(route0.item())
     assert host_route == ql.QL_ROUTE_NVFP4, "the benchmark block must be a stable (NVFP4) block"
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
+    def step():
         # Gamma of this block; the decision is read one step later (Gamma_{t-1})
-        if ev is not None:
-            ev["route"][0].record(stream)
-        g, r = ql.qlinear_route(bin_d, bout_d, THRESHOLD)
-        route_pinned.copy_(r, non_blocking=True)
-        if ev is not None:
-            ev["route"][1].record(stream)
-        for i, (lin, _, _) in enumerate(lins):
-            if ev is not None:
-                ev["amax"][i][0].record(stream)
+        ql.qlinear_route(bin_d, bout_d, THRESHOLD, gamma=gamma_d, route=route_d, ws=route_ws)
+        route_pinned.copy_(route_d, non_blocking=True)
+        for i in range(len(lins)):
             ql.qlinear_tensor_amax(xs[i], True, out=amax[i], ws=amax_ws[i])
-            if ev is not None:
-                ev["quant"][i][0].record(stream)
             ql.qlinear_quantize_act(xs[i], host_route, True, amax_in=amax[i], out=qbufs[i])
-            if ev is not None:
-                ev["gemm"][i][0].record(stream)
             ql.qlinear_gemm(host_route, qbufs[i], M_TOKENS, pws[i], Y=ys[i])
-            if ev is not None:
-                ev["gemm"][i][1].record(stream)
 
-    for _ in range(args.warmup):
+    # Eager warm-up surfaces errors; the timed steps replay the step as one
+    # CUDA graph (13 kernel launches and the route copy, no host gaps).
+    for _ in range(max(1, args.warmup)):
         step()
     torch.cuda.synchronize()
     assert ql.qlinear_device_status() == 0
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
 
     def pair():
         return (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
 
-    evs = [{"route": pair(), "amax": [pair() for _ in lins], "quant": [pair() for _ in lins],
-            "gemm": [pair() for _ in lins]} for _ in range(args.steps)]
     sampler = ClockSampler(local)
     dist_barrier(world)
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)     # let the sampler start before the timed region
     t0, t1 = pair()
+    th0 = time.time()
     t0.record(stream)
-    for k in range(args.steps):
-        step(evs[k])
+    for _ in range(args.steps):
+        graph.replay()
     t1.record(stream)
     torch.cuda.synchronize()
-    clocks = sampler.stop()
+    th1 = time.time()
+    clocks = sampler.stop(th0, th1)
     dist_barrier(world)
     assert ql.qlinear_device_status() == 0
     ms = t0.elapsed_time(t1)
     ms_max = dist_max(ms, world)
+    del graph
 
-    def tot(key, i=None):
-        s = 0.0
-        for e in evs:
-            if key == "route":
-                s += e["route"][0].elapsed_time(e["route"][1])
-            elif key == "amax":
-                s += e["amax"][i][0].elapsed_time(e["quant"][i][0])
-            elif key == "quant":
-                s += e["quant"][i][0].elapsed_time(e["gemm"][i][0])
-            else:
-                s += e["gemm"][i][0].elapsed_time(e["gemm"][i][1])
-        return s / len(evs)
+    # Per-kernel breakdown: each kernel alone, 10 launches per CUDA graph,
+    # CUDA events around `reps` replays (device time per launch, us).
+    def launch_us(fn, reps=20, per_graph=10):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(per_graph):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = pair()
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        del g
+        return 1e3 * a.elapsed_time(b) / (reps * per_graph)
+
+    route_us = launch_us(lambda: ql.qlinear_route(bin_d, bout_d, THRESHOLD, gamma=gamma_d, route=route_d,
+                                                  ws=route_ws))
+    kt = []
+    for i in range(len(lins)):
+        kt.append({
+            "amax": launch_us(lambda i=i: ql.qlinear_tensor_amax(xs[i], True, out=amax[i], ws=amax_ws[i])),
+            "quant": launch_us(lambda i=i: ql.qlinear_quantize_act(xs[i], host_route, True, amax_in=amax[i],
+                                                                   out=qbufs[i])),
+            "gemm": launch_us(lambda i=i: ql.qlinear_gemm(host_route, qbufs[i], M_TOKENS, pws[i], Y=ys[i]))})
+    assert ql.qlinear_device_status() == 0
+
+    def tot(key, i):
+        return kt[i][key] * 1e-3     # ms
 
     per = {}
     for i, (lin, _, _) in enumerate(lins):
         per[lin.name] = {"amax_us": 1e3 * tot("amax", i), "quant_us": 1e3 * tot("quant", i),
                          "gemm_us": 1e3 * tot("gemm", i),
                          "gemm_tflops": 2.0 * M_TOKENS * lin.n * lin.k / (tot("gemm", i) * 1e-3) / 1e12}
-    route_us = 1e3 * tot("route")
     gemm_ms = sum(tot("gemm", i) for i in range(len(lins)))
     quant_ms = sum(tot("quant", i) for i in range(len(lins)))
     amax_ms = sum(tot("amax", i) for i in range(len(lins)))
@@ -346,6 +376,7 @@ def run_ours(args, rank, world, local):
                          "gbs": 4.0 * M_TOKENS * 1920 / (route_us * 1e-6) / 1e9},
         "per_linear": per,
         "gpu_launches": args.steps * (1 + 3 * len(lins)),
+        "timing": "step replayed as one CUDA graph; per-kernel figures from CUDA-graph replays of each kernel alone",
         "clocks": clocks,
         "gemm_source_sha": sha,
     }
@@ -478,9 +509,129 @@ def run_reference(args, rank, world):
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
+# ---------------------------------------------------------------------------
+# --configs: every kernel of the five workload configurations
+# ---------------------------------------------------------------------------
+def run_configs(reps: int = 20):
+    """Device time (CUDA events around CUDA-graph replays of 10 launches,
+    median of `reps` replays) of each kernel of the five configurations,
+    with its roofline fraction: HBM
+    kernels against the measured copy bandwidth, GEMMs against the measured
+    sustained bf16 rate times the nominal ratio of their MMA kind (FP4 4x,
+    INT8 2x, f16 1x)."""
+    from bit_quantized_linear_block_b200 import qlinear as ql
+    dev = torch.device("cuda", 0)
+    peaks, kind = measured_peaks()
+    hbm, bf16 = peaks["hbm_gbs"], peaks["bf16_tflops_sustained"]
+
+    def med(fn, per_graph=10):
+        # Launches replayed from a CUDA graph (no host launch gaps): median
+        # over `reps` replays of the mean time per launch.
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for _ in range(per_graph):
+                fn()
+        graph.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            graph.replay()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3 / per_graph)
+        del graph
+        return statistics.median(ts)
+
+    def hbm_rec(us, nbytes):
+        return {"us": round(us, 2), "gbs": round(nbytes / us / 1e3, 1), "hbm_frac": round(nbytes / us / 1e3 / hbm, 3)}
+
+    def mma_rec(us, m, n, k, ratio):
+        t = 2.0 * m * n * k / us / 1e6
+        return {"us": round(us, 2), "tflops": round(t, 1), "frac": round(t / (bf16 * ratio), 3)}
+
+    out = {"peaks": {"hbm_gbs": hbm, "bf16_tflops_sustained": bf16, "kind": kind}}
+
+    def w4a4_linear(x, w, m, n, k):
+        xd, wd = x.to(dev), w.to(dev)
+        pw = ql.qlinear_prepare_weights(wd, ql.QL_W_NVFP4, hadamard=True)
+        aws = torch.zeros(ql.lib.qlinear_quantize_ws_bytes(m, k, ql.QL_ROUTE_NVFP4), dtype=torch.uint8, device=dev)
+        amax = ql.qlinear_tensor_amax(xd, True, ws=aws)
+        q = ql.qlinear_quantize_act(xd, ql.QL_ROUTE_NVFP4, True, rowmajor_scales=False, amax_in=amax)
+        y = ql.qlinear_gemm(ql.QL_ROUTE_NVFP4, q, m, pw)
+        rec = {"amax": hbm_rec(med(lambda: ql.qlinear_tensor_amax(xd, True, out=amax, ws=aws)), 2.0 * m * k),
+               "quant_nvfp4": hbm_rec(med(lambda: ql.qlinear_quantize_act(xd, ql.QL_ROUTE_NVFP4, True, amax_in=amax,
+                                                                          out=q)), NVFP4_BYTES_PER_ELEM * m * k),
+               "gemm_w4a4": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ROUTE_NVFP4, q, m, pw, Y=y)), m, n, k, 4.0)}
+        return rec
+
+    # 1: single linear [256,1920] x [1920,1920]
+    x, w = S.single_linear(0)
+    out["cfg1_single_linear"] = w4a4_linear(x, w, 256, 1920, 1920)
+    # 2: CogVideoX-2B block linears
+    for lin in S.COGVIDEOX_2B:
+        x, w = S.cogvideox2b_linear(lin)
+        out[f"cfg2_{lin.name}"] = w4a4_linear(x, w, M_TOKENS, lin.n, lin.k)
+    # 3: routing sweep (4 of the 30 blocks for timing) and the INT8-routed FFN-up
+    wd = S.dmpq_ffn_up_weights().to(dev)
+    pw = ql.qlinear_prepare_weights(wd, ql.QL_W_NVFP4, hadamard=True)
+    routes = {}
+    for blk in (0, 1, 2, 3):
+        bi, bo, sigma = S.dmpq_block_pair(blk)
+        bi, bo = bi.to(dev), bo.to(dev)
+        rws = torch.zeros(ql.lib.qlinear_route_ws_bytes(bi.numel()), dtype=torch.uint8, device=dev)
+        g, r = ql.qlinear_route(bi, bo, THRESHOLD, ws=rws)
+        gg, rr = g.clone(), r.clone()
+        us = med(lambda: ql.qlinear_route(bi, bo, THRESHOLD, gamma=gg, route=rr, ws=rws))
+        routes[f"block{blk}"] = dict(hbm_rec(us, 4.0 * M_TOKENS * 1920), sigma=round(sigma, 5),
+                                     gamma=float(g.item()), route=int(r.item()))
+    out["cfg3_route"] = routes
+    q = ql.qlinear_quantize_act(bi, ql.QL_ROUTE_INT8, True)
+    y = ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, M_TOKENS, pw)
+    out["cfg3_int8_ffn_up"] = {
+        "quant_int8_token": hbm_rec(med(lambda: ql.qlinear_quantize_act(bi, ql.QL_ROUTE_INT8, True, out=q)),
+                                    M_TOKENS * 1920 * (3.0 + 4.0 / 1920)),
+        "gemm_w4a8": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, M_TOKENS, pw, Y=y)),
+                             M_TOKENS, 7680, 1920, 1.0)}
+    del bi, bo, q, y, pw, wd
+    # 4: CogVideoX-5B linears, Q-ARVD dual-scale weights, per-tensor INT8
+    for lin in S.COGVIDEOX_5B:
+        x, w = S.cogvideox5b_qarvd_linear(lin)
+        xd, wd = x.to(dev), w.to(dev)
+        pw = ql.qlinear_prepare_weights(wd, ql.QL_W_QARVD_INT4, hadamard=False)
+        kp = pw.desc.Kp
+        aws = torch.zeros(ql.lib.qlinear_quantize_ws_bytes(M_TOKENS, lin.k, ql.QL_ROUTE_NVFP4), dtype=torch.uint8,
+                          device=dev)
+        amax = ql.qlinear_tensor_amax(xd, False, ws=aws)
+        q = ql.qlinear_quantize_act(xd, ql.QL_ACT_INT8_TENSOR, False, w=pw, amax_in=amax)
+        y = ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q, M_TOKENS, pw)
+        out[f"cfg4_{lin.name}"] = {
+            "amax": hbm_rec(med(lambda: ql.qlinear_tensor_amax(xd, False, out=amax, ws=aws)), 2.0 * M_TOKENS * lin.k),
+            "quant_int8_tensor": hbm_rec(med(lambda: ql.qlinear_quantize_act(xd, ql.QL_ACT_INT8_TENSOR, False, w=pw,
+                                                                              amax_in=amax, out=q)),
+                                         M_TOKENS * (2.0 * lin.k + kp)),
+            "gemm_qarvd": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q, M_TOKENS, pw, Y=y)),
+                                  M_TOKENS, lin.n, lin.k, 2.0)}
+        del xd, wd, pw, q, y
+    # 5: Wan-14B linears
+    for lin in S.WAN_14B:
+        x, w = S.wan14b_linear(lin)
+        out[f"cfg5_{lin.name}"] = w4a4_linear(x, w, S.M_WAN, lin.n, lin.k)
+        torch.cuda.empty_cache()
+    out["device_status"] = ql.qlinear_device_status()
+    return out
+
+
 
 def main():
     args = parse()
+    if args.configs:
+        print(json.dumps({"configs": run_configs()}), flush=True)
+        return
     if args.profile_case:
         profile_case(args.profile_case)
         return

@@ -144,14 +144,21 @@ def qlinear_prepare_weights(W: torch.Tensor, fmt: int = QL_W_NVFP4, hadamard: bo
     return pw
 
 
-def qlinear_route(inp: torch.Tensor, out: torch.Tensor, threshold: float = 0.05, stream=None):
-    """Returns device tensors (gamma float64 [1], route int32 [1])."""
+def qlinear_route(inp: torch.Tensor, out: torch.Tensor, threshold: float = 0.05, stream=None,
+                  gamma: torch.Tensor | None = None, route: torch.Tensor | None = None,
+                  ws: torch.Tensor | None = None):
+    """Returns device tensors (gamma float64 [1], route int32 [1]); reuses
+    the given output and workspace tensors (a workspace stays valid across
+    calls on one stream)."""
     assert inp.dtype == torch.bfloat16 and out.dtype == torch.bfloat16
     assert inp.shape == out.shape and inp.is_contiguous() and out.is_contiguous()
     n = inp.numel()
-    gamma = torch.empty(1, dtype=torch.float64, device=inp.device)
-    route = torch.empty(1, dtype=torch.int32, device=inp.device)
-    ws = _bytes(lib.qlinear_route_ws_bytes(n), inp.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float64, device=inp.device)
+    if route is None:
+        route = torch.empty(1, dtype=torch.int32, device=inp.device)
+    if ws is None:
+        ws = _bytes(lib.qlinear_route_ws_bytes(n), inp.device)
     _check("qlinear_route", lib.qlinear_route(_ptr(inp), _ptr(out), n, threshold, _ptr(gamma),
                                               _ptr(route), _ptr(ws), ws.numel(), _stream(stream)))
     return gamma, route
