@@ -579,6 +579,7 @@ def run_configs(reps: int = 20):
     # 3: routing sweep (4 of the 30 blocks for timing) and the INT8-routed FFN-up
     wd = S.dmpq_ffn_up_weights().to(dev)
     pw = ql.qlinear_prepare_weights(wd, ql.QL_W_NVFP4, hadamard=True)
+    pwx = ql.qlinear_prepare_weights(wd, ql.QL_W_NVFP4, hadamard=True, expand_f16=True)
     routes = {}
     for blk in (0, 1, 2, 3):
         bi, bo, sigma = S.dmpq_block_pair(blk)
@@ -591,13 +592,20 @@ def run_configs(reps: int = 20):
                                      gamma=float(g.item()), route=int(r.item()))
     out["cfg3_route"] = routes
     q = ql.qlinear_quantize_act(bi, ql.QL_ROUTE_INT8, True)
+    q16 = ql.qlinear_quantize_act(bi, ql.QL_ACT_INT8_F16, True)
     y = ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, M_TOKENS, pw)
     out["cfg3_int8_ffn_up"] = {
+        # the path qlinear_forward takes with an f16 weight copy: f16-coded INT8 activations
+        "quant_int8_token_f16": hbm_rec(med(lambda: ql.qlinear_quantize_act(bi, ql.QL_ACT_INT8_F16, True, out=q16)),
+                                        M_TOKENS * 1920 * (4.0 + 4.0 / 1920)),
+        "gemm_w4a8": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q16, M_TOKENS, pwx, Y=y)),
+                             M_TOKENS, 7680, 1920, 1.0),
+        # int8 codes, FP4 weights expanded on chip (no f16 weight copy)
         "quant_int8_token": hbm_rec(med(lambda: ql.qlinear_quantize_act(bi, ql.QL_ROUTE_INT8, True, out=q)),
                                     M_TOKENS * 1920 * (3.0 + 4.0 / 1920)),
-        "gemm_w4a8": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, M_TOKENS, pw, Y=y)),
-                             M_TOKENS, 7680, 1920, 1.0)}
-    del bi, bo, q, y, pw, wd
+        "gemm_w4a8_onchip": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, M_TOKENS, pw, Y=y)),
+                                    M_TOKENS, 7680, 1920, 1.0)}
+    del bi, bo, q, q16, y, pw, pwx, wd
     # 4: CogVideoX-5B linears, Q-ARVD dual-scale weights, per-tensor INT8
     for lin in S.COGVIDEOX_5B:
         x, w = S.cogvideox5b_qarvd_linear(lin)

@@ -199,11 +199,14 @@ struct Carver {  // sequential 256-byte aligned sub-buffers of one allocation
   }
 };
 
-size_t forward_act_bytes(int64_t M, int32_t K, int32_t Kp, int32_t fmt) {
+// f16_codes: the INT8 route keeps its codes as f16 values (weights with an
+// f16 copy), 2 bytes per element.
+size_t forward_act_bytes(int64_t M, int32_t K, int32_t Kp, int32_t fmt, bool f16_codes = false) {
   if (fmt == QL_ROUTE_NVFP4)
     return kAmaxWsBytes + 256 + 256 + align256(static_cast<size_t>(M) * K / 2) +
            align256(qlinear_sf_bytes(M, K));
-  if (fmt == QL_ROUTE_INT8) return align256(static_cast<size_t>(M) * K) + align256(4 * static_cast<size_t>(M));
+  if (fmt == QL_ROUTE_INT8)
+    return align256(static_cast<size_t>(M) * K * (f16_codes ? 2 : 1)) + align256(4 * static_cast<size_t>(M));
   return kAmaxWsBytes + 256 + 256 + align256(static_cast<size_t>(M) * Kp);
 }
 
@@ -253,7 +256,8 @@ size_t qlinear_sf_bytes(int64_t rows, int32_t K) {
 size_t qlinear_weights_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg) {
   if (cfg == nullptr || N <= 0 || check_k(K) != QL_OK) return 0;
   const size_t n = N, k = K;
-  if (cfg->fmt == QL_W_NVFP4) return align256(n * k / 2) + align256(qlinear_sf_bytes(N, K)) + 256;
+  if (cfg->fmt == QL_W_NVFP4)
+    return align256(n * k / 2) + align256(qlinear_sf_bytes(N, K)) + 256 + (cfg->expand_f16 ? align256(n * k * 2) : 0);
   if (cfg->fmt == QL_W_QARVD_INT4) {
     const size_t kp = qarvd_kp(K);
     return align256(n * kp / 2) + align256(k) + align256(4 * k) + align256(4 * kp) + 256 +
@@ -275,6 +279,7 @@ ql_status qlinear_prepare_weights(const void* W, int32_t N, int32_t K, const ql_
   if (W == nullptr || cfg == nullptr || wbuf == nullptr || out == nullptr || ws == nullptr)
     return QL_ERR_INVALID_ARG;
   if (cfg->fmt != QL_W_NVFP4 && cfg->fmt != QL_W_QARVD_INT4) return QL_ERR_INVALID_ARG;
+  if (cfg->fmt == QL_W_QARVD_INT4 && cfg->expand_f16 != 0) return QL_ERR_INVALID_ARG;
   QL_TRY(check_k(K));
   if (N <= 0 || N % 16 != 0 || N > (1 << 24)) return QL_ERR_UNSUPPORTED_SHAPE;
   QL_TRY(check_mk(N, K));
@@ -300,6 +305,10 @@ ql_status qlinear_prepare_weights(const void* W, int32_t N, int32_t K, const ql_
     float* amax = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kAmaxWsBytes);
     QL_TRY(launch_amax(W, N, K, w.hadamard, amax, ws, st));
     QL_TRY(launch_quant_nvfp4(W, N, K, w.hadamard, amax, w.codes, w.sf, nullptr, w.gscale, st));
+    if (cfg->expand_f16) {
+      w.w16 = c.take<uint16_t>(static_cast<size_t>(N) * K * 2);
+      QL_TRY(launch_expand_nvfp4_f16(w.codes, w.sf, N, K, w.w16, st));
+    }
   } else {
     w.Kp = qarvd_kp(K);
     w.codes = c.take<uint8_t>(static_cast<size_t>(N) * w.Kp / 2);
@@ -341,7 +350,9 @@ ql_status qlinear_route(const void* in, const void* out, int64_t numel, float th
 // ---------------------------------------------------------------- activations
 size_t qlinear_quantize_ws_bytes(int64_t M, int32_t K, int32_t act_fmt) {
   if (M < 0 || check_k(K) != QL_OK) return 0;
-  if (act_fmt != QL_ROUTE_NVFP4 && act_fmt != QL_ROUTE_INT8 && act_fmt != QL_ACT_INT8_TENSOR) return 0;
+  if (act_fmt != QL_ROUTE_NVFP4 && act_fmt != QL_ROUTE_INT8 && act_fmt != QL_ACT_INT8_TENSOR &&
+      act_fmt != QL_ACT_INT8_F16)
+    return 0;
   return kAmaxWsBytes + 256;
 }
 
@@ -371,7 +382,7 @@ ql_status qlinear_quantize_act(const void* X, int64_t M, int32_t K, int32_t act_
   } else if (act_fmt == QL_ACT_INT8_TENSOR) {
     QL_TRY(check_w(w));
     if (w->fmt != QL_W_QARVD_INT4 || w->K != K || hadamard != 0) return QL_ERR_INVALID_ARG;
-  } else if (act_fmt != QL_ROUTE_INT8) {
+  } else if (act_fmt != QL_ROUTE_INT8 && act_fmt != QL_ACT_INT8_F16) {
     return QL_ERR_INVALID_ARG;
   }
   if (!aligned(X, 16) || !aligned(codes, 16) || !aligned(sf_mma, 16) || !aligned(sf_rowmajor, 16) ||
@@ -382,6 +393,7 @@ ql_status qlinear_quantize_act(const void* X, int64_t M, int32_t K, int32_t act_
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int had = hadamard ? 1 : 0;
   if (act_fmt == QL_ROUTE_INT8) return launch_quant_int8_token(X, M, K, had, codes, scales, st);
+  if (act_fmt == QL_ACT_INT8_F16) return launch_quant_int8_token(X, M, K, had, codes, scales, st, 1);
   const float* amax = amax_in;
   if (amax == nullptr) {
     float* slot = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kAmaxWsBytes);
@@ -399,8 +411,9 @@ ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf, c
   QL_TRY(check_m(M));
   QL_TRY(check_w(w));
   if (M > 0 && (a_codes == nullptr || a_scales == nullptr || Y == nullptr)) return QL_ERR_INVALID_ARG;
-  if (act_fmt == QL_ROUTE_NVFP4 || act_fmt == QL_ROUTE_INT8) {
+  if (act_fmt == QL_ROUTE_NVFP4 || act_fmt == QL_ROUTE_INT8 || act_fmt == QL_ACT_INT8_F16) {
     if (w->fmt != QL_W_NVFP4) return QL_ERR_INVALID_ARG;
+    if (act_fmt == QL_ACT_INT8_F16 && w->w16 == nullptr) return QL_ERR_INVALID_ARG;
     if (act_fmt == QL_ROUTE_NVFP4 && M > 0 && a_sf == nullptr) return QL_ERR_INVALID_ARG;
   } else if (act_fmt == QL_ACT_INT8_TENSOR) {
     if (w->fmt != QL_W_QARVD_INT4) return QL_ERR_INVALID_ARG;
@@ -416,6 +429,7 @@ ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf, c
   if (act_fmt == QL_ROUTE_NVFP4)
     return launch_gemm_w4a4(a_codes, static_cast<const uint8_t*>(a_sf), a_scales, M, w, Y, st, status);
   if (act_fmt == QL_ROUTE_INT8) return launch_gemm_w4a8(a_codes, a_scales, M, w, Y, st, status);
+  if (act_fmt == QL_ACT_INT8_F16) return launch_gemm_w4a8(a_codes, a_scales, M, w, Y, st, status, 1);
   return launch_gemm_qarvd(a_codes, a_scales, M, w, Y, st, status);
 }
 
@@ -424,7 +438,7 @@ size_t qlinear_forward_ws_bytes(int64_t M, const ql_weights* w, int32_t route) {
   if (M < 0 || check_w(w) != QL_OK) return 0;
   if (w->fmt == QL_W_QARVD_INT4) return forward_act_bytes(M, w->K, w->Kp, QL_ACT_INT8_TENSOR);
   if (route != QL_ROUTE_NVFP4 && route != QL_ROUTE_INT8) return 0;
-  return forward_act_bytes(M, w->K, 0, route);
+  return forward_act_bytes(M, w->K, 0, route, w->w16 != nullptr);
 }
 
 ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t route, void* Y,
@@ -454,10 +468,13 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
     return launch_gemm_w4a4(codes, sf, g, M, w, Y, st, status);
   }
   if (fmt == QL_ROUTE_INT8) {
-    int8_t* codes = c.take<int8_t>(static_cast<size_t>(M) * K);
+    // with an f16 weight copy the codes are written as f16 values and both
+    // GEMM operands go straight from TMA to the MMA
+    const int f16 = w->w16 != nullptr ? 1 : 0;
+    uint8_t* codes = c.take<uint8_t>(static_cast<size_t>(M) * K * (f16 ? 2 : 1));
     float* s = c.take<float>(4 * static_cast<size_t>(M));
-    QL_TRY(launch_quant_int8_token(X, M, K, w->hadamard, codes, s, st));
-    return launch_gemm_w4a8(codes, s, M, w, Y, st, status);
+    QL_TRY(launch_quant_int8_token(X, M, K, w->hadamard, codes, s, st, f16));
+    return launch_gemm_w4a8(codes, s, M, w, Y, st, status, f16);
   }
   void* aws = c.take<uint8_t>(kAmaxWsBytes);
   float* amax = c.take<float>(256);

@@ -26,24 +26,26 @@
 
 namespace ql {
 
-template <int BN, int S>
+template <int BN, int S, int RS, bool PRE, bool A16>
 struct W4A8Cfg {
+  static_assert(!A16 || PRE, "f16 activations need pre-expanded weights");
+  static constexpr bool XFORM = !(PRE && A16);   // any operand expanded on chip
   static constexpr int BM = 128;
   static constexpr int BK = 64;                        // K elements per stage
-  static constexpr int CONV_A = BM * BK * 2;           // f16, 128-byte rows
-  static constexpr int CONV_B = BN * BK * 2;
-  static constexpr int RAW_A = BM * BK;                // int8
-  static constexpr int RAW_B = BN * BK / 2;            // FP4
+  static constexpr int CONV_A = A16 ? 0 : BM * BK * 2;    // f16, 128-byte rows
+  static constexpr int CONV_B = PRE ? 0 : BN * BK * 2;
+  static constexpr int RAW_A = A16 ? BM * BK * 2 : BM * BK;   // f16 (128-byte swizzle) or int8
+  static constexpr int RAW_B = PRE ? BN * BK * 2 : BN * BK / 2;   // f16 (pre-expanded) or FP4
   static constexpr int NSFB = (BN + 127) / 128;
-  static constexpr int RAW_SF = NSFB * 512;            // one 4-scale column of each atom
+  static constexpr int RAW_SF = PRE ? 0 : NSFB * 512;   // one 4-scale column of each atom
   static constexpr int OFF_CA = 0;
   static constexpr int OFF_CB = OFF_CA + S * CONV_A;
   static constexpr int OFF_C = OFF_CB + S * CONV_B;
   static constexpr int OFF_RA = OFF_C + 2 * kEpiChunkBytes;
-  static constexpr int OFF_RB = OFF_RA + S * RAW_A;
-  static constexpr int OFF_RSF = OFF_RB + S * RAW_B;
-  static constexpr int OFF_BAR = OFF_RSF + S * RAW_SF;
-  static constexpr int NBAR = 4 * S + 2 * 2 + 1;
+  static constexpr int OFF_RB = OFF_RA + RS * RAW_A;
+  static constexpr int OFF_RSF = OFF_RB + RS * RAW_B;
+  static constexpr int OFF_BAR = OFF_RSF + RS * RAW_SF;
+  static constexpr int NBAR = 2 * RS + 2 * S + 2 * 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
   static constexpr int THREADS = 512;
@@ -70,34 +72,6 @@ __device__ __forceinline__ void i8x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& 
   hi = *reinterpret_cast<const uint32_t*>(&rb);
 }
 
-// Eight E2M1 codes (byte j: elements 2j low nibble, 2j+1 high nibble) times
-// an E4M3 block scale -> four f16x2 words (exact products).
-__device__ __forceinline__ uint4 fp4x8_scaled_to_f16(uint32_t codes, uint32_t sb) {
-  uint32_t h0, h1, h2, h3, s2;
-  const uint16_t sbb = static_cast<uint16_t>(sb | (sb << 8));
-  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
-      "mov.b32 {c0, c1, c2, c3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, c0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, c1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, c2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, c3;\n\t}"
-      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
-      : "r"(codes));
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(sbb));
-  const __half2 s = *reinterpret_cast<const __half2*>(&s2);
-  uint4 r;
-  __half2 t;
-  t = __hmul2(*reinterpret_cast<const __half2*>(&h0), s);
-  r.x = *reinterpret_cast<const uint32_t*>(&t);
-  t = __hmul2(*reinterpret_cast<const __half2*>(&h1), s);
-  r.y = *reinterpret_cast<const uint32_t*>(&t);
-  t = __hmul2(*reinterpret_cast<const __half2*>(&h2), s);
-  r.z = *reinterpret_cast<const uint32_t*>(&t);
-  t = __hmul2(*reinterpret_cast<const __half2*>(&h3), s);
-  r.w = *reinterpret_cast<const uint32_t*>(&t);
-  return r;
-}
-
 // Position of 16-byte chunk c of row r in a 128-byte-swizzled K-major tile.
 __device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t c) {
   return r * 128u + ((c ^ (r & 7u)) << 4);
@@ -112,16 +86,16 @@ __device__ __forceinline__ bool warp_wait2(uint64_t* a, uint32_t pa, uint64_t* b
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-template <int BN, int S>
+template <int BN, int S, int RS, bool PRE, bool A16>
 __global__ void __launch_bounds__(512, 1)
     k_gemm_w4a8(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
-  using C = W4A8Cfg<BN, S>;
+  using C = W4A8Cfg<BN, S, RS, PRE, A16>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* raw_empty = raw_full + S;
-  uint64_t* conv_full = raw_empty + S;
+  uint64_t* raw_empty = raw_full + RS;
+  uint64_t* conv_full = raw_empty + RS;
   uint64_t* conv_empty = conv_full + S;
   uint64_t* tfull = conv_empty + S;
   uint64_t* tempty = tfull + 2;
@@ -134,9 +108,13 @@ __global__ void __launch_bounds__(512, 1)
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_b);
     prefetch_tmap(&tm_y);
-    for (int i = 0; i < S; ++i) {
+    for (int i = 0; i < RS; ++i) {
       mbar_init(&raw_full[i], 1);
-      mbar_init(&raw_empty[i], C::XFORM_THREADS / 32);
+      // consumers of a raw stage: the transform warps (when they expand an
+      // operand) and, when B is read in place, the MMAs' commit
+      mbar_init(&raw_empty[i], (C::XFORM ? C::XFORM_THREADS / 32 : 0) + (PRE ? 1 : 0));
+    }
+    for (int i = 0; i < S; ++i) {
       mbar_init(&conv_full[i], C::XFORM_THREADS / 32);
       mbar_init(&conv_empty[i], 1);
     }
@@ -154,7 +132,7 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 8) {
+  if (warp < 8 && C::XFORM) {
     // ------------------------------------------------------------ transform
     const uint32_t tid = threadIdx.x;
     int it = 0;
@@ -165,17 +143,18 @@ __global__ void __launch_bounds__(512, 1)
       const int n0 = nb * BN;
       const int ra0 = n0 >> 7;
       for (int ks = 0; ks < p.num_kst; ++ks, ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
-        if (!warp_wait2(&raw_full[s], ph, &conv_empty[s], ph ^ 1, p.wait_limit, abort_flag)) {
+        const int s = it % S, rs = it % RS;
+        if (!warp_wait2(&raw_full[rs], (it / RS) & 1, &conv_empty[s], ((it / S) & 1) ^ 1, p.wait_limit,
+                        abort_flag)) {
           ok = false;
           break;
         }
-        const uint8_t* ra = smem + C::OFF_RA + s * C::RAW_A;
-        const uint8_t* rb = smem + C::OFF_RB + s * C::RAW_B;
-        const uint8_t* rsf = smem + C::OFF_RSF + s * C::RAW_SF;
+        const uint8_t* ra = smem + C::OFF_RA + rs * C::RAW_A;
+        const uint8_t* rb = smem + C::OFF_RB + rs * C::RAW_B;
+        const uint8_t* rsf = smem + C::OFF_RSF + rs * C::RAW_SF;
         uint8_t* ca = smem + C::OFF_CA + s * C::CONV_A;
         uint8_t* cb = smem + C::OFF_CB + s * C::CONV_B;
+        if constexpr (!A16)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {            // A: 128 rows x 8 chunks of 8 int8
           const uint32_t idx = tid + C::XFORM_THREADS * i;
@@ -186,6 +165,7 @@ __global__ void __launch_bounds__(512, 1)
           i8x4_to_f16(q.y, o.z, o.w);
           *reinterpret_cast<uint4*>(ca + sw128(r, c)) = o;
         }
+        if constexpr (!PRE)
 #pragma unroll
         for (int i = 0; i < C::B_CHUNKS_PER_THREAD; ++i) {   // B: BN rows x 8 chunks of 8 FP4
           const uint32_t idx = tid + C::XFORM_THREADS * i;
@@ -199,7 +179,7 @@ __global__ void __launch_bounds__(512, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane_id() == 0) {
-          mbar_arrive(&raw_empty[s]);
+          mbar_arrive(&raw_empty[rs]);
           mbar_arrive(&conv_full[s]);
         }
       }
@@ -216,8 +196,8 @@ __global__ void __launch_bounds__(512, 1)
         const int n0 = nb * BN;
         const int ra0 = n0 >> 7;
         for (int ks = 0; ks < p.num_kst; ++ks, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
+          const int s = it % RS;
+          const uint32_t ph = (it / RS) & 1;
           if (*abort_flag || !mbar_wait(&raw_empty[s], ph ^ 1, p.wait_limit)) {
             ok = false;
             break;
@@ -225,11 +205,12 @@ __global__ void __launch_bounds__(512, 1)
           int nsfb = 0;
 #pragma unroll
           for (int r = 0; r < C::NSFB; ++r) nsfb += (ra0 + r < p.sfb_atoms);
+          if (PRE) nsfb = 0;
           mbar_arrive_expect_tx(&raw_full[s], C::RAW_A + C::RAW_B + 512 * nsfb);
           tma_load_2d(smem + C::OFF_RA + s * C::RAW_A, &tm_a, &raw_full[s], ks * C::BK, mb * C::BM);
-          tma_load_2d(smem + C::OFF_RB + s * C::RAW_B, &tm_b, &raw_full[s], ks * (C::BK / 2), n0);
+          tma_load_2d(smem + C::OFF_RB + s * C::RAW_B, &tm_b, &raw_full[s], ks * (PRE ? C::BK : C::BK / 2), n0);
 #pragma unroll
-          for (int r = 0; r < C::NSFB; ++r) {
+          for (int r = 0; r < (PRE ? 0 : C::NSFB); ++r) {
             if (ra0 + r < p.sfb_atoms)
               bulk_load(smem + C::OFF_RSF + s * C::RAW_SF + r * 512,
                         p.sfb + (static_cast<size_t>(ra0 + r) * p.k_atoms + ks) * 512, 512, &raw_full[s]);
@@ -237,7 +218,7 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
       if (!ok) fail_timeout(p.status, abort_flag);
-      drain_loads(raw_full, it, S, p.status);
+      drain_loads(raw_full, it, RS, p.status);
     }
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
@@ -254,22 +235,28 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem + acc * BN;
         for (int ks = 0; ks < p.num_kst; ++ks, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
-          if (*abort_flag || !mbar_wait(&conv_full[s], ph, p.wait_limit)) {
+          const int s = it % S, rs = it % RS;
+          // expanded operands wait for the transform; operands read in place
+          // (both, with A16 and PRE) wait for the raw tiles
+          const bool ready = C::XFORM ? mbar_wait(&conv_full[s], (it / S) & 1, p.wait_limit)
+                                      : mbar_wait(&raw_full[rs], (it / RS) & 1, p.wait_limit);
+          if (*abort_flag || !ready) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + C::OFF_CA + s * C::CONV_A);
-          const uint32_t b_base = smem_u32(smem + C::OFF_CB + s * C::CONV_B);
+          const uint32_t a_base = A16 ? smem_u32(smem + C::OFF_RA + rs * C::RAW_A)
+                                      : smem_u32(smem + C::OFF_CA + s * C::CONV_A);
+          const uint32_t b_base = PRE ? smem_u32(smem + C::OFF_RB + rs * C::RAW_B)
+                                      : smem_u32(smem + C::OFF_CB + s * C::CONV_B);
 #pragma unroll
           for (int i = 0; i < C::BK / 16; ++i) {
             const uint64_t adesc = smem_desc(a_base + 32 * i, 0, 1024, kSwizzle128B);
             const uint64_t bdesc = smem_desc(b_base + 32 * i, 0, 1024, kSwizzle128B);
             tc_mma_f16(d_tmem, adesc, bdesc, C::IDESC, (ks > 0 || i > 0) ? 1u : 0u);
           }
-          tc_commit(&conv_empty[s]);
+          if constexpr (C::XFORM) tc_commit(&conv_empty[s]);
+          if constexpr (PRE) tc_commit(&raw_empty[rs]);   // the in-place tiles are consumed
         }
         if (!ok) break;
         tc_commit(&tfull[acc]);
@@ -301,16 +288,20 @@ __global__ void __launch_bounds__(512, 1)
   if (warp == 10) tmem_dealloc(tmem, 512);
 }
 
-template <int BN, int S>
+template <int BN, int S, int RS, bool PRE, bool A16>
 static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int64_t M,
                                  const ql_weights* w, void* Y, cudaStream_t st, int* status) {
-  using C = W4A8Cfg<BN, S>;
+  using C = W4A8Cfg<BN, S, RS, PRE, A16>;
   const int N = w->N, K = w->K;
   CUtensorMap ta, tb, ty;
-  if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K, M, K, C::BK, C::BM,
-                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, C::BK / 2, BN,
-                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+  if (!(A16 ? make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a_codes, K, M, static_cast<int64_t>(K) * 2, C::BK,
+                           C::BM, CU_TENSOR_MAP_SWIZZLE_128B)
+             : make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K, M, K, C::BK, C::BM,
+                            CU_TENSOR_MAP_SWIZZLE_NONE)) ||
+      !(PRE ? make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w->w16, K, N, static_cast<int64_t>(K) * 2, C::BK,
+                           BN, CU_TENSOR_MAP_SWIZZLE_128B)
+            : make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, C::BK / 2, BN,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) ||
       !make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<int64_t>(N) * 2, 64,
                     128, CU_TENSOR_MAP_SWIZZLE_128B))
     return QL_ERR_CUDA;
@@ -323,7 +314,7 @@ static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int
   p.g_w = w->gscale;
   p.row_scale = a_scales;
   p.alpha_mul = w->hadamard ? (1.0f / 128.0f) : 1.0f;
-  auto kern = k_gemm_w4a8<BN, S>;
+  auto kern = k_gemm_w4a8<BN, S, RS, PRE, A16>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int grid = std::min(p.num_tiles, num_sms());
   kern<<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, ty, p);
@@ -331,10 +322,20 @@ static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int
 }
 
 ql_status launch_gemm_w4a8(const void* a_codes, const float* a_scales, int64_t M, const ql_weights* w,
-                           void* Y, cudaStream_t st, int* status) {
+                           void* Y, cudaStream_t st, int* status, int a_f16) {
   if (M == 0) return QL_OK;
-  if (w->N % 192 == 0) return launch_w4a8_cfg<192, 3>(a_codes, a_scales, M, w, Y, st, status);
-  return launch_w4a8_cfg<128, 4>(a_codes, a_scales, M, w, Y, st, status);
+  const bool n192 = w->N % 192 == 0;
+  if (a_f16) {   // f16 activations and pre-expanded weights: both operands by TMA
+    if (w->w16 == nullptr) return QL_ERR_UNSUPPORTED_SHAPE;
+    if (n192) return launch_w4a8_cfg<192, 1, 4, true, true>(a_codes, a_scales, M, w, Y, st, status);
+    return launch_w4a8_cfg<128, 1, 5, true, true>(a_codes, a_scales, M, w, Y, st, status);
+  }
+  if (w->w16 != nullptr) {   // weights pre-expanded to f16 at preparation
+    if (n192) return launch_w4a8_cfg<192, 2, 4, true, false>(a_codes, a_scales, M, w, Y, st, status);
+    return launch_w4a8_cfg<128, 2, 5, true, false>(a_codes, a_scales, M, w, Y, st, status);
+  }
+  if (n192) return launch_w4a8_cfg<192, 2, 6, false, false>(a_codes, a_scales, M, w, Y, st, status);
+  return launch_w4a8_cfg<128, 2, 8, false, false>(a_codes, a_scales, M, w, Y, st, status);
 }
 
 }  // namespace ql

@@ -27,8 +27,12 @@ ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* 
                       cudaStream_t st);
 ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, const float* amax_in,
                              void* codes, void* sf_mma, void* sf_rm, float* g_out, cudaStream_t st);
+// f16 copy [N, K] of NVFP4 weights without the tensor scale (INT8 route).
+ql_status launch_expand_nvfp4_f16(const void* codes, const void* sf, int32_t N, int32_t K, void* out,
+                                  cudaStream_t st);
+// f16_codes = 1 writes each INT8 code as the equal f16 value ([M, K] f16).
 ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadamard, void* codes,
-                                  float* scales, cudaStream_t st);
+                                  float* scales, cudaStream_t st, int f16_codes = 0);
 ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int32_t Kp,
                                         const int32_t* gather, const float* amax_in, void* codes,
                                         float* scale_out, cudaStream_t st);
@@ -39,8 +43,10 @@ ql_status launch_qarvd_prepare(const void* W, int32_t N, int32_t K, float tau, f
 
 ql_status launch_gemm_w4a4(const void* a_codes, const uint8_t* a_sf, const float* g_a, int64_t M,
                            const ql_weights* w, void* Y, cudaStream_t st, int* status);
+// a_f16 = 1: activations are f16 [M, K] holding the INT8 codes (needs
+// weights prepared with expand_f16).
 ql_status launch_gemm_w4a8(const void* a_codes, const float* a_scales, int64_t M,
-                           const ql_weights* w, void* Y, cudaStream_t st, int* status);
+                           const ql_weights* w, void* Y, cudaStream_t st, int* status, int a_f16 = 0);
 ql_status launch_gemm_qarvd(const void* a_codes, const float* s_x, int64_t M, const ql_weights* w,
                             void* Y, cudaStream_t st, int* status);
 

@@ -10,6 +10,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include "../../include/qlinear.h"
@@ -338,6 +339,34 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// Eight E2M1 codes (byte j: elements 2j low nibble, 2j+1 high nibble) times
+// an E4M3 block scale -> four f16x2 words (exact products).
+__device__ __forceinline__ uint4 fp4x8_scaled_to_f16(uint32_t codes, uint32_t sb) {
+  uint32_t h0, h1, h2, h3, s2;
+  const uint16_t sbb = static_cast<uint16_t>(sb | (sb << 8));
+  asm("{\n\t.reg .b8 c0, c1, c2, c3;\n\t"
+      "mov.b32 {c0, c1, c2, c3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, c0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, c1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, c2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, c3;\n\t}"
+      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+      : "r"(codes));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(s2) : "h"(sbb));
+  const __half2 s = *reinterpret_cast<const __half2*>(&s2);
+  uint4 r;
+  __half2 t;
+  t = __hmul2(*reinterpret_cast<const __half2*>(&h0), s);
+  r.x = *reinterpret_cast<const uint32_t*>(&t);
+  t = __hmul2(*reinterpret_cast<const __half2*>(&h1), s);
+  r.y = *reinterpret_cast<const uint32_t*>(&t);
+  t = __hmul2(*reinterpret_cast<const __half2*>(&h2), s);
+  r.z = *reinterpret_cast<const uint32_t*>(&t);
+  t = __hmul2(*reinterpret_cast<const __half2*>(&h3), s);
+  r.w = *reinterpret_cast<const uint32_t*>(&t);
+  return r;
+}
 
 // Offset of block-scale j of row r in the MMA layout (512-byte atoms).
 __device__ __forceinline__ size_t sf_mma_offset(int64_t r, int32_t j, int32_t k_atoms) {

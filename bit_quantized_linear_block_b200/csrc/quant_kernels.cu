@@ -308,7 +308,28 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
 // A row of at most 2048 elements is rotated once and stays in registers;
 // longer rows are rotated again, from shared memory, for the second pass.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv, int8_t* dst) {
+// F16 = true writes each code as the equal f16 value (an integer in
+// [-127, 127], exact), the operand layout of the f16 MMA.
+template <bool F16>
+__device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv, uint8_t* dst) {
+  if constexpr (F16) {
+    uint32_t w[32];   // element pairs (4i+b) and (32+4i+b) -> f16 words
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int ql0 = max(-127, min(127, __float2int_rn(__fmul_rn(P[2 * i].x, inv))));
+      const int ql1 = max(-127, min(127, __float2int_rn(__fmul_rn(P[2 * i + 1].x, inv))));
+      const int qh0 = max(-127, min(127, __float2int_rn(__fmul_rn(P[2 * i].y, inv))));
+      const int qh1 = max(-127, min(127, __float2int_rn(__fmul_rn(P[2 * i + 1].y, inv))));
+      const __half2 lo = __halves2half2(__int2half_rn(ql0), __int2half_rn(ql1));
+      const __half2 hi = __halves2half2(__int2half_rn(qh0), __int2half_rn(qh1));
+      w[i] = *reinterpret_cast<const uint32_t*>(&lo);          // elements 2i, 2i+1
+      w[16 + i] = *reinterpret_cast<const uint32_t*>(&hi);     // elements 32+2i, 32+2i+1
+    }
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    return;
+  }
   uint32_t w[16];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {   // elements 4i..4i+3 (.x halves) and 32+4i.. (.y halves)
@@ -328,9 +349,10 @@ __device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv
   for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
+template <bool F16>
 __global__ void __launch_bounds__(kThreadsHbm)
     k_quant_int8_token(const uint8_t* __restrict__ x, int64_t M, int32_t K, int hadamard,
-                       int8_t* __restrict__ codes, float* __restrict__ scales) {
+                       uint8_t* __restrict__ codes, float* __restrict__ scales) {
   extern __shared__ __align__(128) uint8_t s_rows[];
   const uint32_t lane = lane_id();
   const int wid = threadIdx.x >> 5;
@@ -379,11 +401,12 @@ __global__ void __launch_bounds__(kThreadsHbm)
     m = warp_max(m);
     const float inv = (m == 0.f) ? 0.f : __fdiv_rn(127.f, m);
     if (lane == 0) scales[r] = (m == 0.f) ? 0.f : __fdiv_rn(m, 127.f);
-    int8_t* crow = codes + r * K;
+    constexpr int kElemBytes = F16 ? 2 : 1;
+    uint8_t* crow = codes + r * K * kElemBytes;
     for (int p = 0; p < passes; ++p) {
       if (passes > 1) load_half(row, p, P);    // one pass: P still holds the rotated half
       const int32_t hb = 32 * p + static_cast<int32_t>(lane);
-      if (hb < halves) quant_int8_half(P, inv, crow + 64 * hb);
+      if (hb < halves) quant_int8_half<F16>(P, inv, crow + 64 * kElemBytes * hb);
     }
     __syncwarp();
   }
@@ -458,6 +481,26 @@ __global__ void __launch_bounds__(kPermThreads)
   cp_async_wait<0>();
 }
 
+// ---------------------------------------------------------------------------
+// f16 expansion of NVFP4 weights for the INT8 route's GEMM: out[n, k] =
+// e2m1(code[n, k]) * e4m3(sb[n, k/16]) (without the tensor scale), exact in
+// f16 (at most 6 significant bits, magnitudes 2^-10 .. 2688).  A thread
+// expands 8 consecutive codes (one 32-bit word, half a scale block).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreadsHbm)
+    k_expand_nvfp4_f16(const uint32_t* __restrict__ codes, const uint8_t* __restrict__ sf, int32_t N, int32_t K,
+                       uint4* __restrict__ out) {
+  const int64_t words = static_cast<int64_t>(N) * (K / 8);
+  const int32_t wpr = K / 8, k_atoms = K / 64;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < words;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / wpr;
+    const int32_t c8 = static_cast<int32_t>(i - n * wpr);
+    const uint32_t sb = sf[sf_mma_offset(n, c8 >> 1, k_atoms)];
+    out[i] = fp4x8_scaled_to_f16(__ldg(codes + i), sb);
+  }
+}
+
 // --------------------------------------------------------------------------
 // Host launchers
 // --------------------------------------------------------------------------
@@ -501,8 +544,16 @@ ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, 
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
+ql_status launch_expand_nvfp4_f16(const void* codes, const void* sf, int32_t N, int32_t K, void* out,
+                                  cudaStream_t st) {
+  const int grid = hbm_grid(static_cast<int64_t>(N) * (K / 8), kThreadsHbm);
+  k_expand_nvfp4_f16<<<grid, kThreadsHbm, 0, st>>>(static_cast<const uint32_t*>(codes),
+                                                   static_cast<const uint8_t*>(sf), N, K, static_cast<uint4*>(out));
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
 ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadamard, void* codes,
-                                  float* scales, cudaStream_t st) {
+                                  float* scales, cudaStream_t st, int f16_codes) {
   if (M == 0) return QL_OK;
   const int64_t per_warp = 4 * static_cast<int64_t>(K);   // two bf16 row buffers
   const int warps = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kThreadsHbm / 32, (200 * 1024) / per_warp)));
@@ -510,9 +561,10 @@ ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadam
   const size_t smem = static_cast<size_t>(warps) * per_warp;
   const int64_t want = (M + warps - 1) / warps;
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 2 * num_sms())));
-  if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_int8_token), static_cast<int>(smem))) return QL_ERR_CUDA;
-  k_quant_int8_token<<<grid, 32 * warps, smem, st>>>(static_cast<const uint8_t*>(x), M, K, hadamard,
-                                                     static_cast<int8_t*>(codes), scales);
+  auto kern = f16_codes ? k_quant_int8_token<true> : k_quant_int8_token<false>;
+  if (!set_smem_attr(reinterpret_cast<const void*>(kern), static_cast<int>(smem))) return QL_ERR_CUDA;
+  kern<<<grid, 32 * warps, smem, st>>>(static_cast<const uint8_t*>(x), M, K, hadamard,
+                                       static_cast<uint8_t*>(codes), scales);
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 

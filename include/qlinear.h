@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define QLINEAR_ABI_VERSION 1
+#define QLINEAR_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define QL_API __attribute__((visibility("default")))
@@ -89,7 +89,10 @@ typedef enum {
 typedef enum {
   QL_ROUTE_NVFP4 = 0,       /* W4A4: NVFP4 activations                       */
   QL_ROUTE_INT8 = 1,        /* W4A8: per-token INT8 activations              */
-  QL_ACT_INT8_TENSOR = 2    /* Q-ARVD: per-tensor INT8, permuted K           */
+  QL_ACT_INT8_TENSOR = 2,   /* Q-ARVD: per-tensor INT8, permuted K           */
+  QL_ACT_INT8_F16 = 3       /* W4A8: per-token INT8 codes stored as the equal
+                               f16 values, f16 [M, K]; the GEMM needs weights
+                               prepared with expand_f16                      */
 } ql_act_format;
 
 typedef struct {
@@ -98,6 +101,12 @@ typedef struct {
                         activations' setting); Q-ARVD: must be 0              */
   float tau;         /* Q-ARVD modified z-score threshold (3.5)                */
   float alpha;       /* Q-ARVD minimum magnitude factor (2.0)                  */
+  int32_t expand_f16;/* NVFP4: 1 = also keep an f16 copy of the dequantized
+                        weights (E2M1 x E4M3, without g_w; exact in f16) for
+                        the INT8 route's GEMM, which then reads it directly
+                        instead of expanding the FP4 codes on chip.  Costs
+                        2 bytes per weight in the weight buffer.              */
+  int32_t reserved;  /* 0                                                      */
 } ql_weight_cfg;
 
 /* Packed weights.  Filled by qlinear_prepare_weights(); every pointer points
@@ -116,6 +125,8 @@ typedef struct {
   float* s_norm;         /* Q-ARVD [N] scale of the normal channels             */
   float* s_out;          /* Q-ARVD [N] scale of the outlier channels            */
   double* norms;         /* Q-ARVD [K] input-channel L2 norms                   */
+  void* w16;             /* NVFP4 with expand_f16: f16 [N, K] = E2M1 x E4M3
+                            (no g_w); NULL otherwise                            */
 } ql_weights;
 
 /* ---- library ------------------------------------------------------------ */
@@ -198,6 +209,7 @@ QL_API ql_status qlinear_tensor_amax(const void* X_bf16, int64_t M, int32_t K, i
                        sf_rowmajor [M, K/16] (optional, may be NULL);
                        scales = fp32[1] tensor scale g_x.
    QL_ROUTE_INT8:      codes int8 [M, K]; scales = fp32 [M]; sf_* unused.
+   QL_ACT_INT8_F16:    as QL_ROUTE_INT8, codes f16 [M, K] (exact integers).
    QL_ACT_INT8_TENSOR: needs Q-ARVD weights `w`; codes int8 [M, w->Kp] in the
                        weights' channel order with zero padding; scales =
                        fp32[1]; hadamard must be 0.
@@ -216,8 +228,11 @@ QL_API ql_status qlinear_quantize_act(const void* X_bf16, int64_t M, int32_t K,
    Y[m, n] = bf16(alpha_m * sum_k a[m,k] w[n,k]) with fp32 accumulation:
    QL_ROUTE_NVFP4:     tcgen05 block-scaled FP4 MMA; alpha = g_x g_w / 128 if
                        the weights are rotated, else g_x g_w.
-   QL_ROUTE_INT8:      INT8 x NVFP4 weights expanded on chip to bf16;
+   QL_ROUTE_INT8:      INT8 x NVFP4 weights (their f16 copy when prepared with
+                       expand_f16, else expanded on chip to f16);
                        alpha_m = s_m g_w (/128 if rotated).
+   QL_ACT_INT8_F16:    as QL_ROUTE_INT8 with f16 codes; needs the f16 copy;
+                       both operands go straight to the f16 MMA.
    QL_ACT_INT8_TENSOR: INT8 x INT4 integer MMA, two class accumulators;
                        y = s_x (s_norm[n] acc_normal + s_out[n] acc_outlier).
    Operands are the outputs of qlinear_quantize_act for the same format. */
@@ -228,7 +243,10 @@ QL_API ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* 
 /* ---- forward: quantize + GEMM ----------------------------------------------
    route: QL_ROUTE_NVFP4 or QL_ROUTE_INT8 for NVFP4 weights (the activation
    rotation follows w->hadamard); ignored for Q-ARVD weights (per-tensor
-   INT8).  Scratch for the quantized activations lives in `ws`. */
+   INT8).  Scratch for the quantized activations lives in `ws`.  On the INT8
+   route with weights prepared with expand_f16, the INT8 codes are kept as
+   the equal f16 values (2 bytes each) so that the GEMM reads both operands
+   straight into the f16 MMA. */
 QL_API size_t qlinear_forward_ws_bytes(int64_t M, const ql_weights* w, int32_t route);
 QL_API ql_status qlinear_forward(const void* X_bf16, int64_t M, const ql_weights* w,
                           int32_t route, void* Y_bf16,

@@ -58,6 +58,9 @@ def test_size_queries(ql):
     cfg = ql.WeightCfg(ql.QL_W_NVFP4, 1, 3.5, 2.0)
     assert ql.lib.qlinear_weights_bytes(1920, 1920, C.byref(cfg)) >= 1920 * 960 + 1920 * 120
     assert ql.lib.qlinear_weights_bytes(1920, 1000, C.byref(cfg)) == 0          # K % 128
+    ce = ql.WeightCfg(ql.QL_W_NVFP4, 1, 3.5, 2.0, 1, 0)                           # + f16 copy
+    assert (ql.lib.qlinear_weights_bytes(1920, 1920, C.byref(ce))
+            == ql.lib.qlinear_weights_bytes(1920, 1920, C.byref(cfg)) + 1920 * 1920 * 2)
     cq = ql.WeightCfg(ql.QL_W_QARVD_INT4, 0, 3.5, 2.0)
     assert ql.lib.qlinear_weights_bytes(384, 640, C.byref(cq)) >= 384 * (640 + 64) // 2
     assert ql.lib.qlinear_quantize_ws_bytes(10, 130, 0) == 0

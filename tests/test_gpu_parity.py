@@ -212,21 +212,39 @@ def test_gemm_timeout_path_reports_and_recovers(ql):
 W4A8_CASES = [(256, 1920, 1920), (300, 384, 640), (129, 640, 384), (1000, 5760, 1920), (1, 192, 128)]
 
 
+@pytest.mark.parametrize("expand", [False, True])
 @pytest.mark.parametrize("m,n,k", W4A8_CASES)
-def test_forward_w4a8_int8_route_parity(ql, m, n, k):
+def test_forward_w4a8_int8_route_parity(ql, m, n, k, expand):
     x = _x(m, k, seed=m * 3 + n)
     w = S.weights(n, k, 0.02, 7, m + n + k)
     xb, wb = S.bf16_bits(x), S.bf16_bits(w)
     wq = O.prepare_weights_nvfp4(wb)
     rows = np.arange(m) if m <= 512 else np.unique(np.r_[np.random.default_rng(1).choice(m, 256, replace=False), m - 1])
     ref = O.forward(xb, wq, O.ROUTE_INT8, rows=rows)
-    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True, expand_f16=expand)
+    if expand:   # the f16 copy is E2M1 x E4M3 exactly (no tensor scale)
+        w16 = _np(pw.view("w16", torch.float16, n * k).reshape(n, k).float()).astype(np.float64)
+        deq = (O.e2m1_decode(O.unpack_nibbles(wq["packed"])).astype(np.float64)
+               * np.repeat(O.e4m3_decode(wq["sb"]).astype(np.float64), 16, axis=1))
+        assert np.array_equal(w16, deq)
     y = ql.qlinear_forward(x.cuda(), pw, ql.QL_ROUTE_INT8)
     torch.cuda.synchronize()
     assert ql.qlinear_device_status() == 0
     yn = _np(y.float())[rows].astype(np.float64)
     assert np.isfinite(yn).all()
     assert excess_err(yn, ref) <= 1e-3
+    if expand:   # int8 codes through qlinear_gemm: on-chip A expansion, f16 weight copy
+        q = ql.qlinear_quantize_act(x.cuda(), ql.QL_ROUTE_INT8, hadamard=True)
+        y2 = ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, m, pw)
+        # the same codes stored as f16 values, both GEMM operands by TMA
+        q3 = ql.qlinear_quantize_act(x.cuda(), ql.QL_ACT_INT8_F16, hadamard=True)
+        y3 = ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q3, m, pw)
+        torch.cuda.synchronize()
+        assert ql.qlinear_device_status() == 0
+        assert np.array_equal(_np(q3["codes"].float()), _np(q["codes"].float()))
+        assert np.array_equal(_np(q3["scales"]), _np(q["scales"]))
+        assert excess_err(_np(y2.float())[rows].astype(np.float64), ref) <= 1e-3
+        assert excess_err(_np(y3.float())[rows].astype(np.float64), ref) <= 1e-3
 
 
 # ---------------------------------------------------------------- Q-ARVD
