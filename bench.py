@@ -611,6 +611,7 @@ def run_configs(reps: int = 20):
         x, w = S.cogvideox5b_qarvd_linear(lin)
         xd, wd = x.to(dev), w.to(dev)
         pw = ql.qlinear_prepare_weights(wd, ql.QL_W_QARVD_INT4, hadamard=False)
+        pw8 = ql.qlinear_prepare_weights(wd, ql.QL_W_QARVD_INT4, hadamard=False, expand_i8=True)
         kp = pw.desc.Kp
         aws = torch.zeros(ql.lib.qlinear_quantize_ws_bytes(M_TOKENS, lin.k, ql.QL_ROUTE_NVFP4), dtype=torch.uint8,
                           device=dev)
@@ -622,9 +623,13 @@ def run_configs(reps: int = 20):
             "quant_int8_tensor": hbm_rec(med(lambda: ql.qlinear_quantize_act(xd, ql.QL_ACT_INT8_TENSOR, False, w=pw,
                                                                               amax_in=amax, out=q)),
                                          M_TOKENS * (2.0 * lin.k + kp)),
-            "gemm_qarvd": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q, M_TOKENS, pw, Y=y)),
-                                  M_TOKENS, lin.n, lin.k, 2.0)}
-        del xd, wd, pw, q, y
+            # int8 weight copy: both operands by TMA
+            "gemm_qarvd": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q, M_TOKENS, pw8, Y=y)),
+                                  M_TOKENS, lin.n, lin.k, 2.0),
+            # INT4 codes widened on chip
+            "gemm_qarvd_onchip": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q, M_TOKENS, pw, Y=y)),
+                                         M_TOKENS, lin.n, lin.k, 2.0)}
+        del xd, wd, pw, pw8, q, y
     # 5: Wan-14B linears
     for lin in S.WAN_14B:
         x, w = S.wan14b_linear(lin)

@@ -261,7 +261,7 @@ size_t qlinear_weights_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg) {
   if (cfg->fmt == QL_W_QARVD_INT4) {
     const size_t kp = qarvd_kp(K);
     return align256(n * kp / 2) + align256(k) + align256(4 * k) + align256(4 * kp) + 256 +
-           2 * align256(4 * n) + align256(8 * k);
+           2 * align256(4 * n) + align256(8 * k) + (cfg->expand_i8 ? align256(n * kp) : 0);
   }
   return 0;
 }
@@ -280,6 +280,7 @@ ql_status qlinear_prepare_weights(const void* W, int32_t N, int32_t K, const ql_
     return QL_ERR_INVALID_ARG;
   if (cfg->fmt != QL_W_NVFP4 && cfg->fmt != QL_W_QARVD_INT4) return QL_ERR_INVALID_ARG;
   if (cfg->fmt == QL_W_QARVD_INT4 && cfg->expand_f16 != 0) return QL_ERR_INVALID_ARG;
+  if (cfg->fmt == QL_W_NVFP4 && cfg->expand_i8 != 0) return QL_ERR_INVALID_ARG;
   QL_TRY(check_k(K));
   if (N <= 0 || N % 16 != 0 || N > (1 << 24)) return QL_ERR_UNSUPPORTED_SHAPE;
   QL_TRY(check_mk(N, K));
@@ -320,6 +321,10 @@ ql_status qlinear_prepare_weights(const void* W, int32_t N, int32_t K, const ql_
     w.s_out = c.take<float>(4 * static_cast<size_t>(N));
     w.norms = c.take<double>(8 * static_cast<size_t>(K));
     QL_TRY(launch_qarvd_prepare(W, N, K, cfg->tau, cfg->alpha, &w, ws, st));
+    if (cfg->expand_i8) {
+      w.w8 = c.take<int8_t>(static_cast<size_t>(N) * w.Kp);
+      QL_TRY(launch_expand_int4_i8(w.codes, N, w.Kp, w.w8, st));
+    }
   }
   *out = w;
   return QL_OK;

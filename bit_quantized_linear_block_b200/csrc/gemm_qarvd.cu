@@ -287,9 +287,368 @@ __global__ void __launch_bounds__(512, 1)
   if (warp == 10) tmem_dealloc(tmem, 512);
 }
 
+// --------------------------------------------------------------------------
+// Weights kept as int8 (prepared with expand_i8): both operands come by TMA
+// in the 128-byte-swizzled K-major layout and no warp touches them.
+//
+// 384 threads per CTA, one CTA per SM, the W4A4 kernel's roles:
+//   warp 0      TMA producer;
+//   warp 1      MMA issuer (kind::i8, each 32-wide K step to its class's
+//               accumulator);
+//   warp 2      tensor-memory allocation (2 tiles x 2 classes x 128 columns);
+//   warps 4-11  epilogue, two warps per TMEM lane quarter, each with half
+//               of the tile's columns, storing 32 x 32 boxes by TMA.
+//   PAIR = true   two SMs of a cluster share each 256 x 128 tile through
+//                 tcgen05 cta_group::2 (each CTA holds its 128 activation
+//                 rows and 64 of the 128 weight rows); the leader issues.
+//   PAIR = false  one SM per 128 x 128 tile (M <= 128).
+// --------------------------------------------------------------------------
+template <bool PAIR, int STAGES>
+struct QarvdPreCfg {
+  static constexpr int CTAS = PAIR ? 2 : 1;
+  static constexpr int BM = 128;              // activation rows per CTA
+  static constexpr int BN = 128;              // tile columns (MMA N)
+  static constexpr int BNL = BN / CTAS;       // weight rows held by each CTA
+  static constexpr int BK = 128;              // K bytes (= int8 elements) per stage
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BNL * BK;
+  static constexpr int EPI_WARPS = 8;
+  static constexpr int EPI_BUF = 2;
+  static constexpr int EPI_CH = BN / 2 / kWarpBoxCols;   // boxes per epilogue warp per tile
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_C = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_BAR = OFF_C + EPI_WARPS * EPI_BUF * kWarpBoxBytes;
+  static constexpr int NBAR = 2 * STAGES + 2 * 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(B_BYTES % 1024 == 0, "1024-byte aligned stages");
+  static constexpr uint32_t IDESC = (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) |
+                                    (uint32_t((BM * CTAS) >> 4) << 24);
+};
+
+template <bool PAIR, int STAGES>
+__global__ void __launch_bounds__(384, 1)
+    k_gemm_qarvd_pre(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
+  using C = QarvdPreCfg<PAIR, STAGES>;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);   // pair: the leader's is used
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;                                     // pair: the leader's is used
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const int k_norm_pad = p.kinfo[1];
+  const int k_out_pad = p.kinfo[3];
+  const int k_used = k_norm_pad + k_out_pad;
+  const int num_kst = (k_used + C::BK - 1) / C::BK;
+
+  const uint32_t rank = PAIR ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int warp = threadIdx.x >> 5;
+  const int unit = PAIR ? (blockIdx.x >> 1) : blockIdx.x;
+  const int nunits = PAIR ? (gridDim.x >> 1) : gridDim.x;
+
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_y);
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], C::EPI_WARPS * C::CTAS);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if constexpr (PAIR) cluster_sync();   // both CTAs' barriers exist before any remote use
+  if (warp == 2) {
+    if constexpr (PAIR)
+      tmem_alloc_pair(tmem_slot, 512);
+    else
+      tmem_alloc(tmem_slot, 512);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (elect_one()) {
+      int it = 0;
+      bool ok = true;
+      constexpr uint32_t tx = C::A_BYTES + C::B_BYTES;
+      for (int t = unit; t < p.num_tiles && ok; t += nunits) {
+        int mb, nb;
+        tile_coords(t, p, mb, nb);
+        const int a_row = mb * C::BM * C::CTAS + static_cast<int>(rank) * C::BM;
+        const int b_row = nb * BN + static_cast<int>(rank) * C::BNL;
+        for (int ks = 0; ks < num_kst; ++ks, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1, p.wait_limit)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + C::OFF_A + s * C::A_BYTES;
+          uint8_t* sb = smem + C::OFF_B + s * C::B_BYTES;
+          if constexpr (PAIR) {
+            // Both CTAs' bytes complete on the leader's barrier.
+            if (leader) mbar_arrive_expect_tx(&full[s], 2 * tx);
+            const uint32_t bar = map_to_rank(smem_u32(&full[s]), 0);
+            tma_load_2d_pair(sa, &tm_a, bar, ks * C::BK, a_row);
+            tma_load_2d_pair(sb, &tm_b, bar, ks * C::BK, b_row);
+          } else {
+            mbar_arrive_expect_tx(&full[s], tx);
+            tma_load_2d(sa, &tm_a, &full[s], ks * C::BK, a_row);
+            tma_load_2d(sb, &tm_b, &full[s], ks * C::BK, b_row);
+          }
+        }
+      }
+      if (!ok) fail_timeout(p.status, abort_flag);
+      if (leader) {
+        drain_loads(full, it, STAGES, p.status);   // pair: covers both CTAs' bytes
+      } else {
+        // The peer's loads complete on the leader's barriers; the leader frees
+        // each stage (empty) only after the MMAs consumed both halves.
+        for (int j = max(0, it - STAGES); j < it; ++j)
+          if (!mbar_wait(&empty[j % STAGES], (j / STAGES) & 1, kDrainLimit)) record_error(p.status, QL_ERR_TIMEOUT);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (leader && elect_one()) {
+      int it = 0, local = 0;
+      bool ok = true;
+      auto commit_to = [&](uint64_t* bar) {
+        if constexpr (PAIR) {
+          tc_commit_pair(map_to_rank(smem_u32(bar), 0));
+          tc_commit_pair(map_to_rank(smem_u32(bar), 1));
+        } else {
+          tc_commit(bar);
+        }
+      };
+      for (int t = unit; t < p.num_tiles && ok; t += nunits, ++local) {
+        const int acc = local & 1;
+        if (*abort_flag || !mbar_wait(&tempty[acc], ((local >> 1) & 1) ^ 1, p.wait_limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_norm = tmem + acc * 2 * BN;
+        const uint32_t d_out = d_norm + BN;
+        bool started_norm = false, started_out = false;
+        for (int ks = 0; ks < num_kst; ++ks, ++it) {
+          const int s = it % STAGES;
+          if (*abort_flag || !mbar_wait(&full[s], (it / STAGES) & 1, p.wait_limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + C::OFF_A + s * C::A_BYTES);
+          const uint32_t b_base = smem_u32(smem + C::OFF_B + s * C::B_BYTES);
+#pragma unroll
+          for (int i = 0; i < C::BK / 32; ++i) {
+            const int kk = ks * C::BK + 32 * i;
+            if (kk >= k_used) break;
+            const bool normal = kk < k_norm_pad;
+            const uint64_t adesc = smem_desc(a_base + 32 * i, 0, 1024, kSwizzle128B);
+            const uint64_t bdesc = smem_desc(b_base + 32 * i, 0, 1024, kSwizzle128B);
+            const uint32_t accum = (normal ? started_norm : started_out) ? 1u : 0u;
+            if constexpr (PAIR)
+              tc_mma_i8_pair(normal ? d_norm : d_out, adesc, bdesc, C::IDESC, accum);
+            else
+              tc_mma_i8(normal ? d_norm : d_out, adesc, bdesc, C::IDESC, accum);
+            if (normal) started_norm = true; else started_out = true;
+          }
+          commit_to(&empty[s]);
+        }
+        if (!ok) break;
+        commit_to(&tfull[acc]);
+      }
+      if (!ok) fail_timeout(p.status, abort_flag);
+      if constexpr (PAIR) {
+        tc_commit_pair(map_to_rank(smem_u32(drain), 0));
+        if (!mbar_wait(drain, 0, kDrainLimit)) record_error(p.status, QL_ERR_TIMEOUT);
+      } else {
+        drain_mma(drain, p.status);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    // y = bf16(s_x * (s_norm[n] * acc_normal + s_out[n] * acc_outlier)); a
+    // class without channels contributes 0 (its accumulator is never written).
+    const float sx = *p.g_a;
+    const int quarter = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int lane = lane_id();
+    const bool has_norm = k_norm_pad != 0, has_out = k_out_pad != 0;
+    uint8_t* stage = smem + C::OFF_C + (warp - 4) * C::EPI_BUF * kWarpBoxBytes;
+    const uint32_t swz = (lane >> 1) & 3;
+    int next_buf = 0;
+    int local = 0;
+    for (int t = unit; t < p.num_tiles; t += nunits, ++local) {
+      int mb, nb;
+      tile_coords(t, p, mb, nb);
+      const int acc = local & 1;
+      const int row0 = mb * C::BM * C::CTAS + static_cast<int>(rank) * C::BM + 32 * quarter;
+      const int c0 = nb * BN + half * (BN / 2);
+      // lane i holds the scales of column c0 + 32 c + i (0 past N)
+      float sn[C::EPI_CH], so[C::EPI_CH];
+#pragma unroll
+      for (int c = 0; c < C::EPI_CH; ++c) {
+        const int n = c0 + kWarpBoxCols * c + lane;
+        sn[c] = (n < p.N) ? __ldg(p.col_scale0 + n) : 0.f;
+        so[c] = (n < p.N) ? __ldg(p.col_scale1 + n) : 0.f;
+      }
+      if (!warp_wait_uniform(&tfull[acc], (local >> 1) & 1, p.wait_limit, abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t release = PAIR ? map_to_rank(smem_u32(&tempty[acc]), 0) : smem_u32(&tempty[acc]);
+      const uint32_t taddr = tmem + acc * 2 * BN + half * (BN / 2) + (static_cast<uint32_t>(32 * quarter) << 16);
+      uint32_t packed[C::EPI_CH][16];
+#pragma unroll
+      for (int c = 0; c < C::EPI_CH; ++c) {
+        uint32_t an[32], ao[32];
+        tmem_ld32(taddr + kWarpBoxCols * c, an);
+        tmem_ld32(taddr + BN + kWarpBoxCols * c, ao);
+        tmem_ld_wait();
+        if (c == C::EPI_CH - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(release);
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          float y[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int jj = 2 * j + e;
+            const float fn = has_norm ? static_cast<float>(static_cast<int32_t>(an[jj])) : 0.f;
+            const float fo = has_out ? static_cast<float>(static_cast<int32_t>(ao[jj])) : 0.f;
+            const float cn = __shfl_sync(0xffffffffu, sn[c], jj);
+            const float co = __shfl_sync(0xffffffffu, so[c], jj);
+            y[e] = __fmul_rn(sx, __fadd_rn(__fmul_rn(cn, fn), __fmul_rn(co, fo)));
+          }
+          packed[c][j] = pack_bf16x2(y[0], y[1]);
+        }
+      }
+      if (row0 >= p.M) continue;   // warp-uniform
+#pragma unroll
+      for (int c = 0; c < C::EPI_CH; ++c) {
+        const int col = c0 + kWarpBoxCols * c;
+        if (col >= p.N) break;   // warp-uniform; TMA clips partial boxes
+        uint8_t* buf = stage + next_buf * kWarpBoxBytes;
+        if (lane == 0) bulk_wait_read<C::EPI_BUF - 1>();
+        __syncwarp();
+        uint8_t* dst = buf + lane * 64;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<uint4*>(dst + ((q ^ swz) << 4)) =
+              make_uint4(packed[c][4 * q], packed[c][4 * q + 1], packed[c][4 * q + 2], packed[c][4 * q + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, buf, col, row0);
+          bulk_commit();
+        }
+        next_buf = (next_buf + 1 == C::EPI_BUF) ? 0 : next_buf + 1;
+      }
+    }
+    epilogue_warp_finish();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // no CTA leaves while its peer may still signal it
+  tc_fence_after();
+  if (warp == 2) {
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem, 512);
+    else
+      tmem_dealloc(tmem, 512);
+  }
+}
+
+template <bool PAIR, int STAGES>
+static ql_status launch_qarvd_pre(const void* a_codes, const float* s_x, int64_t M, const ql_weights* w, void* Y,
+                                  cudaStream_t st, int* status) {
+  using C = QarvdPreCfg<PAIR, STAGES>;
+  const int N = w->N, Kp = w->Kp;
+  CUtensorMap ta, tb, ty;
+  if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kp, M, Kp, C::BK, C::BM,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->w8, Kp, N, Kp, C::BK, C::BNL,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<int64_t>(N) * 2,
+                    kWarpBoxCols, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return QL_ERR_CUDA;
+  GemmArgs p{};
+  fill_gemm_args(p, M, N, Kp, C::BN, status);
+  p.tiles_m = static_cast<int32_t>((M + C::BM * C::CTAS - 1) / (C::BM * C::CTAS));
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.g_a = s_x;
+  p.col_scale0 = w->s_norm;
+  p.col_scale1 = w->s_out;
+  p.kinfo = w->kinfo;
+  auto kern = k_gemm_qarvd_pre<PAIR, STAGES>;
+  if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
+  const int units = std::min(p.num_tiles, num_sms() / C::CTAS);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(units * C::CTAS));
+  cfg.blockDim = dim3(384);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C::CTAS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
+// Sign-extend the packed INT4 weight codes to int8 ([N, Kp/2] bytes ->
+// [N, Kp] int8), 8 bytes per thread.
+__global__ void k_expand_int4_i8(const uint2* __restrict__ in, uint4* __restrict__ out, int64_t n8) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint2 q = in[i];
+    const uint2 a = int4x8_to_int8(q.x);
+    const uint2 b = int4x8_to_int8(q.y);
+    out[i] = make_uint4(a.x, a.y, b.x, b.y);
+  }
+}
+
+ql_status launch_expand_int4_i8(const void* codes, int32_t N, int32_t Kp, void* out, cudaStream_t st) {
+  const int64_t n8 = static_cast<int64_t>(N) * Kp / 16;   // 8-byte groups (Kp % 32 == 0)
+  const int grid = hbm_grid(n8, 256 * 4);
+  k_expand_int4_i8<<<grid, 256, 0, st>>>(static_cast<const uint2*>(codes), static_cast<uint4*>(out), n8);
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
 ql_status launch_gemm_qarvd(const void* a_codes, const float* s_x, int64_t M, const ql_weights* w, void* Y,
                             cudaStream_t st, int* status) {
   if (M == 0) return QL_OK;
+  if (w->w8 != nullptr) {
+    if (M > 128) return launch_qarvd_pre<true, 8>(a_codes, s_x, M, w, Y, st, status);
+    return launch_qarvd_pre<false, 5>(a_codes, s_x, M, w, Y, st, status);
+  }
   constexpr int S = 4;
   using C = QarvdCfg<S>;
   const int N = w->N, Kp = w->Kp;

@@ -47,6 +47,9 @@ ql_status launch_gemm_w4a4(const void* a_codes, const uint8_t* a_sf, const float
 // weights prepared with expand_f16).
 ql_status launch_gemm_w4a8(const void* a_codes, const float* a_scales, int64_t M,
                            const ql_weights* w, void* Y, cudaStream_t st, int* status, int a_f16 = 0);
+// int8 copy [N, Kp] of the Q-ARVD INT4 codes (sign-extended).
+ql_status launch_expand_int4_i8(const void* codes, int32_t N, int32_t Kp, void* out, cudaStream_t st);
+// Uses the int8 weight copy (w->w8) when the weights carry one.
 ql_status launch_gemm_qarvd(const void* a_codes, const float* s_x, int64_t M, const ql_weights* w,
                             void* Y, cudaStream_t st, int* status);
 

@@ -31,7 +31,7 @@ QL_ACT_INT8_F16 = 3
 
 class WeightCfg(C.Structure):
     _fields_ = [("fmt", C.c_int32), ("hadamard", C.c_int32), ("tau", C.c_float), ("alpha", C.c_float),
-                ("expand_f16", C.c_int32), ("reserved", C.c_int32)]
+                ("expand_f16", C.c_int32), ("expand_i8", C.c_int32)]
 
 
 class Weights(C.Structure):
@@ -40,7 +40,7 @@ class Weights(C.Structure):
                 ("codes", C.c_void_p), ("sf", C.c_void_p), ("gscale", C.c_void_p),
                 ("outlier_mask", C.c_void_p), ("perm", C.c_void_p), ("gather", C.c_void_p),
                 ("kinfo", C.c_void_p), ("s_norm", C.c_void_p), ("s_out", C.c_void_p),
-                ("norms", C.c_void_p), ("w16", C.c_void_p)]
+                ("norms", C.c_void_p), ("w16", C.c_void_p), ("w8", C.c_void_p)]
 
 
 class QLinearError(RuntimeError):
@@ -128,12 +128,14 @@ class PackedWeights:
 
 def qlinear_prepare_weights(W: torch.Tensor, fmt: int = QL_W_NVFP4, hadamard: bool = True,
                             tau: float = 3.5, alpha: float = 2.0, stream=None,
-                            expand_f16: bool = False) -> PackedWeights:
+                            expand_f16: bool = False, expand_i8: bool = False) -> PackedWeights:
     """expand_f16 (NVFP4 only) also keeps an f16 copy of the dequantized
-    weights for the INT8 route's GEMM."""
+    weights for the INT8 route's GEMM; expand_i8 (Q-ARVD only) keeps the
+    INT4 codes sign-extended to int8 for the Q-ARVD GEMM."""
     assert W.dtype == torch.bfloat16 and W.is_cuda and W.dim() == 2 and W.is_contiguous()
     N, K = W.shape
-    cfg = WeightCfg(fmt, int(bool(hadamard)) if fmt == QL_W_NVFP4 else 0, tau, alpha, int(bool(expand_f16)), 0)
+    cfg = WeightCfg(fmt, int(bool(hadamard)) if fmt == QL_W_NVFP4 else 0, tau, alpha, int(bool(expand_f16)),
+                    int(bool(expand_i8)))
     wbytes = lib.qlinear_weights_bytes(N, K, C.byref(cfg))
     wsbytes = lib.qlinear_prepare_ws_bytes(N, K, C.byref(cfg))
     if wbytes == 0:

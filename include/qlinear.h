@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define QLINEAR_ABI_VERSION 2
+#define QLINEAR_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define QL_API __attribute__((visibility("default")))
@@ -106,7 +106,10 @@ typedef struct {
                         the INT8 route's GEMM, which then reads it directly
                         instead of expanding the FP4 codes on chip.  Costs
                         2 bytes per weight in the weight buffer.              */
-  int32_t reserved;  /* 0                                                      */
+  int32_t expand_i8; /* Q-ARVD: 1 = also keep the INT4 codes sign-extended to
+                        int8 ([N, Kp], exact) for the GEMM, which then loads
+                        both operands by TMA instead of widening the weights
+                        on chip.  Costs 1 byte per code in the weight buffer. */
 } ql_weight_cfg;
 
 /* Packed weights.  Filled by qlinear_prepare_weights(); every pointer points
@@ -127,6 +130,8 @@ typedef struct {
   double* norms;         /* Q-ARVD [K] input-channel L2 norms                   */
   void* w16;             /* NVFP4 with expand_f16: f16 [N, K] = E2M1 x E4M3
                             (no g_w); NULL otherwise                            */
+  void* w8;              /* Q-ARVD with expand_i8: int8 [N, Kp] = the INT4
+                            codes sign-extended; NULL otherwise                 */
 } ql_weights;
 
 /* ---- library ------------------------------------------------------------ */

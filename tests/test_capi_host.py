@@ -63,6 +63,9 @@ def test_size_queries(ql):
             == ql.lib.qlinear_weights_bytes(1920, 1920, C.byref(cfg)) + 1920 * 1920 * 2)
     cq = ql.WeightCfg(ql.QL_W_QARVD_INT4, 0, 3.5, 2.0)
     assert ql.lib.qlinear_weights_bytes(384, 640, C.byref(cq)) >= 384 * (640 + 64) // 2
+    cq8 = ql.WeightCfg(ql.QL_W_QARVD_INT4, 0, 3.5, 2.0, 0, 1)                     # + int8 copy
+    assert (ql.lib.qlinear_weights_bytes(384, 640, C.byref(cq8))
+            == ql.lib.qlinear_weights_bytes(384, 640, C.byref(cq)) + 384 * 672)    # Kp = 640 + 32
     assert ql.lib.qlinear_quantize_ws_bytes(10, 130, 0) == 0
     assert ql.lib.qlinear_route_ws_bytes(-1) == 0 and ql.lib.qlinear_route_ws_bytes(10) > 0
 
@@ -102,6 +105,10 @@ def test_other_entry_points_reject_bad_arguments(ql):
     desc = ql.Weights()
     assert L.qlinear_prepare_weights(FAKE, 256, 256, C.byref(cfg), FAKE, 1 << 30, C.byref(desc),
                                      FAKE, 1 << 30, None) == 1
+    for bad in (ql.WeightCfg(ql.QL_W_NVFP4, 1, 3.5, 2.0, 0, 1),                  # int8 copy of NVFP4
+                ql.WeightCfg(ql.QL_W_QARVD_INT4, 0, 3.5, 2.0, 1, 0)):            # f16 copy of Q-ARVD
+        assert L.qlinear_prepare_weights(FAKE, 256, 256, C.byref(bad), FAKE, 1 << 30, C.byref(desc),
+                                         FAKE, 1 << 30, None) == 1
     assert L.qlinear_gemm(0, FAKE, FAKE, FAKE, 10, None, FAKE, None) == 1
 
 

@@ -166,8 +166,9 @@ def test_dmpq_routing_sweep_and_routed_ffn_up(ql):
     assert checked == {0, 1}, routes       # the sweep exercises both routes
 
 
+@pytest.mark.parametrize("expand", [False, True])
 @pytest.mark.parametrize("name", [l.name for l in S.COGVIDEOX_5B])
-def test_cogvideox5b_qarvd_linear(ql, name):
+def test_cogvideox5b_qarvd_linear(ql, name, expand):
     lin = [l for l in S.COGVIDEOX_5B if l.name == name][0]
     x, w = S.cogvideox5b_qarvd_linear(lin)
     wb = S.bf16_bits(w)
@@ -175,7 +176,7 @@ def test_cogvideox5b_qarvd_linear(ql, name):
     zs = pk["zscore"][np.isfinite(pk["zscore"])]
     assert np.all(np.abs(zs - 3.5) > 3.5e-9)
     assert np.all(np.abs(pk["norms"] - 2.0 * pk["median"]) > 1e-9 * pk["median"])
-    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_QARVD_INT4, hadamard=False)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_QARVD_INT4, hadamard=False, expand_i8=expand)
     torch.cuda.synchronize()
     n, k, kp = lin.n, lin.k, pw.desc.Kp
     assert np.array_equal(_np(pw.view("outlier_mask", torch.uint8, k)).astype(bool), pk["mask"])
@@ -186,6 +187,8 @@ def test_cogvideox5b_qarvd_linear(ql, name):
     want[:, :pk["codes"].shape[1]] = pk["codes"]
     got = _np(pw.view("codes", torch.uint8, n * kp // 2)).reshape(n, kp // 2)
     assert np.array_equal(got, O.pack_int4(want))
+    if expand:
+        assert np.array_equal(_np(pw.view("w8", torch.int8, n * kp)).reshape(n, kp), want)
     xb = S.bf16_bits(x)
     xd = x.cuda()
     q = ql.qlinear_quantize_act(xd, ql.QL_ACT_INT8_TENSOR, hadamard=False, w=pw)

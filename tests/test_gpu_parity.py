@@ -283,21 +283,29 @@ def test_prepare_weights_qarvd_bit_exact(ql, n, k, frac):
     assert np.array_equal(got, O.pack_int4(want))
 
 
-@pytest.mark.parametrize("m,n,k", [(300, 384, 640), (256, 256, 3072), (77, 128, 128)])
-def test_qarvd_activation_quant_and_forward_parity(ql, m, n, k):
-    w = _qarvd_weights(n, k, seed=m + n)
+@pytest.mark.parametrize("expand", [False, True])
+@pytest.mark.parametrize("m,n,k,frac", [(300, 384, 640, 0.05), (256, 256, 3072, 0.05), (77, 128, 128, 0.05),
+                                        (513, 200 - 8, 1024, 0.0), (130, 64, 512, 0.3)])
+def test_qarvd_activation_quant_and_forward_parity(ql, m, n, k, frac, expand):
+    w = _qarvd_weights(n, k, seed=m + n, frac=frac)
     pk = O.qarvd_pack(S.bf16_bits(w), 3.5, 2.0)
+    _assert_guard_band(pk)
     x = _x(m, k, seed=m + 5 * k)
     xb = S.bf16_bits(x)
     qx, sx = O.int8_per_tensor(O.bf16_bits_to_f32(xb))
     qxp = O.qarvd_permute_activations(qx, pk["perm"], pk["k_norm"], pk["k_norm_pad"], pk["n_out"], pk["k_out_pad"])
-    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_QARVD_INT4, hadamard=False)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_QARVD_INT4, hadamard=False, expand_i8=expand)
     xc = x.cuda()
     q = ql.qlinear_quantize_act(xc, ql.QL_ACT_INT8_TENSOR, hadamard=False, w=pw)
     y = ql.qlinear_forward(xc, pw)
     torch.cuda.synchronize()
     assert ql.qlinear_device_status() == 0
     kp = pw.desc.Kp
+    assert (pw.desc.w8 is not None) == expand
+    if expand:   # the int8 copy is the INT4 codes sign-extended, zero in the padding
+        want_w = np.zeros((n, kp), np.int8)
+        want_w[:, :pk["codes"].shape[1]] = pk["codes"]
+        assert np.array_equal(_np(pw.view("w8", torch.int8, n * kp)).reshape(n, kp), want_w)
     want = np.zeros((m, kp), np.int8)
     want[:, :qxp.shape[1]] = qxp
     assert _np(q["scales"])[0] == sx
