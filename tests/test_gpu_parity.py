@@ -285,7 +285,8 @@ def test_prepare_weights_qarvd_bit_exact(ql, n, k, frac):
 
 @pytest.mark.parametrize("expand", [False, True])
 @pytest.mark.parametrize("m,n,k,frac", [(300, 384, 640, 0.05), (256, 256, 3072, 0.05), (77, 128, 128, 0.05),
-                                        (513, 200 - 8, 1024, 0.0), (130, 64, 512, 0.3)])
+                                        (513, 200 - 8, 1024, 0.0), (130, 64, 512, 0.3),
+                                        (2048, 1920, 512, 0.05)])   # several tiles per SM pair
 def test_qarvd_activation_quant_and_forward_parity(ql, m, n, k, frac, expand):
     w = _qarvd_weights(n, k, seed=m + n, frac=frac)
     pk = O.qarvd_pack(S.bf16_bits(w), 3.5, 2.0)
