@@ -52,20 +52,25 @@ namespace ql {
 
 constexpr int kResKSteps = 30;   // K steps (64 wide) of resident activation scales
 
-template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES>
+template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES, int BKB_ = 128>
 struct W4A4Cfg {
   static constexpr int CTAS = PAIR ? 2 : 1;
   static constexpr int BM = 128;                     // rows per CTA
-  static constexpr int BKB = 128;                    // K bytes per stage = 256 FP4 values
+  static constexpr int BKB = BKB_;                   // K bytes per stage (2 FP4 values a byte)
+  static constexpr int KC = BKB / 128;               // 128-byte K chunks (one swizzle span each)
+  static constexpr int KSTEPS = BKB / 32;            // 64-wide MMA K steps (scale atoms) per stage
   static constexpr int BNL = BN / CTAS;              // B rows held by each CTA
-  static constexpr int A_BYTES = BM * BKB;
-  static constexpr int B_BYTES = BNL * BKB;
+  static constexpr int A_CHUNK = BM * 128;
+  static constexpr int B_CHUNK = BNL * 128;
+  static constexpr int A_BYTES = KC * A_CHUNK;
+  static constexpr int B_BYTES = KC * B_CHUNK;
   // 128-row scale atoms per B tile.  Each CTA of a pair holds the weight
   // scales of all BN rows: each SM's MMA reads every B row's scales from its
   // own tensor memory.
   static constexpr int NSFB = (BN + 127) / 128;
-  static constexpr int SFA_BYTES = RES ? 0 : 4 * 512;           // per stage
-  static constexpr int SFB_BYTES = NSFB * 4 * 512;              // per stage
+  static constexpr int SFA_BYTES = RES ? 0 : KSTEPS * 512;      // per stage
+  static constexpr int SFB_GROUP = KSTEPS * 512;                // one 128-row atom column per stage
+  static constexpr int SFB_BYTES = NSFB * SFB_GROUP;            // per stage
   static constexpr int SFA_RES_BYTES = RES ? kResKSteps * 512 : 0;
   static constexpr int ACC = ACC_;
   static constexpr int EPI_WARPS = 8;
@@ -95,7 +100,8 @@ struct W4A4Cfg {
   static_assert(RES ? SFB_SLOTS >= 1 : (SF_SLOTS >= 2 && SF_SLOTS < STAGES), "scale slots");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(BN % 64 == 0 && BN <= 256 && BNL % 16 == 0, "tile width");
-  static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "1024-byte aligned stages");
+  static_assert(A_CHUNK % 1024 == 0 && B_CHUNK % 1024 == 0, "1024-byte aligned chunks");
+  static_assert(BKB % 128 == 0 && (RES || BKB == 128), "streamed scales take 128-byte stages");
   static_assert(EPI_BUF >= 1 && EPI_BUF <= EPI_CH, "staging buffers");
   // Instruction descriptor (block-scaled): A/B = E2M1 (1), scale = UE4M3 (0),
   // both K-major, N >> 3 at bit 17, M >> 4 at bit 24, dense K = 64.
@@ -130,12 +136,12 @@ struct TileWalk {
   }
 };
 
-template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES>
+template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES, int BKB_>
 __global__ void __launch_bounds__(384, 1)
     k_gemm_w4a4(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                 const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
-  using C = W4A4Cfg<BN, STAGES, PAIR, ACC_, EPI_BUF, RES>;
+  using C = W4A4Cfg<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);   // pair: the leader's is used
@@ -223,7 +229,7 @@ __global__ void __launch_bounds__(384, 1)
         int nsfb = 0;
 #pragma unroll
         for (int r = 0; r < C::NSFB; ++r) nsfb += (ra0 + r < p.sfb_atoms);
-        const uint32_t tx = C::A_BYTES + C::B_BYTES + C::SFA_BYTES + nsfb * 2048;
+        const uint32_t tx = C::A_BYTES + C::B_BYTES + C::SFA_BYTES + nsfb * C::SFB_GROUP;
         for (int ks = 0; ks < p.num_kst; ++ks, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
@@ -239,20 +245,28 @@ __global__ void __launch_bounds__(384, 1)
             // Both CTAs' bytes complete on the leader's barrier.
             if (leader) mbar_arrive_expect_tx(&full[s], 2 * tx);
             const uint32_t bar = map_to_rank(smem_u32(&full[s]), 0);
-            tma_load_2d_pair(sa, &tm_a, bar, ks * C::BKB, a_row);
-            tma_load_2d_pair(sb, &tm_b, bar, ks * C::BKB, b_row);
-            if constexpr (!RES) tma_load_3d_pair(ssfa, &tm_sfa, bar, 0, 4 * ks, sfa_group);
+#pragma unroll
+            for (int c = 0; c < C::KC; ++c) {
+              tma_load_2d_pair(sa + c * C::A_CHUNK, &tm_a, bar, ks * C::BKB + 128 * c, a_row);
+              tma_load_2d_pair(sb + c * C::B_CHUNK, &tm_b, bar, ks * C::BKB + 128 * c, b_row);
+            }
+            if constexpr (!RES) tma_load_3d_pair(ssfa, &tm_sfa, bar, 0, C::KSTEPS * ks, sfa_group);
 #pragma unroll
             for (int r = 0; r < C::NSFB; ++r)
-              if (ra0 + r < p.sfb_atoms) tma_load_3d_pair(ssfb + r * 2048, &tm_sfb, bar, 0, 4 * ks, ra0 + r);
+              if (ra0 + r < p.sfb_atoms)
+                tma_load_3d_pair(ssfb + r * C::SFB_GROUP, &tm_sfb, bar, 0, C::KSTEPS * ks, ra0 + r);
           } else {
             mbar_arrive_expect_tx(&full[s], tx);
-            tma_load_2d(sa, &tm_a, &full[s], ks * C::BKB, a_row);
-            tma_load_2d(sb, &tm_b, &full[s], ks * C::BKB, b_row);
-            if constexpr (!RES) tma_load_3d(ssfa, &tm_sfa, &full[s], 0, 4 * ks, sfa_group);
+#pragma unroll
+            for (int c = 0; c < C::KC; ++c) {
+              tma_load_2d(sa + c * C::A_CHUNK, &tm_a, &full[s], ks * C::BKB + 128 * c, a_row);
+              tma_load_2d(sb + c * C::B_CHUNK, &tm_b, &full[s], ks * C::BKB + 128 * c, b_row);
+            }
+            if constexpr (!RES) tma_load_3d(ssfa, &tm_sfa, &full[s], 0, C::KSTEPS * ks, sfa_group);
 #pragma unroll
             for (int r = 0; r < C::NSFB; ++r)
-              if (ra0 + r < p.sfb_atoms) tma_load_3d(ssfb + r * 2048, &tm_sfb, &full[s], 0, 4 * ks, ra0 + r);
+              if (ra0 + r < p.sfb_atoms)
+                tma_load_3d(ssfb + r * C::SFB_GROUP, &tm_sfb, &full[s], 0, C::KSTEPS * ks, ra0 + r);
           }
         }
       }
@@ -320,18 +334,18 @@ __global__ void __launch_bounds__(384, 1)
             break;
           }
           tc_fence_after();
-          const int nk = min(4, p.k_atoms - 4 * ks);
+          const int nk = min(C::KSTEPS, p.k_atoms - C::KSTEPS * ks);
           const uint32_t a_base = smem_u32(smem + C::OFF_A + s * C::A_BYTES);
           const uint32_t b_base = smem_u32(smem + C::OFF_B + s * C::B_BYTES);
           const uint32_t sfa_base = smem_u32(smem + C::OFF_SFA + s * C::SFA_BYTES);
           const uint32_t sfb_base = smem_u32(smem + C::OFF_SFB + s * C::SFB_BYTES);
           const uint32_t t_slot = tmem + C::TM_SF + (it % C::SF_SLOTS) * C::SF_COLS;   // streaming
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < C::KSTEPS; ++i) {
             if (i >= nk) break;
             uint32_t t_sfa, t_sfb;
             if constexpr (RES) {
-              t_sfa = tmem + C::TM_SF + 4 * (4 * ks + i);
+              t_sfa = tmem + C::TM_SF + 4 * (C::KSTEPS * ks + i);
               t_sfb = tmem + C::TM_SFB_RES + (gk % C::SFB_SLOTS) * C::SFB_KCOLS;
               ++gk;
             } else {
@@ -340,9 +354,10 @@ __global__ void __launch_bounds__(384, 1)
               cp_sf(t_sfa, sfa_base + 512 * i);
             }
 #pragma unroll
-            for (int r = 0; r < C::NSFB; ++r) cp_sf(t_sfb + 4 * r, sfb_base + 2048 * r + 512 * i);
-            const uint64_t adesc = smem_desc(a_base + 32 * i, 0, 1024, kSwizzle128B);
-            const uint64_t bdesc = smem_desc(b_base + 32 * i, 0, 1024, kSwizzle128B);
+            for (int r = 0; r < C::NSFB; ++r) cp_sf(t_sfb + 4 * r, sfb_base + C::SFB_GROUP * r + 512 * i);
+            const uint32_t koff = 32 * (i & 3);
+            const uint64_t adesc = smem_desc(a_base + (i >> 2) * C::A_CHUNK + koff, 0, 1024, kSwizzle128B);
+            const uint64_t bdesc = smem_desc(b_base + (i >> 2) * C::B_CHUNK + koff, 0, 1024, kSwizzle128B);
             const uint32_t accum = (ks > 0 || i > 0) ? 1u : 0u;
             if constexpr (PAIR)
               tc_mma_nvf4_pair(d_tmem, adesc, bdesc, C::IDESC, t_sfa, t_sfb + sfb_shift, accum);
@@ -401,11 +416,11 @@ __global__ void __launch_bounds__(384, 1)
 // --------------------------------------------------------------------------
 // Host side
 // --------------------------------------------------------------------------
-template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES>
+template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES, int BKB_ = 128>
 static ql_status launch_w4a4_cfg(const void* a_codes, const uint8_t* a_sf, const float* g_a,
                                  int64_t M, const ql_weights* w, void* Y, cudaStream_t st,
                                  int* status) {
-  using C = W4A4Cfg<BN, STAGES, PAIR, ACC_, EPI_BUF, RES>;
+  using C = W4A4Cfg<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_>;
   const int N = w->N, K = w->K;
   if (RES && K / 64 > kResKSteps) return QL_ERR_UNSUPPORTED_SHAPE;
   CUtensorMap ta, tb, tsa, tsb, ty;
@@ -413,7 +428,7 @@ static ql_status launch_w4a4_cfg(const void* a_codes, const uint8_t* a_sf, const
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, 128, C::BNL,
                     CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_sf_tmap(&tsa, a_sf, M, K, RES ? K / 64 : 4) || !make_sf_tmap(&tsb, w->sf, N, K, 4) ||
+      !make_sf_tmap(&tsa, a_sf, M, K, RES ? K / 64 : C::KSTEPS) || !make_sf_tmap(&tsb, w->sf, N, K, C::KSTEPS) ||
       !make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<int64_t>(N) * 2,
                     kWarpBoxCols, 32, CU_TENSOR_MAP_SWIZZLE_64B))
     return QL_ERR_CUDA;
@@ -421,13 +436,13 @@ static ql_status launch_w4a4_cfg(const void* a_codes, const uint8_t* a_sf, const
   fill_gemm_args(p, M, N, K, BN, status);
   p.tiles_m = static_cast<int32_t>((M + C::BM * C::CTAS - 1) / (C::BM * C::CTAS));
   p.num_tiles = p.tiles_m * p.tiles_n;
-  p.num_kst = (K + 255) / 256;
+  p.num_kst = (K + 2 * C::BKB - 1) / (2 * C::BKB);
   p.k_atoms = K / 64;
   p.sfb_atoms = (N + 127) / 128;
   p.g_a = g_a;
   p.g_w = w->gscale;
   p.alpha_mul = w->hadamard ? (1.0f / 128.0f) : 1.0f;
-  auto kern = k_gemm_w4a4<BN, STAGES, PAIR, ACC_, EPI_BUF, RES>;
+  auto kern = k_gemm_w4a4<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int units = std::min(p.num_tiles, num_sms() / C::CTAS);
   cudaLaunchConfig_t cfg{};

@@ -228,6 +228,47 @@ def nvfp4_dequantize(packed: np.ndarray, sb: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Activation decomposition (SemanticDialect, Methodology 2.2 "Activation
+# Decomposition": the activation is quantized, the quantization error -- the
+# residual -- is quantized again, and its product is added to the output).
+# Readings of what the page leaves open:
+#   * both parts are NVFP4 with the SAME fp32 tensor scale g (the tensor
+#     amax of h); the residual's own 16-element E4M3 block scales follow its
+#     smaller magnitude.  With one g the layer's product is one contraction
+#     over the K-concatenated pair [q1 | q2] against [W | W];
+#   * the residual is taken against the value the GEMM multiplies:
+#     v1 = RN(e2m1(q1) * RN(E4M3(sb1) * g)), r = RN(h - v1);
+#   * every token is decomposed (the page's attention-based salient-token
+#     selection needs attention maps and is not part of this layer).
+# ---------------------------------------------------------------------------
+
+def nvfp4_values(packed: np.ndarray, sb: np.ndarray, g) -> np.ndarray:
+    """fp32 [R, K]: RN(e2m1 value * RN(E4M3 block scale * g)) per element."""
+    q = unpack_nibbles(packed)
+    rows, k = q.shape
+    s = (e4m3_decode(sb) * np.float32(g)).astype(np.float32)            # RN(sb * g)
+    v = e2m1_decode(q).astype(np.float32).reshape(rows, k // NVFP4_BLOCK, NVFP4_BLOCK)
+    return (v * s[:, :, None]).astype(np.float32).reshape(rows, k)      # RN(value * s)
+
+
+def nvfp4_decompose(h: np.ndarray, g: np.float32 | None = None):
+    """h: fp32 [R, K].  Returns (packed uint8 [R, K] = [q1 (K/2 bytes) | q2
+    (K/2 bytes)], block scales uint8 [R, K/8] = [sb1 | sb2], g)."""
+    h = np.asarray(h, dtype=np.float32)
+    g = nvfp4_tensor_scale(h) if g is None else np.float32(g)
+    p1, s1, g = nvfp4_quantize(h, g)
+    r = (h - nvfp4_values(p1, s1, g)).astype(np.float32)               # RN(h - v1)
+    p2, s2, _ = nvfp4_quantize(r, g)
+    return np.concatenate([p1, p2], axis=1), np.concatenate([s1, s2], axis=1), g
+
+
+def decompose_weights(wq: dict) -> dict:
+    """NVFP4 weights repeated along K ([W | W]) to pair with decomposed activations."""
+    return dict(packed=np.concatenate([wq["packed"], wq["packed"]], axis=1),
+                sb=np.concatenate([wq["sb"], wq["sb"]], axis=1), g=wq["g"])
+
+
+# ---------------------------------------------------------------------------
 # a4: per-token INT8 (6Bit-Diffusion, Methodology B.1: INT8 for the blocks the
 # router marks sensitive; per-token granularity and symmetric +-127 range
 # are readings).  a10 activations: per-tensor INT8 (Q-ARVD, Technical
@@ -442,9 +483,15 @@ def prepare_weights_nvfp4(w_bits: np.ndarray, hadamard: bool = True):
     return dict(packed=packed, sb=sb, g=g)
 
 
+ROUTE_NVFP4_DECOMP = 4   # NVFP4 activations with the residual decomposition
+
+
 def quantize_activations(x_bits: np.ndarray, route: int, hadamard: bool = True):
     x = bf16_bits_to_f32(x_bits)
     h = block_hadamard(x) if hadamard else x
+    if route == ROUTE_NVFP4_DECOMP:
+        packed, sb, g = nvfp4_decompose(h)
+        return dict(packed=packed, sb=sb, g=g)
     if route == ROUTE_NVFP4:
         packed, sb, g = nvfp4_quantize(h)
         return dict(packed=packed, sb=sb, g=g)
@@ -455,6 +502,9 @@ def quantize_activations(x_bits: np.ndarray, route: int, hadamard: bool = True):
 def forward(x_bits, wq: dict, route: int, hadamard: bool = True, rows=None) -> np.ndarray:
     """Quantize the activations on the given route and multiply (fp64)."""
     aq = quantize_activations(x_bits, route, hadamard)
+    if route == ROUTE_NVFP4_DECOMP:
+        wd = decompose_weights(wq)
+        return gemm_w4a4(aq["packed"], aq["sb"], aq["g"], wd["packed"], wd["sb"], wd["g"], rows)
     if route == ROUTE_NVFP4:
         return gemm_w4a4(aq["packed"], aq["sb"], aq["g"], wq["packed"], wq["sb"], wq["g"], rows)
     return gemm_w4a8_token(aq["q"], aq["s"], wq["packed"], wq["sb"], wq["g"], hadamard, rows)
