@@ -172,9 +172,11 @@ ql_status check_mk(int64_t M, int64_t K) {
 }
 ql_status check_w(const ql_weights* w) {
   if (w == nullptr || w->codes == nullptr) return QL_ERR_INVALID_ARG;
-  if (w->fmt != QL_W_NVFP4 && w->fmt != QL_W_QARVD_INT4) return QL_ERR_INVALID_ARG;
+  if (w->fmt != QL_W_NVFP4 && w->fmt != QL_W_QARVD_INT4 && w->fmt != QL_W_NVFP4_DECOMP) return QL_ERR_INVALID_ARG;
   if (check_k(w->K) != QL_OK || w->N <= 0 || w->N % 16 != 0) return QL_ERR_UNSUPPORTED_SHAPE;
-  if (w->fmt == QL_W_NVFP4 && (w->sf == nullptr || w->gscale == nullptr)) return QL_ERR_INVALID_ARG;
+  if ((w->fmt == QL_W_NVFP4 || w->fmt == QL_W_NVFP4_DECOMP) && (w->sf == nullptr || w->gscale == nullptr))
+    return QL_ERR_INVALID_ARG;
+  if (w->fmt == QL_W_NVFP4_DECOMP && check_k(2 * w->K) != QL_OK) return QL_ERR_UNSUPPORTED_SHAPE;
   if (w->fmt == QL_W_QARVD_INT4 &&
       (w->gather == nullptr || w->kinfo == nullptr || w->s_norm == nullptr || w->s_out == nullptr ||
        w->Kp != qarvd_kp(w->K)))
@@ -202,9 +204,11 @@ struct Carver {  // sequential 256-byte aligned sub-buffers of one allocation
 // f16_codes: the INT8 route keeps its codes as f16 values (weights with an
 // f16 copy), 2 bytes per element.
 size_t forward_act_bytes(int64_t M, int32_t K, int32_t Kp, int32_t fmt, bool f16_codes = false) {
-  if (fmt == QL_ROUTE_NVFP4)
-    return kAmaxWsBytes + 256 + 256 + align256(static_cast<size_t>(M) * K / 2) +
-           align256(qlinear_sf_bytes(M, K));
+  if (fmt == QL_ROUTE_NVFP4 || fmt == QL_ACT_NVFP4_DECOMP) {
+    const int32_t kq = fmt == QL_ACT_NVFP4_DECOMP ? 2 * K : K;
+    return kAmaxWsBytes + 256 + 256 + align256(static_cast<size_t>(M) * kq / 2) +
+           align256(qlinear_sf_bytes(M, kq));
+  }
   if (fmt == QL_ROUTE_INT8)
     return align256(static_cast<size_t>(M) * K * (f16_codes ? 2 : 1)) + align256(4 * static_cast<size_t>(M));
   return kAmaxWsBytes + 256 + 256 + align256(static_cast<size_t>(M) * Kp);
@@ -258,6 +262,7 @@ size_t qlinear_weights_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg) {
   const size_t n = N, k = K;
   if (cfg->fmt == QL_W_NVFP4)
     return align256(n * k / 2) + align256(qlinear_sf_bytes(N, K)) + 256 + (cfg->expand_f16 ? align256(n * k * 2) : 0);
+  if (cfg->fmt == QL_W_NVFP4_DECOMP) return align256(n * k) + align256(qlinear_sf_bytes(N, 2 * K)) + 256;
   if (cfg->fmt == QL_W_QARVD_INT4) {
     const size_t kp = qarvd_kp(K);
     return align256(n * kp / 2) + align256(k) + align256(4 * k) + align256(4 * kp) + 256 +
@@ -269,6 +274,8 @@ size_t qlinear_weights_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg) {
 size_t qlinear_prepare_ws_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg) {
   if (cfg == nullptr || N <= 0 || check_k(K) != QL_OK) return 0;
   if (cfg->fmt == QL_W_NVFP4) return kAmaxWsBytes + 256;
+  if (cfg->fmt == QL_W_NVFP4_DECOMP)   // + the codes and scales of one copy before the repeat
+    return kAmaxWsBytes + 256 + align256(static_cast<size_t>(N) * K / 2) + align256(qlinear_sf_bytes(N, K));
   if (cfg->fmt == QL_W_QARVD_INT4) return align256(static_cast<size_t>(qarvd_slices(N)) * K * 8);
   return 0;
 }
@@ -278,9 +285,11 @@ ql_status qlinear_prepare_weights(const void* W, int32_t N, int32_t K, const ql_
                                   size_t ws_bytes, void* stream) {
   if (W == nullptr || cfg == nullptr || wbuf == nullptr || out == nullptr || ws == nullptr)
     return QL_ERR_INVALID_ARG;
-  if (cfg->fmt != QL_W_NVFP4 && cfg->fmt != QL_W_QARVD_INT4) return QL_ERR_INVALID_ARG;
-  if (cfg->fmt == QL_W_QARVD_INT4 && cfg->expand_f16 != 0) return QL_ERR_INVALID_ARG;
-  if (cfg->fmt == QL_W_NVFP4 && cfg->expand_i8 != 0) return QL_ERR_INVALID_ARG;
+  if (cfg->fmt != QL_W_NVFP4 && cfg->fmt != QL_W_QARVD_INT4 && cfg->fmt != QL_W_NVFP4_DECOMP)
+    return QL_ERR_INVALID_ARG;
+  if (cfg->fmt != QL_W_NVFP4 && cfg->expand_f16 != 0) return QL_ERR_INVALID_ARG;
+  if (cfg->fmt != QL_W_QARVD_INT4 && cfg->expand_i8 != 0) return QL_ERR_INVALID_ARG;
+  if (cfg->fmt == QL_W_NVFP4_DECOMP && check_k(2 * K) != QL_OK) return QL_ERR_UNSUPPORTED_SHAPE;
   QL_TRY(check_k(K));
   if (N <= 0 || N % 16 != 0 || N > (1 << 24)) return QL_ERR_UNSUPPORTED_SHAPE;
   QL_TRY(check_mk(N, K));
@@ -298,7 +307,31 @@ ql_status qlinear_prepare_weights(const void* W, int32_t N, int32_t K, const ql_
   w.N = N;
   w.K = K;
   Carver c{static_cast<uint8_t*>(wbuf)};
-  if (cfg->fmt == QL_W_NVFP4) {
+  if (cfg->fmt == QL_W_NVFP4_DECOMP) {
+    // quantize once into the workspace, then repeat along K: codes [c | c]
+    // per row; per 128-row group the scale atoms of K twice in a row
+    w.hadamard = cfg->hadamard ? 1 : 0;
+    w.codes = c.take<uint8_t>(static_cast<size_t>(N) * K);
+    w.sf = c.take<uint8_t>(qlinear_sf_bytes(N, 2 * K));
+    w.gscale = c.take<float>(256);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    float* amax = reinterpret_cast<float*>(wsb + kAmaxWsBytes);
+    uint8_t* tcodes = wsb + kAmaxWsBytes + 256;
+    uint8_t* tsf = tcodes + align256(static_cast<size_t>(N) * K / 2);
+    QL_TRY(launch_amax(W, N, K, w.hadamard, amax, ws, st));
+    QL_TRY(launch_quant_nvfp4(W, N, K, w.hadamard, amax, tcodes, tsf, nullptr, w.gscale, st));
+    const size_t half = static_cast<size_t>(K) / 2, group = static_cast<size_t>(K / 64) * 512;
+    const size_t groups = (static_cast<size_t>(N) + 127) / 128;
+    uint8_t* wc = static_cast<uint8_t*>(w.codes);
+    uint8_t* wf = static_cast<uint8_t*>(w.sf);
+    for (int part = 0; part < 2; ++part) {
+      if (cudaMemcpy2DAsync(wc + part * half, 2 * half, tcodes, half, half, N, cudaMemcpyDeviceToDevice, st) !=
+              cudaSuccess ||
+          cudaMemcpy2DAsync(wf + part * group, 2 * group, tsf, group, group, groups, cudaMemcpyDeviceToDevice,
+                            st) != cudaSuccess)
+        return QL_ERR_CUDA;
+    }
+  } else if (cfg->fmt == QL_W_NVFP4) {
     w.hadamard = cfg->hadamard ? 1 : 0;
     w.codes = c.take<uint8_t>(static_cast<size_t>(N) * K / 2);
     w.sf = c.take<uint8_t>(qlinear_sf_bytes(N, K));
@@ -352,11 +385,59 @@ ql_status qlinear_route(const void* in, const void* out, int64_t numel, float th
                             static_cast<cudaStream_t>(stream));
 }
 
+// ---------------------------------------------------------------- temporal delta cache
+namespace {
+bool tdc_params_ok(const ql_tdc_params* p) {
+  return p != nullptr && p->gamma_threshold == p->gamma_threshold && p->eps_threshold == p->eps_threshold &&
+         p->acc_max == p->acc_max && p->max_skips >= 0;
+}
+}  // namespace
+
+ql_status qlinear_tdc_init(ql_tdc_state* state_dev, void* stream) {
+  if (state_dev == nullptr) return QL_ERR_INVALID_ARG;
+  if (!aligned(state_dev, 8)) return QL_ERR_ALIGNMENT;
+  QL_TRY(device_ready());
+  return launch_tdc_init(state_dev, static_cast<cudaStream_t>(stream));
+}
+
+size_t qlinear_tdc_ws_bytes(int64_t numel) {
+  if (numel < 0) return 0;
+  return kTdcPartialBytes + 256;
+}
+
+ql_status qlinear_tdc_refresh(const void* in, const void* out, int64_t numel, void* delta0, void* delta1,
+                              ql_tdc_state* state_dev, const ql_tdc_params* params, void* ws, size_t ws_bytes,
+                              void* stream) {
+  if (numel < 0 || state_dev == nullptr || ws == nullptr || !tdc_params_ok(params)) return QL_ERR_INVALID_ARG;
+  if (numel > 0 && (in == nullptr || out == nullptr || delta0 == nullptr || delta1 == nullptr))
+    return QL_ERR_INVALID_ARG;
+  if (!aligned(in, 16) || !aligned(out, 16) || !aligned(delta0, 16) || !aligned(delta1, 16) ||
+      !aligned(state_dev, 8) || !aligned(ws, 256))
+    return QL_ERR_ALIGNMENT;
+  if (ws_bytes < qlinear_tdc_ws_bytes(numel)) return QL_ERR_WORKSPACE;
+  QL_TRY(device_ready());
+  return launch_tdc_refresh(in, out, numel, delta0, delta1, state_dev, *params, ws,
+                            static_cast<cudaStream_t>(stream));
+}
+
+ql_status qlinear_tdc_skip(const void* in, int64_t numel, const void* delta0, const void* delta1,
+                           ql_tdc_state* state_dev, const ql_tdc_params* params, void* out, void* stream) {
+  if (numel < 0 || state_dev == nullptr || !tdc_params_ok(params)) return QL_ERR_INVALID_ARG;
+  if (numel > 0 && (in == nullptr || out == nullptr || delta0 == nullptr || delta1 == nullptr))
+    return QL_ERR_INVALID_ARG;
+  if (!aligned(in, 16) || !aligned(out, 16) || !aligned(delta0, 16) || !aligned(delta1, 16) ||
+      !aligned(state_dev, 8))
+    return QL_ERR_ALIGNMENT;
+  QL_TRY(device_ready());
+  return launch_tdc_skip(in, numel, delta0, delta1, state_dev, *params, out, status_word(),
+                         static_cast<cudaStream_t>(stream));
+}
+
 // ---------------------------------------------------------------- activations
 size_t qlinear_quantize_ws_bytes(int64_t M, int32_t K, int32_t act_fmt) {
   if (M < 0 || check_k(K) != QL_OK) return 0;
   if (act_fmt != QL_ROUTE_NVFP4 && act_fmt != QL_ROUTE_INT8 && act_fmt != QL_ACT_INT8_TENSOR &&
-      act_fmt != QL_ACT_INT8_F16)
+      act_fmt != QL_ACT_INT8_F16 && act_fmt != QL_ACT_NVFP4_DECOMP)
     return 0;
   return kAmaxWsBytes + 256;
 }
@@ -382,7 +463,7 @@ ql_status qlinear_quantize_act(const void* X, int64_t M, int32_t K, int32_t act_
   QL_TRY(check_mk(M, K));
   if (codes == nullptr || scales == nullptr || ws == nullptr || (M > 0 && X == nullptr))
     return QL_ERR_INVALID_ARG;
-  if (act_fmt == QL_ROUTE_NVFP4) {
+  if (act_fmt == QL_ROUTE_NVFP4 || act_fmt == QL_ACT_NVFP4_DECOMP) {
     if (sf_mma == nullptr) return QL_ERR_INVALID_ARG;
   } else if (act_fmt == QL_ACT_INT8_TENSOR) {
     QL_TRY(check_w(w));
@@ -405,8 +486,9 @@ ql_status qlinear_quantize_act(const void* X, int64_t M, int32_t K, int32_t act_
     QL_TRY(launch_amax(X, M, K, had, slot, ws, st));
     amax = slot;
   }
-  if (act_fmt == QL_ROUTE_NVFP4)
-    return launch_quant_nvfp4(X, M, K, had, amax, codes, sf_mma, sf_rowmajor, scales, st);
+  if (act_fmt == QL_ROUTE_NVFP4 || act_fmt == QL_ACT_NVFP4_DECOMP)
+    return launch_quant_nvfp4(X, M, K, had, amax, codes, sf_mma, sf_rowmajor, scales, st,
+                              act_fmt == QL_ACT_NVFP4_DECOMP ? 1 : 0);
   return launch_quant_int8_tensor_perm(X, M, K, w->Kp, w->gather, amax, codes, scales, st);
 }
 
@@ -422,6 +504,8 @@ ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf, c
     if (act_fmt == QL_ROUTE_NVFP4 && M > 0 && a_sf == nullptr) return QL_ERR_INVALID_ARG;
   } else if (act_fmt == QL_ACT_INT8_TENSOR) {
     if (w->fmt != QL_W_QARVD_INT4) return QL_ERR_INVALID_ARG;
+  } else if (act_fmt == QL_ACT_NVFP4_DECOMP) {
+    if (w->fmt != QL_W_NVFP4_DECOMP || (M > 0 && a_sf == nullptr)) return QL_ERR_INVALID_ARG;
   } else {
     return QL_ERR_INVALID_ARG;
   }
@@ -433,6 +517,11 @@ ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf, c
   int* status = status_word();
   if (act_fmt == QL_ROUTE_NVFP4)
     return launch_gemm_w4a4(a_codes, static_cast<const uint8_t*>(a_sf), a_scales, M, w, Y, st, status);
+  if (act_fmt == QL_ACT_NVFP4_DECOMP) {   // one W4A4 contraction over K' = 2K
+    ql_weights w2 = *w;
+    w2.K = 2 * w->K;
+    return launch_gemm_w4a4(a_codes, static_cast<const uint8_t*>(a_sf), a_scales, M, &w2, Y, st, status);
+  }
   if (act_fmt == QL_ROUTE_INT8) return launch_gemm_w4a8(a_codes, a_scales, M, w, Y, st, status);
   if (act_fmt == QL_ACT_INT8_F16) return launch_gemm_w4a8(a_codes, a_scales, M, w, Y, st, status, 1);
   return launch_gemm_qarvd(a_codes, a_scales, M, w, Y, st, status);
@@ -442,6 +531,8 @@ ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf, c
 size_t qlinear_forward_ws_bytes(int64_t M, const ql_weights* w, int32_t route) {
   if (M < 0 || check_w(w) != QL_OK) return 0;
   if (w->fmt == QL_W_QARVD_INT4) return forward_act_bytes(M, w->K, w->Kp, QL_ACT_INT8_TENSOR);
+  if (w->fmt == QL_W_NVFP4_DECOMP)
+    return route == QL_ROUTE_NVFP4 ? forward_act_bytes(M, w->K, 0, QL_ACT_NVFP4_DECOMP) : 0;
   if (route != QL_ROUTE_NVFP4 && route != QL_ROUTE_INT8) return 0;
   return forward_act_bytes(M, w->K, 0, route, w->w16 != nullptr);
 }
@@ -452,8 +543,12 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
   QL_TRY(check_w(w));
   QL_TRY(check_mk(M, w->K));
   if (ws == nullptr || (M > 0 && (X == nullptr || Y == nullptr))) return QL_ERR_INVALID_ARG;
-  const int32_t fmt = (w->fmt == QL_W_QARVD_INT4) ? int32_t(QL_ACT_INT8_TENSOR) : route;
-  if (fmt != QL_ROUTE_NVFP4 && fmt != QL_ROUTE_INT8 && fmt != QL_ACT_INT8_TENSOR) return QL_ERR_INVALID_ARG;
+  if (w->fmt == QL_W_NVFP4_DECOMP && route != QL_ROUTE_NVFP4) return QL_ERR_INVALID_ARG;
+  const int32_t fmt = (w->fmt == QL_W_QARVD_INT4)     ? int32_t(QL_ACT_INT8_TENSOR)
+                      : (w->fmt == QL_W_NVFP4_DECOMP) ? int32_t(QL_ACT_NVFP4_DECOMP)
+                                                      : route;
+  if (fmt != QL_ROUTE_NVFP4 && fmt != QL_ROUTE_INT8 && fmt != QL_ACT_INT8_TENSOR && fmt != QL_ACT_NVFP4_DECOMP)
+    return QL_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256)) return QL_ERR_ALIGNMENT;
   if (ws_bytes < qlinear_forward_ws_bytes(M, w, route)) return QL_ERR_WORKSPACE;
   QL_TRY(device_ready());
@@ -462,15 +557,19 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
   const int K = w->K;
   Carver c{static_cast<uint8_t*>(ws)};
   int* status = status_word();
-  if (fmt == QL_ROUTE_NVFP4) {
+  if (fmt == QL_ROUTE_NVFP4 || fmt == QL_ACT_NVFP4_DECOMP) {
+    const int decomp = fmt == QL_ACT_NVFP4_DECOMP ? 1 : 0;
+    const int kq = decomp ? 2 * K : K;
     void* aws = c.take<uint8_t>(kAmaxWsBytes);
     float* amax = c.take<float>(256);
     float* g = c.take<float>(256);
-    uint8_t* codes = c.take<uint8_t>(static_cast<size_t>(M) * K / 2);
-    uint8_t* sf = c.take<uint8_t>(qlinear_sf_bytes(M, K));
+    uint8_t* codes = c.take<uint8_t>(static_cast<size_t>(M) * kq / 2);
+    uint8_t* sf = c.take<uint8_t>(qlinear_sf_bytes(M, kq));
     QL_TRY(launch_amax(X, M, K, w->hadamard, amax, aws, st));
-    QL_TRY(launch_quant_nvfp4(X, M, K, w->hadamard, amax, codes, sf, nullptr, g, st));
-    return launch_gemm_w4a4(codes, sf, g, M, w, Y, st, status);
+    QL_TRY(launch_quant_nvfp4(X, M, K, w->hadamard, amax, codes, sf, nullptr, g, st, decomp));
+    ql_weights w2 = *w;
+    w2.K = kq;
+    return launch_gemm_w4a4(codes, sf, g, M, &w2, Y, st, status);
   }
   if (fmt == QL_ROUTE_INT8) {
     // with an f16 weight copy the codes are written as f16 values and both

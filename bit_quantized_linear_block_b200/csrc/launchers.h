@@ -15,6 +15,7 @@ constexpr int kMaxPartials = 4096;               // upper bound of any streaming
 constexpr size_t kAmaxPartialBytes = kMaxPartials * sizeof(float);
 constexpr size_t kAmaxWsBytes = kAmaxPartialBytes + 256;   // partials + ticket
 constexpr size_t kRoutePartialBytes = 2 * kMaxPartials * sizeof(double);
+constexpr size_t kTdcPartialBytes = 4 * kMaxPartials * sizeof(double);
 
 int num_sms();
 bool set_smem_attr(const void* kernel, int bytes);
@@ -25,8 +26,11 @@ int qarvd_slices(int32_t N);
 // kAmaxWsBytes (partials + ticket).
 ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* amax_out, void* ws,
                       cudaStream_t st);
+// decomp = 1: activation decomposition, codes [M, K] bytes = [q1 | q2] per
+// row and scales over K' = 2K.
 ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, const float* amax_in,
-                             void* codes, void* sf_mma, void* sf_rm, float* g_out, cudaStream_t st);
+                             void* codes, void* sf_mma, void* sf_rm, float* g_out, cudaStream_t st,
+                             int decomp = 0);
 // f16 copy [N, K] of NVFP4 weights without the tensor scale (INT8 route).
 ql_status launch_expand_nvfp4_f16(const void* codes, const void* sf, int32_t N, int32_t K, void* out,
                                   cudaStream_t st);
@@ -40,6 +44,12 @@ ql_status launch_gamma_route(const void* in, const void* out, int64_t numel, flo
                              double* gamma, int32_t* route, void* ws, cudaStream_t st);
 ql_status launch_qarvd_prepare(const void* W, int32_t N, int32_t K, float tau, float alpha,
                                const ql_weights* w, void* ws, cudaStream_t st);
+
+ql_status launch_tdc_init(ql_tdc_state* st, cudaStream_t s);
+ql_status launch_tdc_refresh(const void* in, const void* out, int64_t numel, void* slot0, void* slot1,
+                             ql_tdc_state* st, const ql_tdc_params& prm, void* ws, cudaStream_t s);
+ql_status launch_tdc_skip(const void* in, int64_t numel, const void* slot0, const void* slot1,
+                          ql_tdc_state* st, const ql_tdc_params& prm, void* out, int* status, cudaStream_t s);
 
 ql_status launch_gemm_w4a4(const void* a_codes, const uint8_t* a_sf, const float* g_a, int64_t M,
                            const ql_weights* w, void* Y, cudaStream_t st, int* status);

@@ -223,6 +223,47 @@ __device__ __forceinline__ uint32_t e2m1x8(float a0, float a1, float a2, float a
   return r;
 }
 
+// E2M1 code (bits 0-3: sign bit 3, magnitude code 0..7) -> its fp32 value
+// {0, 0.5, 1, 1.5, 2, 3, 4, 6} with the sign (code 8 is -0).
+__device__ __forceinline__ float e2m1_to_f32(uint32_t code) {
+  const uint32_t m = code & 7u;
+  uint32_t bits = (m >= 2u) ? ((((m >> 1) + 126u) << 23) | ((m & 1u) << 22)) : (m ? 0x3F000000u : 0u);
+  bits |= (code & 8u) << 28;
+  return __uint_as_float(bits);
+}
+
+// NVFP4 of one half block (64 values in the pair layout: 16-element blocks
+// b = 0, 1 in P[16b..16b+15].x, b = 2, 3 in the .y halves).  Writes the four
+// E4M3 scales, the codes (cw[i]: elements 8i .. 8i+7 of the half) and each
+// block's RN(E4M3 value * g) (den[b] for blocks b and b + 2).
+__device__ __forceinline__ void nvfp4_half(const float2 (&P)[32], float g, float d, uint32_t (&sb)[4],
+                                           uint32_t (&cw)[8], float2 (&den)[2]) {
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int t = 0; t < 16; t += 2) {
+      a.x = fmax3(a.x, fabsf(P[16 * b + t].x), fabsf(P[16 * b + t + 1].x));
+      a.y = fmax3(a.y, fabsf(P[16 * b + t].y), fabsf(P[16 * b + t + 1].y));
+    }
+    sb[b] = e4m3_code(__fdiv_rn(a.x, d));
+    sb[b + 2] = e4m3_code(__fdiv_rn(a.y, d));
+    den[b] = make_float2(__fmul_rn(e4m3_value(sb[b]), g), __fmul_rn(e4m3_value(sb[b + 2]), g));
+    const float2 inv = make_float2(sb[b] ? __frcp_rn(den[b].x) : 0.f, sb[b + 2] ? __frcp_rn(den[b].y) : 0.f);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = 16 * b + 8 * h;
+      float2 y[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) y[t] = __fmul2_rn(P[j + t], inv);
+      const uint32_t lo = e2m1x8(y[0].x, y[1].x, y[2].x, y[3].x, y[4].x, y[5].x, y[6].x, y[7].x);
+      const uint32_t hi = e2m1x8(y[0].y, y[1].y, y[2].y, y[3].y, y[4].y, y[5].y, y[6].y, y[7].y);
+      cw[2 * b + h] = sb[b] ? lo : 0u;           // all-zero block -> +0 codes
+      cw[4 + 2 * b + h] = sb[b + 2] ? hi : 0u;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // NVFP4 quantizer.  g = amax / 2688 (1 if amax == 0) from the device amax.
 // Per 16-element block: sb = E4M3(RN(amax_b / RN(6 g))); if sb == 0 all
@@ -231,10 +272,17 @@ __device__ __forceinline__ uint32_t e2m1x8(float a0, float a1, float a2, float a
 // and two in the .y halves of its registers, so two blocks are scaled by one
 // packed multiply.  Rows M .. Mpad-1 (padding of the last
 // 128-row atom) get zero scales.
+//
+// DECOMP (activation decomposition, SemanticDialect, Methodology 2.2): the
+// residual r = RN(h - RN(e2m1(q1) * RN(sb1 * g))) is quantized again with
+// the same g; a row of the output holds [q1 | q2] (K/2 bytes each) and its
+// scales cover K' = 2K (q1's at scale indices 0 .. K/16-1, q2's after them),
+// the operand of a W4A4 GEMM over K' against the weights repeated along K.
 // ---------------------------------------------------------------------------
+template <bool DECOMP>
 __global__ void __launch_bounds__(kQuantThreads, 1)
     k_quant_nvfp4(const uint8_t* __restrict__ x, int64_t M, int32_t K, int hadamard,
-                  const float* __restrict__ amax_in, uint4* __restrict__ codes,
+                  const float* __restrict__ amax_in, uint8_t* __restrict__ codes,
                   uint8_t* __restrict__ sf_mma, uint8_t* __restrict__ sf_rm,
                   float* __restrict__ g_out) {
   extern __shared__ __align__(128) uint8_t ring_all[];
@@ -243,58 +291,58 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   if (blockIdx.x == 0 && threadIdx.x == 0 && g_out != nullptr) *g_out = g;
   const float d = __fmul_rn(6.f, g);
   const uint32_t upr = static_cast<uint32_t>(K >> 7);
-  const int32_t k_atoms = K >> 6;
+  const int32_t kq = DECOMP ? 2 * K : K;           // K of the quantized operand
+  const int32_t k_atoms = kq >> 6;
+  const int64_t row_bytes = kq >> 1;
   const int64_t units = M * upr;
   const int64_t halves = 2 * units;
   stream_blocks<kQuantWarps>(x, M * K * 2, hadamard, ring_all, [&](float2 (&P)[32], int64_t hu) {
     if (hu >= halves) return;
-    // 16-element blocks of this half: b = 0, 1 in P[16b..16b+15].x, b = 2, 3
-    // in the .y halves of the same registers.
-    uint32_t sb[4];
-    uint32_t cw[8];   // codes of elements 8i .. 8i+7 of this half in cw[i]
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      float2 a = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int t = 0; t < 16; t += 2) {
-        a.x = fmax3(a.x, fabsf(P[16 * b + t].x), fabsf(P[16 * b + t + 1].x));
-        a.y = fmax3(a.y, fabsf(P[16 * b + t].y), fabsf(P[16 * b + t + 1].y));
-      }
-      sb[b] = e4m3_code(__fdiv_rn(a.x, d));
-      sb[b + 2] = e4m3_code(__fdiv_rn(a.y, d));
-      const float2 inv = make_float2(sb[b] ? __frcp_rn(__fmul_rn(e4m3_value(sb[b]), g)) : 0.f,
-                                     sb[b + 2] ? __frcp_rn(__fmul_rn(e4m3_value(sb[b + 2]), g)) : 0.f);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int j = 16 * b + 8 * h;
-        float2 y[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) y[t] = __fmul2_rn(P[j + t], inv);
-        const uint32_t lo = e2m1x8(y[0].x, y[1].x, y[2].x, y[3].x, y[4].x, y[5].x, y[6].x, y[7].x);
-        const uint32_t hi = e2m1x8(y[0].y, y[1].y, y[2].y, y[3].y, y[4].y, y[5].y, y[6].y, y[7].y);
-        cw[2 * b + h] = sb[b] ? lo : 0u;           // all-zero block -> +0 codes
-        cw[4 + 2 * b + h] = sb[b + 2] ? hi : 0u;
-      }
-    }
-    uint4* dst = codes + hu * 2;
-    dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-    dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-    // half index -> (row, first scale index); 32-bit division (units < 2^32)
+    // half index -> (row, first scale index, first code byte); 32-bit division (units < 2^32)
     const uint32_t u = static_cast<uint32_t>(hu >> 1);
     const uint32_t row = u / upr;
     const uint32_t j0 = (u - row * upr) * 8 + (static_cast<uint32_t>(hu) & 1u) * 4;
-    const uint32_t sw = sb[0] | (sb[1] << 8) | (sb[2] << 16) | (sb[3] << 24);
-    *reinterpret_cast<uint32_t*>(sf_mma + sf_mma_offset(row, j0, k_atoms)) = sw;
-    if (sf_rm != nullptr) *reinterpret_cast<uint32_t*>(sf_rm + static_cast<size_t>(row) * (K >> 4) + j0) = sw;
+    uint8_t* cdst = codes + static_cast<int64_t>(row) * row_bytes + j0 * 8;
+    uint32_t sb[4], cw[8];
+    float2 den[2];
+    nvfp4_half(P, g, d, sb, cw, den);
+    auto store = [&](int part) {
+      uint4* dst = reinterpret_cast<uint4*>(cdst + part * (K >> 1));
+      dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      const uint32_t j = j0 + part * (K >> 4);
+      const uint32_t sw = sb[0] | (sb[1] << 8) | (sb[2] << 16) | (sb[3] << 24);
+      *reinterpret_cast<uint32_t*>(sf_mma + sf_mma_offset(row, j, k_atoms)) = sw;
+      if (sf_rm != nullptr) *reinterpret_cast<uint32_t*>(sf_rm + static_cast<size_t>(row) * (kq >> 4) + j) = sw;
+    };
+    store(0);
+    if constexpr (DECOMP) {
+      // residual in place: P <- RN(P - RN(e2m1(q1) * den))
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int j = 16 * b + 8 * h;
+          const uint32_t lo = cw[2 * b + h], hi = cw[4 + 2 * b + h];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            P[j + t].x = __fsub_rn(P[j + t].x, __fmul_rn(e2m1_to_f32(lo >> (4 * t)), den[b].x));
+            P[j + t].y = __fsub_rn(P[j + t].y, __fmul_rn(e2m1_to_f32(hi >> (4 * t)), den[b].y));
+          }
+        }
+      }
+      nvfp4_half(P, g, d, sb, cw, den);
+      store(1);
+    }
   });
   // zero scales of the padding rows of the last 128-row atom
   const int64_t mpad = (M + 127) & ~int64_t(127);
-  const int64_t pad_words = (mpad - M) * (K >> 6);
+  const int64_t pad_words = (mpad - M) * k_atoms;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < pad_words;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = M + i / (K >> 6);
-    const int32_t j0 = static_cast<int32_t>(i % (K >> 6)) * 4;
-    *reinterpret_cast<uint32_t*>(sf_mma + sf_mma_offset(row, j0, k_atoms)) = 0u;
+    const int64_t row = M + i / k_atoms;
+    const int32_t j = static_cast<int32_t>(i % k_atoms) * 4;
+    *reinterpret_cast<uint32_t*>(sf_mma + sf_mma_offset(row, j, k_atoms)) = 0u;
   }
 }
 
@@ -532,15 +580,16 @@ ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* 
 }
 
 ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, const float* amax_in,
-                             void* codes, void* sf_mma, void* sf_rm, float* g_out, cudaStream_t st) {
+                             void* codes, void* sf_mma, void* sf_rm, float* g_out, cudaStream_t st, int decomp) {
   if (M == 0) return QL_OK;
   const int64_t nchunks = (M * K * 2 + kChunkBytes - 1) / kChunkBytes;
   const int grid = static_cast<int>(std::max<int64_t>(
       1, std::min<int64_t>((nchunks + kQuantWarps - 1) / kQuantWarps, num_sms())));
-  if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_nvfp4), kQuantRingBytes)) return QL_ERR_CUDA;
-  k_quant_nvfp4<<<grid, kQuantThreads, kQuantRingBytes, st>>>(
-      static_cast<const uint8_t*>(x), M, K, hadamard, amax_in, static_cast<uint4*>(codes),
-      static_cast<uint8_t*>(sf_mma), static_cast<uint8_t*>(sf_rm), g_out);
+  auto kern = decomp ? k_quant_nvfp4<true> : k_quant_nvfp4<false>;
+  if (!set_smem_attr(reinterpret_cast<const void*>(kern), kQuantRingBytes)) return QL_ERR_CUDA;
+  kern<<<grid, kQuantThreads, kQuantRingBytes, st>>>(static_cast<const uint8_t*>(x), M, K, hadamard, amax_in,
+                                                     static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf_mma),
+                                                     static_cast<uint8_t*>(sf_rm), g_out);
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 

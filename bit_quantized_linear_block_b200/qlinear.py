@@ -23,10 +23,12 @@ STATUS_NAMES = {0: "QL_OK", 1: "QL_ERR_INVALID_ARG", 2: "QL_ERR_UNSUPPORTED_SHAP
                 6: "QL_ERR_WORKSPACE", 7: "QL_ERR_NO_DEVICE"}
 QL_W_NVFP4 = 0
 QL_W_QARVD_INT4 = 2
+QL_W_NVFP4_DECOMP = 3
 QL_ROUTE_NVFP4 = 0
 QL_ROUTE_INT8 = 1
 QL_ACT_INT8_TENSOR = 2
 QL_ACT_INT8_F16 = 3
+QL_ACT_NVFP4_DECOMP = 4
 
 
 class WeightCfg(C.Structure):
@@ -41,6 +43,18 @@ class Weights(C.Structure):
                 ("outlier_mask", C.c_void_p), ("perm", C.c_void_p), ("gather", C.c_void_p),
                 ("kinfo", C.c_void_p), ("s_norm", C.c_void_p), ("s_out", C.c_void_p),
                 ("norms", C.c_void_p), ("w16", C.c_void_p), ("w8", C.c_void_p)]
+
+
+class TdcState(C.Structure):
+    _fields_ = [("gamma", C.c_double), ("eps", C.c_double), ("acc", C.c_double),
+                ("n_delta", C.c_int32), ("cur", C.c_int32), ("skips", C.c_int32), ("last_skipped", C.c_int32),
+                ("next_skip", C.c_int32), ("next_route", C.c_int32), ("steps", C.c_int32),
+                ("reserved", C.c_int32)]
+
+
+class TdcParams(C.Structure):
+    _fields_ = [("gamma_threshold", C.c_float), ("eps_threshold", C.c_float), ("acc_max", C.c_float),
+                ("max_skips", C.c_int32)]
 
 
 class QLinearError(RuntimeError):
@@ -74,6 +88,10 @@ def _load() -> C.CDLL:
         "qlinear_gemm": (C.c_int, [i32, vp, vp, vp, i64, C.POINTER(Weights), vp, vp]),
         "qlinear_forward_ws_bytes": (sz, [i64, C.POINTER(Weights), i32]),
         "qlinear_forward": (C.c_int, [vp, i64, C.POINTER(Weights), i32, vp, vp, sz, vp]),
+        "qlinear_tdc_init": (C.c_int, [vp, vp]),
+        "qlinear_tdc_ws_bytes": (sz, [i64]),
+        "qlinear_tdc_refresh": (C.c_int, [vp, vp, i64, vp, vp, vp, C.POINTER(TdcParams), vp, sz, vp]),
+        "qlinear_tdc_skip": (C.c_int, [vp, i64, vp, vp, vp, C.POINTER(TdcParams), vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -134,7 +152,8 @@ def qlinear_prepare_weights(W: torch.Tensor, fmt: int = QL_W_NVFP4, hadamard: bo
     INT4 codes sign-extended to int8 for the Q-ARVD GEMM."""
     assert W.dtype == torch.bfloat16 and W.is_cuda and W.dim() == 2 and W.is_contiguous()
     N, K = W.shape
-    cfg = WeightCfg(fmt, int(bool(hadamard)) if fmt == QL_W_NVFP4 else 0, tau, alpha, int(bool(expand_f16)),
+    cfg = WeightCfg(fmt, int(bool(hadamard)) if fmt in (QL_W_NVFP4, QL_W_NVFP4_DECOMP) else 0, tau, alpha,
+                    int(bool(expand_f16)),
                     int(bool(expand_i8)))
     wbytes = lib.qlinear_weights_bytes(N, K, C.byref(cfg))
     wsbytes = lib.qlinear_prepare_ws_bytes(N, K, C.byref(cfg))
@@ -203,11 +222,12 @@ def qlinear_quantize_act(X: torch.Tensor, act_fmt: int, hadamard: bool = True,
         return out
     out = {}
     sf_mma = sf_rm = None
-    if act_fmt == QL_ROUTE_NVFP4:
-        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
-        sf_mma = _bytes(lib.qlinear_sf_bytes(M, K), dev)
+    if act_fmt in (QL_ROUTE_NVFP4, QL_ACT_NVFP4_DECOMP):
+        kq = 2 * K if act_fmt == QL_ACT_NVFP4_DECOMP else K     # decomposed: [q1 | q2] per row
+        codes = torch.empty((M, kq // 2), dtype=torch.uint8, device=dev)
+        sf_mma = _bytes(lib.qlinear_sf_bytes(M, kq), dev)
         if rowmajor_scales:
-            sf_rm = torch.empty((M, K // 16), dtype=torch.uint8, device=dev)
+            sf_rm = torch.empty((M, kq // 16), dtype=torch.uint8, device=dev)
         scales = torch.empty(1, dtype=torch.float32, device=dev)
     elif act_fmt == QL_ROUTE_INT8:
         codes = torch.empty((M, K), dtype=torch.int8, device=dev)
@@ -262,6 +282,59 @@ def qlinear_forward(X: torch.Tensor, w: PackedWeights, route: int = QL_ROUTE_NVF
            lib.qlinear_forward(_ptr(X), M, C.byref(w.desc), route, _ptr(Y), _ptr(plan.ws),
                                plan.ws.numel(), _stream(stream)))
     return Y
+
+
+# ----------------------------------------------------------------------------
+# Temporal delta cache
+# ----------------------------------------------------------------------------
+
+class TdcCache:
+    """Device buffers of one block's delta cache: two bf16 delta slots, the
+    state (read with ``state()``) and the refresh workspace."""
+
+    def __init__(self, numel: int, device, gamma_threshold=0.05, eps_threshold=0.1, acc_max=0.3,
+                 max_skips=3, stream=None):
+        self.numel = int(numel)
+        # each slot starts on a 16-byte boundary
+        self.slots = torch.empty(2, max(8, (self.numel + 7) // 8 * 8), dtype=torch.bfloat16, device=device)
+        self.state_buf = torch.zeros(C.sizeof(TdcState), dtype=torch.uint8, device=device)
+        self.ws = _bytes(lib.qlinear_tdc_ws_bytes(self.numel), device)
+        self.params = TdcParams(gamma_threshold, eps_threshold, acc_max, int(max_skips))
+        qlinear_tdc_init(self, stream)
+
+    def state(self) -> TdcState:
+        """Host copy of the device state (synchronizes with the device)."""
+        return TdcState.from_buffer_copy(bytes(self.state_buf.cpu().numpy()))
+
+    def delta(self, which: str = "latest") -> torch.Tensor:
+        st = self.state()
+        i = st.cur if which == "latest" else 1 - st.cur
+        return self.slots[i, :self.numel]
+
+
+def qlinear_tdc_init(cache: TdcCache, stream=None):
+    _check("qlinear_tdc_init", lib.qlinear_tdc_init(_ptr(cache.state_buf), _stream(stream)))
+
+
+def qlinear_tdc_refresh(inp: torch.Tensor, out: torch.Tensor, cache: TdcCache, stream=None):
+    """After computing the block: new delta, Gamma, E and the next decision (on the device)."""
+    assert inp.dtype == torch.bfloat16 and out.dtype == torch.bfloat16 and inp.shape == out.shape
+    assert inp.is_contiguous() and out.is_contiguous() and inp.numel() == cache.numel
+    _check("qlinear_tdc_refresh",
+           lib.qlinear_tdc_refresh(_ptr(inp), _ptr(out), cache.numel, _ptr(cache.slots[0]), _ptr(cache.slots[1]),
+                                   _ptr(cache.state_buf), C.byref(cache.params), _ptr(cache.ws), cache.ws.numel(),
+                                   _stream(stream)))
+
+
+def qlinear_tdc_skip(inp: torch.Tensor, cache: TdcCache, out: torch.Tensor | None = None, stream=None):
+    """Skip the block: out = bf16(in + latest delta)."""
+    assert inp.dtype == torch.bfloat16 and inp.is_contiguous() and inp.numel() == cache.numel
+    if out is None:
+        out = torch.empty_like(inp)
+    _check("qlinear_tdc_skip",
+           lib.qlinear_tdc_skip(_ptr(inp), cache.numel, _ptr(cache.slots[0]), _ptr(cache.slots[1]),
+                                _ptr(cache.state_buf), C.byref(cache.params), _ptr(out), _stream(stream)))
+    return out
 
 
 def qlinear_device_status(stream=None) -> int:

@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define QLINEAR_ABI_VERSION 3
+#define QLINEAR_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define QL_API __attribute__((visibility("default")))
@@ -82,7 +82,10 @@ typedef enum {
 /* Weight formats. */
 typedef enum {
   QL_W_NVFP4 = 0,       /* NVFP4 (E2M1 + E4M3/16 + fp32), optional Hadamard  */
-  QL_W_QARVD_INT4 = 2   /* Q-ARVD dual-scale signed INT4, K permuted         */
+  QL_W_QARVD_INT4 = 2,  /* Q-ARVD dual-scale signed INT4, K permuted         */
+  QL_W_NVFP4_DECOMP = 3 /* NVFP4 repeated along K for decomposed activations:
+                           codes [N, K] bytes = [c | c] per row, scales over
+                           2K; pairs only with QL_ACT_NVFP4_DECOMP           */
 } ql_weight_format;
 
 /* Activation routes / formats. */
@@ -90,9 +93,15 @@ typedef enum {
   QL_ROUTE_NVFP4 = 0,       /* W4A4: NVFP4 activations                       */
   QL_ROUTE_INT8 = 1,        /* W4A8: per-token INT8 activations              */
   QL_ACT_INT8_TENSOR = 2,   /* Q-ARVD: per-tensor INT8, permuted K           */
-  QL_ACT_INT8_F16 = 3       /* W4A8: per-token INT8 codes stored as the equal
+  QL_ACT_INT8_F16 = 3,      /* W4A8: per-token INT8 codes stored as the equal
                                f16 values, f16 [M, K]; the GEMM needs weights
                                prepared with expand_f16                      */
+  QL_ACT_NVFP4_DECOMP = 4   /* activation decomposition (SemanticDialect,
+                               Methodology 2.2): NVFP4 of h, then NVFP4 of the
+                               residual r = RN(h - RN(e2m1(q1) RN(sb1 g))) with
+                               the same tensor scale g; codes [M, K] bytes =
+                               [q1 | q2] per row, scales over K' = 2K (q1's
+                               first); the GEMM needs QL_W_NVFP4_DECOMP      */
 } ql_act_format;
 
 typedef struct {
@@ -256,6 +265,66 @@ QL_API size_t qlinear_forward_ws_bytes(int64_t M, const ql_weights* w, int32_t r
 QL_API ql_status qlinear_forward(const void* X_bf16, int64_t M, const ql_weights* w,
                           int32_t route, void* Y_bf16,
                           void* ws, size_t ws_bytes, void* stream);
+
+/* ---- temporal delta cache ------------------------------------------------
+   "6Bit-Diffusion", Methodology A.2 / B.2 (TDC) and B.3 (PDR).  A block's
+   residual delta D = bf16(out - in) changes little between adjacent
+   timesteps; a block whose last two computed deltas are close is skipped
+   and reuses the latest delta.  The caller owns, per transformer block, two
+   bf16 delta slots of the block's activation size and one ql_tdc_state in
+   device memory.  Each step it reads next_skip (and next_route) from the
+   state -- written by the previous step's kernel -- and either computes
+   the block and calls qlinear_tdc_refresh, or calls qlinear_tdc_skip.
+
+   Definitions (fp32 differences of bf16 values, RN; fp64 sums):
+     Gamma = sum |out - in| / sum |in|                  (+inf if sum |in| = 0)
+     E     = sum |D_new - D_prev| / sum |D_prev|        (+inf with < 2 deltas
+                                                          or sum |D_prev| = 0)
+     skip next   iff n_delta == 2, E < eps_threshold, acc + E <= acc_max and
+                 skips < max_skips  (acc sums E over the current run of skips)
+     next_route  INT8 if the step just taken was a skip or Gamma >
+                 gamma_threshold (strict), else NVFP4; INT8 before any Gamma. */
+typedef struct {
+  double gamma;          /* Gamma of the last computed step                   */
+  double eps;            /* E between the two cached deltas                   */
+  double acc;            /* summed E over the current run of skips            */
+  int32_t n_delta;       /* cached deltas, 0..2                               */
+  int32_t cur;           /* slot (0 or 1) holding the latest delta            */
+  int32_t skips;         /* consecutive skips so far                          */
+  int32_t last_skipped;  /* 1 when the last step was a skip                   */
+  int32_t next_skip;     /* decision for the next step: 1 = skip              */
+  int32_t next_route;    /* QL_ROUTE_* of the next step if it is computed     */
+  int32_t steps;         /* steps taken since qlinear_tdc_init                */
+  int32_t reserved;
+} ql_tdc_state;
+
+typedef struct {
+  float gamma_threshold; /* DMPQ route threshold (0.05)                       */
+  float eps_threshold;   /* skip while E is below this                        */
+  float acc_max;         /* cap on the summed E of one run of skips           */
+  int32_t max_skips;     /* cap on consecutive skips (>= 0)                   */
+} ql_tdc_params;
+
+/* Reset a block's cache state (device pointer, 8-byte aligned): no deltas,
+   Gamma = E = +inf, next step computed on the INT8 route. */
+QL_API ql_status qlinear_tdc_init(ql_tdc_state* state_dev, void* stream);
+QL_API size_t qlinear_tdc_ws_bytes(int64_t numel);
+/* After computing the block: one pass over in, out [numel] bf16 and the
+   latest delta; writes D_new = bf16(RN(out - in)) into the other slot, then
+   Gamma, E, the state and the next decision.  delta0/delta1: the block's two
+   slots (bf16 [numel] each, 16-byte aligned).  ws: zero-filled before first
+   use, qlinear_tdc_ws_bytes(numel) bytes, 256-byte aligned; calls that share
+   a workspace must not overlap on the GPU. */
+QL_API ql_status qlinear_tdc_refresh(const void* in_bf16, const void* out_bf16, int64_t numel,
+                                     void* delta0, void* delta1, ql_tdc_state* state_dev,
+                                     const ql_tdc_params* params, void* ws, size_t ws_bytes,
+                                     void* stream);
+/* Skip the block: out = bf16(RN(in + D_latest)), then acc += E, skips += 1
+   and the next decision (route INT8).  Skipping with no cached delta writes
+   nothing and records QL_ERR_INVALID_ARG in the device status word. */
+QL_API ql_status qlinear_tdc_skip(const void* in_bf16, int64_t numel, const void* delta0,
+                                  const void* delta1, ql_tdc_state* state_dev,
+                                  const ql_tdc_params* params, void* out_bf16, void* stream);
 
 #ifdef __cplusplus
 }
