@@ -606,6 +606,37 @@ def run_configs(reps: int = 20):
         "gemm_w4a8_onchip": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, M_TOKENS, pw, Y=y)),
                                     M_TOKENS, 7680, 1920, 1.0)}
     del bi, bo, q, q16, y, pw, pwx, wd
+    # Temporal delta cache on a sweep block pair [17776, 1920] (6Bit-Diffusion,
+    # B.2): the fused refresh reads in, out and the latest delta and writes
+    # the new delta (8 B/elem); the skip reads in and the delta and writes
+    # the output (6 B/elem)
+    bi, bo, _ = S.dmpq_block_pair(0)
+    bi, bo = bi.to(dev), bo.to(dev)
+    nel = bi.numel()
+    cache = ql.TdcCache(nel, dev)
+    ql.qlinear_tdc_refresh(bi, bo, cache)        # a delta is cached: the timed refreshes read it
+    ys = torch.empty_like(bi)
+    out["tdc"] = {"refresh": hbm_rec(med(lambda: ql.qlinear_tdc_refresh(bi, bo, cache)), 8.0 * nel),
+                  "skip": hbm_rec(med(lambda: ql.qlinear_tdc_skip(bi, cache, out=ys)), 6.0 * nel)}
+    del bi, bo, ys, cache
+    # Activation decomposition (SemanticDialect 2.2) on the CogVideoX-2B FFN
+    # linears: the quantizer reads 2 B/elem and writes both levels' codes and
+    # scales (1 + 1/8 B/elem); the GEMM contracts over K' = 2K
+    for lin in [l for l in S.COGVIDEOX_2B if l.name in ("ffn_up", "ffn_down")]:
+        x, w = S.cogvideox2b_linear(lin)
+        xd, wd = x.to(dev), w.to(dev)
+        pwd = ql.qlinear_prepare_weights(wd, ql.QL_W_NVFP4_DECOMP, hadamard=True)
+        aws = torch.zeros(ql.lib.qlinear_quantize_ws_bytes(M_TOKENS, lin.k, ql.QL_ROUTE_NVFP4), dtype=torch.uint8,
+                          device=dev)
+        amax = ql.qlinear_tensor_amax(xd, True, ws=aws)
+        q = ql.qlinear_quantize_act(xd, ql.QL_ACT_NVFP4_DECOMP, True, rowmajor_scales=False, amax_in=amax)
+        y = ql.qlinear_gemm(ql.QL_ACT_NVFP4_DECOMP, q, M_TOKENS, pwd)
+        out[f"decomp_{lin.name}"] = {
+            "quant_nvfp4_decomp": hbm_rec(med(lambda: ql.qlinear_quantize_act(
+                xd, ql.QL_ACT_NVFP4_DECOMP, True, amax_in=amax, out=q)), 3.125 * M_TOKENS * lin.k),
+            "gemm_w4a4_2k": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ACT_NVFP4_DECOMP, q, M_TOKENS, pwd, Y=y)),
+                                    M_TOKENS, lin.n, 2 * lin.k, 4.0)}
+        del xd, wd, pwd, q, y
     # 4: CogVideoX-5B linears, Q-ARVD dual-scale weights, per-tensor INT8
     for lin in S.COGVIDEOX_5B:
         x, w = S.cogvideox5b_qarvd_linear(lin)

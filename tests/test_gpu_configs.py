@@ -226,3 +226,33 @@ def test_wan14b_linear(ql, name):
     lin = [l for l in S.WAN_14B if l.name == name][0]
     x, w = S.wan14b_linear(lin)
     run_w4a4_linear(ql, x, w, seed=4)
+
+
+def test_cogvideox2b_ffn_down_decomposed(ql):
+    """Activation decomposition (SemanticDialect, Methodology 2.2) on the
+    CogVideoX-2B FFN-down linear ([17776, 7680] -> 1920, K' = 15360): every
+    code and scale of both levels bit-exact over all rows, the product on
+    sampled rows within the W4A4 tolerance."""
+    lin = [l for l in S.COGVIDEOX_2B if l.name == "ffn_down"][0]
+    x, w = S.cogvideox2b_linear(lin)
+    bits = S.bf16_bits(x)
+    m, k = bits.shape
+    g = O.nvfp4_tensor_scale(np.array([oracle_rotated_amax(bits)], np.float32))
+    xd = x.cuda()
+    q = ql.qlinear_quantize_act(xd, ql.QL_ACT_NVFP4_DECOMP, hadamard=True)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4_DECOMP, hadamard=True)
+    y = ql.qlinear_forward(xd, pw, ql.QL_ROUTE_NVFP4)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    assert _np(q["scales"])[0] == g
+    codes, sfr = _np(q["codes"]), _np(q["sf_rowmajor"])
+    for i in range(0, m, CHUNK):
+        packed, sb, _ = O.nvfp4_decompose(O.block_hadamard(O.bf16_bits_to_f32(bits[i:i + CHUNK])), g)
+        assert np.array_equal(codes[i:i + CHUNK], packed), f"codes differ in rows {i}.."
+        assert np.array_equal(sfr[i:i + CHUNK], sb)
+    wref = O.decompose_weights(O.prepare_weights_nvfp4(S.bf16_bits(w)))
+    rows = sample_rows(m, seed=7)
+    packed, sb, _ = O.nvfp4_decompose(O.block_hadamard(O.bf16_bits_to_f32(bits[rows])), g)
+    ref = O.gemm_w4a4(packed, sb, g, wref["packed"], wref["sb"], wref["g"])
+    yn = _np(y.float())[rows].astype(np.float64)
+    assert np.isfinite(yn).all() and normwise_err(yn, ref) <= 1e-2
