@@ -223,13 +223,13 @@ __device__ __forceinline__ uint32_t e2m1x8(float a0, float a1, float a2, float a
   return r;
 }
 
-// E2M1 code (bits 0-3: sign bit 3, magnitude code 0..7) -> its fp32 value
-// {0, 0.5, 1, 1.5, 2, 3, 4, 6} with the sign (code 8 is -0).
-__device__ __forceinline__ float e2m1_to_f32(uint32_t code) {
-  const uint32_t m = code & 7u;
-  uint32_t bits = (m >= 2u) ? ((((m >> 1) + 126u) << 23) | ((m & 1u) << 22)) : (m ? 0x3F000000u : 0u);
-  bits |= (code & 8u) << 28;
-  return __uint_as_float(bits);
+// Two E2M1 codes (bits 0-7 of `byte`: the first element in the low nibble)
+// -> their values {0, 0.5, 1, 1.5, 2, 3, 4, 6} with the sign (code 8 is -0),
+// by the hardware convert to f16x2 (exact: every E2M1 value is an f16).
+__device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(r) : "r"(byte));
+  return __half22float2(*reinterpret_cast<const __half2*>(&r));
 }
 
 // NVFP4 of one half block (64 values in the pair layout: 16-element blocks
@@ -325,9 +325,12 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
           const int j = 16 * b + 8 * h;
           const uint32_t lo = cw[2 * b + h], hi = cw[4 + 2 * b + h];
 #pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            P[j + t].x = __fsub_rn(P[j + t].x, __fmul_rn(e2m1_to_f32(lo >> (4 * t)), den[b].x));
-            P[j + t].y = __fsub_rn(P[j + t].y, __fmul_rn(e2m1_to_f32(hi >> (4 * t)), den[b].y));
+          for (int t = 0; t < 4; ++t) {   // elements 2t, 2t+1 of the group
+            const float2 vx = e2m1x2_to_f32x2(lo >> (8 * t)), vy = e2m1x2_to_f32x2(hi >> (8 * t));
+            P[j + 2 * t].x = __fsub_rn(P[j + 2 * t].x, __fmul_rn(vx.x, den[b].x));
+            P[j + 2 * t + 1].x = __fsub_rn(P[j + 2 * t + 1].x, __fmul_rn(vx.y, den[b].x));
+            P[j + 2 * t].y = __fsub_rn(P[j + 2 * t].y, __fmul_rn(vy.x, den[b].y));
+            P[j + 2 * t + 1].y = __fsub_rn(P[j + 2 * t + 1].y, __fmul_rn(vy.y, den[b].y));
           }
         }
       }
