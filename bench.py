@@ -65,7 +65,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--configs", action="store_true",
                     help="time every kernel of the five workload configurations (one JSON line, not the contract line)")
-    ap.add_argument("--profile-case", choices=["quant", "gemm"], default=None,
+    ap.add_argument("--profile-case", choices=["quant", "gemm", "qarvd", "tdc", "decomp"], default=None,
                     help="run one small standalone case for an ncu capture (prints no JSON)")
     return ap.parse_args()
 
@@ -83,6 +83,35 @@ def profile_case(which: str):
         for _ in range(2):
             ql.qlinear_tensor_amax(x, True, out=amax)
             ql.qlinear_quantize_act(x, ql.QL_ROUTE_NVFP4, True, amax_in=amax, out=q)
+    elif which == "qarvd":   # Q-ARVD int8 GEMM, CogVideoX-5B QKV (M=17776, 3072 -> 9216)
+        lin = [l for l in S.COGVIDEOX_5B if l.name == "qkv"][0]
+        x, w = S.cogvideox5b_qarvd_linear(lin)
+        x, w = x.to(dev), w.to(dev)
+        pw = ql.qlinear_prepare_weights(w, ql.QL_W_QARVD_INT4, False, expand_i8=True)
+        q = ql.qlinear_quantize_act(x, ql.QL_ACT_INT8_TENSOR, False, w=pw)
+        y = ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q, x.shape[0], pw)
+        for _ in range(2):
+            ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q, x.shape[0], pw, Y=y)
+    elif which == "tdc":     # TDC refresh + skip on a [17776, 1920] block pair
+        bi, bo, _ = S.dmpq_block_pair(0)
+        bi, bo = bi.to(dev), bo.to(dev)
+        cache = ql.TdcCache(bi.numel(), dev)
+        ql.qlinear_tdc_refresh(bi, bo, cache)
+        ys = torch.empty_like(bi)
+        for _ in range(2):
+            ql.qlinear_tdc_refresh(bi, bo, cache)
+            ql.qlinear_tdc_skip(bi, cache, out=ys)
+    elif which == "decomp":  # decomposed quantizer + GEMM, CogVideoX-2B FFN-up
+        lin = [l for l in S.COGVIDEOX_2B if l.name == "ffn_up"][0]
+        x, w = S.cogvideox2b_linear(lin)
+        x, w = x.to(dev), w.to(dev)
+        pw = ql.qlinear_prepare_weights(w, ql.QL_W_NVFP4_DECOMP, True)
+        amax = ql.qlinear_tensor_amax(x, True)
+        q = ql.qlinear_quantize_act(x, ql.QL_ACT_NVFP4_DECOMP, True, rowmajor_scales=False, amax_in=amax)
+        y = ql.qlinear_gemm(ql.QL_ACT_NVFP4_DECOMP, q, x.shape[0], pw)
+        for _ in range(2):
+            ql.qlinear_quantize_act(x, ql.QL_ACT_NVFP4_DECOMP, True, amax_in=amax, out=q)
+            ql.qlinear_gemm(ql.QL_ACT_NVFP4_DECOMP, q, x.shape[0], pw, Y=y)
     else:                    # W4A4 GEMM M=8192, N=7680, K=1920 (FFN-up shape, fewer tokens)
         m, n, k = 8192, 7680, 1920
         x = S.activations_with_outlier_channels(m, k, 0.01, 30.0, 1, 1).to(dev)
