@@ -238,6 +238,15 @@ void qlinear_debug_set_wait_limit(long long cycles) {
   g_wait_limit = cycles < 0 ? kDefaultWaitLimit : cycles;
 }
 
+ql_status qlinear_debug_div_check(float d, uint32_t a_begin, uint64_t count, unsigned long long* mismatches_dev,
+                                  void* stream) {
+  if (mismatches_dev == nullptr || !(d > 0.f) || d > 3.4028235e38f) return QL_ERR_INVALID_ARG;
+  if (a_begin >= 0x7F800000u || count > 0x7F800000ull - a_begin) return QL_ERR_INVALID_ARG;
+  if (!aligned(mismatches_dev, 8)) return QL_ERR_ALIGNMENT;
+  QL_TRY(device_ready());
+  return launch_debug_div_check(d, a_begin, count, mismatches_dev, static_cast<cudaStream_t>(stream));
+}
+
 ql_status qlinear_device_status(void* stream, int32_t* status_out) {
   if (status_out == nullptr) return QL_ERR_INVALID_ARG;
   QL_TRY(device_ready());

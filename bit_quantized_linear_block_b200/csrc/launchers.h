@@ -45,6 +45,8 @@ ql_status launch_gamma_route(const void* in, const void* out, int64_t numel, flo
 ql_status launch_qarvd_prepare(const void* W, int32_t N, int32_t K, float tau, float alpha,
                                const ql_weights* w, void* ws, cudaStream_t st);
 
+ql_status launch_debug_div_check(float d, uint32_t a_begin, uint64_t count, unsigned long long* mismatches,
+                                 cudaStream_t st);
 ql_status launch_tdc_init(ql_tdc_state* st, cudaStream_t s);
 ql_status launch_tdc_refresh(const void* in, const void* out, int64_t numel, void* slot0, void* slot1,
                              ql_tdc_state* st, const ql_tdc_params& prm, void* ws, cudaStream_t s);

@@ -232,12 +232,56 @@ __device__ __forceinline__ float2 e2m1x2_to_f32x2(uint32_t byte) {
   return __half22float2(*reinterpret_cast<const __half2*>(&r));
 }
 
+// Correctly rounded a / d for a >= 0 from r = RN(1 / d): Markstein's
+// correction step (P. Markstein, "Computation of elementary functions on
+// the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990):
+// q0 = RN(a r) is within one ulp of a / d, so the remainder a - q0 d is
+// exact in one fma, and RN(q0 + (a - q0 d) r) is the correctly rounded
+// quotient when r is within half an ulp of 1 / d (no over- or underflow).
+// The caller takes __fdiv_rn instead when d is outside [2^-100, 2^100].
+__device__ __forceinline__ float div_rn_by(float a, float d, float r) {
+  const float q0 = __fmul_rn(a, r);
+  const float e = __fmaf_rn(-q0, d, a);
+  return __fmaf_rn(e, r, q0);
+}
+
+// Per-launch tables of the NVFP4 block-scale arithmetic for the 128
+// non-negative E4M3 codes: den[c] = RN(E4M3(c) g), inv[c] = RN(1 / den[c])
+// (0 for c = 0).  The same operations the per-block code would run.
+struct Nvfp4Tables {
+  float den[128];
+  float inv[128];
+};
+
+__device__ __forceinline__ void nvfp4_tables_fill(Nvfp4Tables* t, float g) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    const float dn = __fmul_rn(e4m3_value(static_cast<uint32_t>(c)), g);
+    t->den[c] = dn;
+    t->inv[c] = c ? __frcp_rn(dn) : 0.f;
+  }
+}
+
+// Block scale code of a block with absolute maximum a: E4M3(RN(a / d)).
+struct Nvfp4ScaleDiv {
+  float d, r;
+  bool fast;
+  __device__ __forceinline__ explicit Nvfp4ScaleDiv(float d_) {
+    d = d_;
+    r = __frcp_rn(d_);
+    fast = d_ >= 7.8886091e-31f && d_ <= 1.2676506e30f;   // [2^-100, 2^100]
+  }
+  __device__ __forceinline__ uint32_t code(float a) const {
+    return e4m3_code(fast ? div_rn_by(a, d, r) : __fdiv_rn(a, d));
+  }
+};
+
 // NVFP4 of one half block (64 values in the pair layout: 16-element blocks
 // b = 0, 1 in P[16b..16b+15].x, b = 2, 3 in the .y halves).  Writes the four
 // E4M3 scales, the codes (cw[i]: elements 8i .. 8i+7 of the half) and each
 // block's RN(E4M3 value * g) (den[b] for blocks b and b + 2).
-__device__ __forceinline__ void nvfp4_half(const float2 (&P)[32], float g, float d, uint32_t (&sb)[4],
-                                           uint32_t (&cw)[8], float2 (&den)[2]) {
+__device__ __forceinline__ void nvfp4_half(const float2 (&P)[32], const Nvfp4ScaleDiv& sd,
+                                           const Nvfp4Tables* tab, uint32_t (&sb)[4], uint32_t (&cw)[8],
+                                           float2 (&den)[2]) {
 #pragma unroll
   for (int b = 0; b < 2; ++b) {
     float2 a = make_float2(0.f, 0.f);
@@ -246,10 +290,10 @@ __device__ __forceinline__ void nvfp4_half(const float2 (&P)[32], float g, float
       a.x = fmax3(a.x, fabsf(P[16 * b + t].x), fabsf(P[16 * b + t + 1].x));
       a.y = fmax3(a.y, fabsf(P[16 * b + t].y), fabsf(P[16 * b + t + 1].y));
     }
-    sb[b] = e4m3_code(__fdiv_rn(a.x, d));
-    sb[b + 2] = e4m3_code(__fdiv_rn(a.y, d));
-    den[b] = make_float2(__fmul_rn(e4m3_value(sb[b]), g), __fmul_rn(e4m3_value(sb[b + 2]), g));
-    const float2 inv = make_float2(sb[b] ? __frcp_rn(den[b].x) : 0.f, sb[b + 2] ? __frcp_rn(den[b].y) : 0.f);
+    sb[b] = sd.code(a.x);
+    sb[b + 2] = sd.code(a.y);
+    den[b] = make_float2(tab->den[sb[b]], tab->den[sb[b + 2]]);
+    const float2 inv = make_float2(tab->inv[sb[b]], tab->inv[sb[b + 2]]);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int j = 16 * b + 8 * h;
@@ -286,10 +330,13 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
                   uint8_t* __restrict__ sf_mma, uint8_t* __restrict__ sf_rm,
                   float* __restrict__ g_out) {
   extern __shared__ __align__(128) uint8_t ring_all[];
+  __shared__ Nvfp4Tables tab;
   const float amax_t = __ldg(amax_in);
   const float g = (amax_t == 0.f) ? 1.f : __fdiv_rn(amax_t, 2688.f);
   if (blockIdx.x == 0 && threadIdx.x == 0 && g_out != nullptr) *g_out = g;
-  const float d = __fmul_rn(6.f, g);
+  const Nvfp4ScaleDiv sd(__fmul_rn(6.f, g));
+  nvfp4_tables_fill(&tab, g);
+  __syncthreads();
   const uint32_t upr = static_cast<uint32_t>(K >> 7);
   const int32_t kq = DECOMP ? 2 * K : K;           // K of the quantized operand
   const int32_t k_atoms = kq >> 6;
@@ -305,7 +352,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     uint8_t* cdst = codes + static_cast<int64_t>(row) * row_bytes + j0 * 8;
     uint32_t sb[4], cw[8];
     float2 den[2];
-    nvfp4_half(P, g, d, sb, cw, den);
+    nvfp4_half(P, sd, &tab, sb, cw, den);
     auto store = [&](int part) {
       uint4* dst = reinterpret_cast<uint4*>(cdst + part * (K >> 1));
       dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
@@ -334,7 +381,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
           }
         }
       }
-      nvfp4_half(P, g, d, sb, cw, den);
+      nvfp4_half(P, sd, &tab, sb, cw, den);
       store(1);
     }
   });
@@ -552,9 +599,33 @@ __global__ void __launch_bounds__(kThreadsHbm)
   }
 }
 
+// Test hook: counts the dividends a (fp32 bit patterns a_begin ..
+// a_begin + count - 1, non-negative and finite) where the quantizer's
+// block-scale division differs from __fdiv_rn(a, d).
+__global__ void k_debug_div_check(float d, uint32_t a_begin, uint64_t count,
+                                  unsigned long long* mismatches) {
+  const Nvfp4ScaleDiv sd(d);
+  unsigned long long bad = 0;
+  for (uint64_t i = blockIdx.x * static_cast<uint64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+    const float a = __uint_as_float(a_begin + static_cast<uint32_t>(i));
+    const float q = sd.fast ? div_rn_by(a, sd.d, sd.r) : __fdiv_rn(a, d);
+    bad += __float_as_uint(q) != __float_as_uint(__fdiv_rn(a, d));
+  }
+  for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
+  if ((threadIdx.x & 31) == 0 && bad) atomicAdd(mismatches, bad);
+}
+
 // --------------------------------------------------------------------------
 // Host launchers
 // --------------------------------------------------------------------------
+ql_status launch_debug_div_check(float d, uint32_t a_begin, uint64_t count, unsigned long long* mismatches,
+                                 cudaStream_t st) {
+  const int grid = num_sms() * 8;
+  k_debug_div_check<<<grid, 256, 0, st>>>(d, a_begin, count, mismatches);
+  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+}
+
 int hbm_grid(int64_t work_items, int per_cta) {
   const int64_t want = (work_items + per_cta - 1) / per_cta;
   const int64_t cap = static_cast<int64_t>(num_sms()) * kHbmCtasPerSm;

@@ -74,6 +74,7 @@ def _load() -> C.CDLL:
         "qlinear_status_string": (C.c_char_p, [C.c_int]),
         "qlinear_device_status": (C.c_int, [vp, C.POINTER(i32)]),
         "qlinear_debug_set_wait_limit": (None, [C.c_longlong]),
+        "qlinear_debug_div_check": (C.c_int, [f32, C.c_uint32, C.c_uint64, vp, vp]),
         "qlinear_sf_bytes": (sz, [i64, i32]),
         "qlinear_weights_bytes": (sz, [i32, i32, C.POINTER(WeightCfg)]),
         "qlinear_prepare_ws_bytes": (sz, [i32, i32, C.POINTER(WeightCfg)]),
@@ -345,6 +346,15 @@ def qlinear_device_status(stream=None) -> int:
 
 def qlinear_debug_set_wait_limit(cycles: int):
     lib.qlinear_debug_set_wait_limit(int(cycles))
+
+
+def qlinear_debug_div_check(d: float, a_begin: int, count: int, stream=None) -> int:
+    """Number of dividends (fp32 bit patterns a_begin .. a_begin+count-1)
+    where the quantizer's block-scale division by d is not correctly rounded."""
+    out = torch.zeros(1, dtype=torch.int64, device="cuda")
+    _check("qlinear_debug_div_check", lib.qlinear_debug_div_check(float(d), int(a_begin), int(count),
+                                                                  _ptr(out), _stream(stream)))
+    return int(out.item())
 
 
 # --- host-side layout helper for inspection (pure index permutation) --------

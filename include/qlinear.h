@@ -160,6 +160,13 @@ QL_API ql_status qlinear_device_status(void* stream, int32_t* status_out);
    returns.  Negative restores the default.  Host-global, not thread-safe. */
 QL_API void qlinear_debug_set_wait_limit(long long cycles);
 
+/* Test hook: adds to *mismatches_dev (device, 8-byte aligned) the number of
+   dividends a with fp32 bit patterns a_begin .. a_begin + count - 1 (must
+   stay non-negative and finite) for which the NVFP4 quantizer's block-scale
+   division by d differs from the correctly rounded a / d. */
+QL_API ql_status qlinear_debug_div_check(float d, uint32_t a_begin, uint64_t count,
+                                         unsigned long long* mismatches_dev, void* stream);
+
 /* ---- sizes ---------------------------------------------------------------- */
 
 /* Bytes of NVFP4 block scales in the MMA layout for a [rows, K] tensor. */

@@ -61,6 +61,23 @@ def test_nvfp4_quantize_bit_exact(ql, m, k, hadamard):
     assert np.array_equal(_np(q["codes"]), packed)
 
 
+def test_block_scale_division_is_correctly_rounded(ql):
+    """The quantizer divides each block maximum a by d = RN(6 g) with a
+    reciprocal and one Markstein correction.  Against the correctly rounded
+    quotient, for every fp32 dividend from d 2^-12 (below, the E4M3 code is 0
+    whatever the rounding) to 450 d (block maxima never exceed 448 d (1 +
+    2^-22)), for divisors from random, tiny, huge and edge tensor scales."""
+    rng = np.random.default_rng(0)
+    gs = ([1.0, 1.0 / 3.0, 0.1, 7.0, 2.0 ** -20, 2.0 ** 20, 1e-33, 1e33]
+          + list(rng.uniform(1e-3, 10.0, 16)) + list(10.0 ** rng.uniform(-30, 30, 16)))
+    bits = lambda v: int(np.array(v, np.float32).view(np.uint32))
+    for g in gs:
+        d = np.float32(np.float32(6.0) * np.float32(g))
+        lo = bits(d * np.float32(2.0 ** -12))
+        hi = bits(min(np.float32(d) * np.float32(450.0), np.float32(3.0e38)))
+        assert ql.qlinear_debug_div_check(float(d), lo, hi - lo + 1) == 0, float(d)
+
+
 def test_nvfp4_quantize_zero_and_tiny_blocks(ql):
     x = np.zeros((130, 256), np.float32)
     x[0, 0] = 3000.0
