@@ -18,6 +18,7 @@ constexpr size_t kRoutePartialBytes = 2 * kMaxPartials * sizeof(double);
 constexpr size_t kTdcPartialBytes = 4 * kMaxPartials * sizeof(double);
 
 int num_sms();
+int* status_word();   // device status word of the current device (see qlinear_device_status)
 bool set_smem_attr(const void* kernel, int bytes);
 int hbm_grid(int64_t work_items, int per_cta);
 int qarvd_slices(int32_t N);

@@ -14,6 +14,7 @@
 // loads).  Butterfly distances 1..16 stay inside a lane, 32 and 64 are one
 // shuffle each.  A warp covers 8 blocks = 1024 contiguous elements.
 #include "ql_common.cuh"
+#include "gemm_common.cuh"
 #include "launchers.h"
 
 namespace ql {
@@ -30,12 +31,14 @@ __device__ __forceinline__ float warp_max(float m) {
 // 2i and 2i+1.
 //
 // A warp walks the flat tensor in chunks of 16 blocks (4 KB) with a
-// kRing-deep cp.async ring of 4 KB slots in shared memory.  Loads are 16-byte
-// cp.async copies in which lane l takes bytes 16*(l + 32 i) of the chunk, so
-// one instruction moves 512 contiguous bytes.  Each lane's 128 bytes land in
-// their own 128-byte region with 16-byte slot s stored at s ^ (lane % 8);
-// the read-back, where every lane reads its own region slot by slot, is then
-// free of bank conflicts.
+// kRing-deep ring of 4 KB slots in shared memory, each filled by ONE TMA
+// load issued by the warp's first lane and tracked by the slot's mbarrier.
+// The tensor map views the input as rows of 128 bytes (one lane's half
+// block) with a 32-row box and the 128-byte swizzle, so 16-byte piece s of
+// lane l's row lands at s ^ (l % 8): the read-back, where every lane reads
+// its own row piece by piece, is free of bank conflicts.  Slots start on
+// 1024-byte boundaries (the swizzle's period).  Rows past the end read as
+// zeros.
 // ---------------------------------------------------------------------------
 constexpr int kRing = 3;                         // stages per warp
 constexpr int kLaneBytes = 128;                  // 64 bf16
@@ -46,6 +49,12 @@ constexpr int kRingCtasPerSm = 2;
 constexpr int kQuantThreads = 384;                                     // NVFP4: 1 CTA/SM
 constexpr int kQuantWarps = kQuantThreads / 32;
 constexpr int kQuantRingBytes = kQuantWarps * kRing * kChunkBytes;     // 144 KB
+constexpr int kRingAlignPad = 1024;                                    // for the 1024-byte aligned base
+
+__device__ __forceinline__ uint8_t* ring_base(uint8_t* p) {
+  const uint32_t a = smem_u32(p);
+  return p + (((a + 1023u) & ~1023u) - a);
+}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes)
@@ -55,24 +64,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// Issue the copies of chunk `c` (past the end: zero-size copies that read
-// nothing) into ring slot `slot`.
-__device__ __forceinline__ void issue_chunk(uint32_t ring, int slot, const uint8_t* base,
-                                            int64_t total_bytes, int64_t c) {
-  const uint32_t lane = lane_id();
-  const int64_t cbase = c * kChunkBytes;
-  const uint32_t sbase = ring + slot * kChunkBytes;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t o = 16u * (lane + 32u * i);
-    const uint32_t owner = o >> 7, s16 = (o >> 4) & 7u;
-    const uint32_t dst = sbase + owner * kLaneBytes + ((s16 ^ (owner & 7u)) << 4);
-    const bool ok = cbase + o < total_bytes;
-    cp_async16(dst, ok ? static_cast<const void*>(base + cbase + o) : static_cast<const void*>(base),
-               ok ? 16u : 0u);
-  }
 }
 
 // This lane's 64 elements of a landed slot, in pair registers
@@ -129,34 +120,56 @@ __device__ __forceinline__ void fwht128_half(float2 (&P)[32]) {
 }
 
 // Per-warp ring driver: calls body(P, half_index) for each half block this
-// lane owns (half_index = 2 * block + (lane & 1)).
+// lane owns (half_index = 2 * block + (lane & 1)).  `bars` holds kRing
+// mbarriers per warp.  A wait that runs out of its cycle budget records
+// QL_ERR_TIMEOUT, waits (bounded) for the warp's loads still in flight and
+// ends the warp's walk.
 template <int WARPS, class Body>
-__device__ __forceinline__ void stream_blocks(const uint8_t* x, int64_t total_bytes, int hadamard,
-                                              uint8_t* ring_all, Body body) {
+__device__ __forceinline__ void stream_blocks(const CUtensorMap* tm, int64_t total_bytes, int hadamard,
+                                              uint8_t* ring_all, uint64_t* bars, int* status, Body body) {
   const int wid = threadIdx.x >> 5;
   uint8_t* ring_g = ring_all + wid * kRing * kChunkBytes;
-  const uint32_t ring = smem_u32(ring_g);
+  uint64_t* bar = bars + wid * kRing;
+  const bool leader = lane_id() == 0;
   const int64_t nchunks = (total_bytes + kChunkBytes - 1) / kChunkBytes;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * WARPS + wid;
   const int64_t nw = static_cast<int64_t>(gridDim.x) * WARPS;
   const int64_t mine = (gw < nchunks) ? (nchunks - gw + nw - 1) / nw : 0;
+  if (leader) {
 #pragma unroll
-  for (int i = 0; i < kRing - 1; ++i) {
-    issue_chunk(ring, i, x, total_bytes, gw + i * nw);
-    cp_async_commit();
+    for (int i = 0; i < kRing; ++i) mbar_init(&bar[i], 1);
+    fence_mbar_init();
   }
-  for (int64_t k = 0; k < mine; ++k) {
-    issue_chunk(ring, static_cast<int>((k + kRing - 1) % kRing), x, total_bytes, gw + (k + kRing - 1) * nw);
-    cp_async_commit();
-    cp_async_wait<kRing - 1>();
-    __syncwarp();
+  __syncwarp();
+  auto issue = [&](int64_t k) {   // chunk k of this warp into slot k % kRing
+    if (leader) {
+      const int slot = static_cast<int>(k % kRing);
+      mbar_arrive_expect_tx(&bar[slot], kChunkBytes);
+      tma_load_2d(ring_g + slot * kChunkBytes, tm, &bar[slot], 0, static_cast<int32_t>((gw + k * nw) * 32));
+    }
+  };
+  for (int64_t i = 0; i < kRing - 1 && i < mine; ++i) issue(i);
+  int64_t k = 0;
+  for (; k < mine; ++k) {
+    // the slot refilled here was read in the previous iteration, before its
+    // closing __syncwarp
+    if (k + kRing - 1 < mine) issue(k + kRing - 1);
+    const int slot = static_cast<int>(k % kRing);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar[slot], static_cast<uint32_t>((k / kRing) & 1),
+                                                      kDrainLimit));
+    if (!ok) break;
     float2 P[32];
-    read_half(ring_g + (k % kRing) * kChunkBytes, P);
+    read_half(ring_g + slot * kChunkBytes, P);
     __syncwarp();
     if (hadamard) fwht128_half(P);
     body(P, (gw + k * nw) * 32 + lane_id());
   }
-  cp_async_wait<0>();
+  if (k < mine && leader) {   // timed out: let the loads in flight land before the CTA may exit
+    record_error(status, QL_ERR_TIMEOUT);
+    for (int64_t j = k; j < mine && j < k + kRing; ++j)   // chunks k .. k + kRing - 1 were issued
+      (void)mbar_wait(&bar[j % kRing], static_cast<uint32_t>((j / kRing) & 1), kDrainLimit);
+  }
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------------------
@@ -166,12 +179,15 @@ __device__ __forceinline__ void stream_blocks(const uint8_t* x, int64_t total_by
 // the ticket.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreadsHbm, kRingCtasPerSm)
-    k_amax(const uint8_t* __restrict__ x, int64_t total_bytes, int hadamard,
-           float* __restrict__ partials, unsigned int* __restrict__ ticket, float* __restrict__ amax_out) {
-  extern __shared__ __align__(128) uint8_t ring_all[];
+    k_amax(const __grid_constant__ CUtensorMap tm_x, int64_t total_bytes, int hadamard,
+           float* __restrict__ partials, unsigned int* __restrict__ ticket, float* __restrict__ amax_out,
+           int* status) {
+  extern __shared__ uint8_t ring_raw[];
+  __shared__ uint64_t bars[kWarpsPerCta * kRing];
+  uint8_t* ring_all = ring_base(ring_raw);
   const uint32_t lane = lane_id();
   float m = 0.f;
-  stream_blocks<kWarpsPerCta>(x, total_bytes, hadamard, ring_all, [&](float2 (&P)[32], int64_t) {
+  stream_blocks<kWarpsPerCta>(&tm_x, total_bytes, hadamard, ring_all, bars, status, [&](float2 (&P)[32], int64_t) {
     float2 mm = make_float2(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < 32; j += 2) {
@@ -325,12 +341,14 @@ __device__ __forceinline__ void nvfp4_half(const float2 (&P)[32], const Nvfp4Sca
 // ---------------------------------------------------------------------------
 template <bool DECOMP>
 __global__ void __launch_bounds__(kQuantThreads, 1)
-    k_quant_nvfp4(const uint8_t* __restrict__ x, int64_t M, int32_t K, int hadamard,
+    k_quant_nvfp4(const __grid_constant__ CUtensorMap tm_x, int64_t M, int32_t K, int hadamard,
                   const float* __restrict__ amax_in, uint8_t* __restrict__ codes,
                   uint8_t* __restrict__ sf_mma, uint8_t* __restrict__ sf_rm,
-                  float* __restrict__ g_out) {
-  extern __shared__ __align__(128) uint8_t ring_all[];
+                  float* __restrict__ g_out, int* status) {
+  extern __shared__ uint8_t ring_raw[];
   __shared__ Nvfp4Tables tab;
+  __shared__ uint64_t bars[kQuantWarps * kRing];
+  uint8_t* ring_all = ring_base(ring_raw);
   const float amax_t = __ldg(amax_in);
   const float g = (amax_t == 0.f) ? 1.f : __fdiv_rn(amax_t, 2688.f);
   if (blockIdx.x == 0 && threadIdx.x == 0 && g_out != nullptr) *g_out = g;
@@ -343,7 +361,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   const int64_t row_bytes = kq >> 1;
   const int64_t units = M * upr;
   const int64_t halves = 2 * units;
-  stream_blocks<kQuantWarps>(x, M * K * 2, hadamard, ring_all, [&](float2 (&P)[32], int64_t hu) {
+  stream_blocks<kQuantWarps>(&tm_x, M * K * 2, hadamard, ring_all, bars, status, [&](float2 (&P)[32], int64_t hu) {
     if (hu >= halves) return;
     // half index -> (row, first scale index, first code byte); 32-bit division (units < 2^32)
     const uint32_t u = static_cast<uint32_t>(hu >> 1);
@@ -619,6 +637,15 @@ __global__ void k_debug_div_check(float d, uint32_t a_begin, uint64_t count,
 // --------------------------------------------------------------------------
 // Host launchers
 // --------------------------------------------------------------------------
+// The streaming kernels' view of a contiguous bf16 tensor: rows of 128 bytes
+// (half a Hadamard block), a box of 32 rows (one warp's 4 KB chunk), 128-byte
+// swizzle.  total_bytes is a multiple of 256.
+static bool make_stream_tmap(CUtensorMap* tm, const void* x, int64_t total_bytes) {
+  if (total_bytes / kLaneBytes >= (int64_t(1) << 31)) return false;   // row coordinates are 32-bit
+  return make_tmap_2d(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, x, kLaneBytes, total_bytes / kLaneBytes, kLaneBytes,
+                      kLaneBytes, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 ql_status launch_debug_div_check(float d, uint32_t a_begin, uint64_t count, unsigned long long* mismatches,
                                  cudaStream_t st) {
   const int grid = num_sms() * 8;
@@ -647,9 +674,11 @@ ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* 
   const int grid = ring_grid((units * 256 + kChunkBytes - 1) / kChunkBytes);
   float* partials = static_cast<float*>(ws);
   unsigned int* ticket = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + kAmaxPartialBytes);
-  if (!set_smem_attr(reinterpret_cast<const void*>(k_amax), kRingBytesPerCta)) return QL_ERR_CUDA;
-  k_amax<<<grid, kThreadsHbm, kRingBytesPerCta, st>>>(static_cast<const uint8_t*>(x), units * 256,
-                                                      hadamard, partials, ticket, amax_out);
+  CUtensorMap tm;
+  if (!make_stream_tmap(&tm, x, units * 256)) return QL_ERR_CUDA;
+  if (!set_smem_attr(reinterpret_cast<const void*>(k_amax), kRingBytesPerCta + kRingAlignPad)) return QL_ERR_CUDA;
+  k_amax<<<grid, kThreadsHbm, kRingBytesPerCta + kRingAlignPad, st>>>(tm, units * 256, hadamard, partials, ticket,
+                                                                      amax_out, status_word());
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
@@ -660,10 +689,12 @@ ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, 
   const int grid = static_cast<int>(std::max<int64_t>(
       1, std::min<int64_t>((nchunks + kQuantWarps - 1) / kQuantWarps, num_sms())));
   auto kern = decomp ? k_quant_nvfp4<true> : k_quant_nvfp4<false>;
-  if (!set_smem_attr(reinterpret_cast<const void*>(kern), kQuantRingBytes)) return QL_ERR_CUDA;
-  kern<<<grid, kQuantThreads, kQuantRingBytes, st>>>(static_cast<const uint8_t*>(x), M, K, hadamard, amax_in,
-                                                     static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf_mma),
-                                                     static_cast<uint8_t*>(sf_rm), g_out);
+  CUtensorMap tm;
+  if (!make_stream_tmap(&tm, x, M * K * 2)) return QL_ERR_CUDA;
+  if (!set_smem_attr(reinterpret_cast<const void*>(kern), kQuantRingBytes + kRingAlignPad)) return QL_ERR_CUDA;
+  kern<<<grid, kQuantThreads, kQuantRingBytes + kRingAlignPad, st>>>(
+      tm, M, K, hadamard, amax_in, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf_mma),
+      static_cast<uint8_t*>(sf_rm), g_out, status_word());
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
