@@ -415,10 +415,10 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// Per-token INT8: one warp per row.  The bf16 row is copied into shared
-// memory with coalesced 16-byte cp.async (the next row's copy is in flight
-// while this one is quantized; 16-byte slots swizzled as in the streaming
-// ring), lane l takes half blocks 32 p + l (p = 0, 1, ...) with the same
+// Per-token INT8: one warp per row.  The bf16 row comes into one of the
+// warp's two 1024-byte aligned shared-memory buffers by TMA (the streaming
+// kernels' 128-byte-row view and swizzle; the next row's load is in flight
+// while this one is quantized), lane l takes half blocks 32 p + l (p = 0, 1, ...) with the same
 // half-block FWHT as the NVFP4 path.  amax_m = max |h| over the row,
 // q = clamp(rint(RN(h * RN(127 / amax_m))), -127, 127), s_m = RN(amax_m/127).
 // A row of at most 2048 elements is rotated once and stays in registers;
@@ -444,48 +444,54 @@ __device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv
     uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
     for (int i = 0; i < 8; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-    return;
-  }
-  uint32_t w[16];
+  } else {
+    uint32_t w[16];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {   // elements 4i..4i+3 (.x halves) and 32+4i.. (.y halves)
-    uint32_t lo = 0, hi = 0;
+    for (int i = 0; i < 8; ++i) {   // elements 4i..4i+3 (.x halves) and 32+4i.. (.y halves)
+      uint32_t lo = 0, hi = 0;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int ql = max(-127, min(127, __float2int_rn(__fmul_rn(P[4 * i + b].x, inv))));
-      const int qh = max(-127, min(127, __float2int_rn(__fmul_rn(P[4 * i + b].y, inv))));
-      lo |= (static_cast<uint32_t>(ql) & 0xFFu) << (8 * b);
-      hi |= (static_cast<uint32_t>(qh) & 0xFFu) << (8 * b);
+      for (int b = 0; b < 4; ++b) {
+        const int ql = max(-127, min(127, __float2int_rn(__fmul_rn(P[4 * i + b].x, inv))));
+        const int qh = max(-127, min(127, __float2int_rn(__fmul_rn(P[4 * i + b].y, inv))));
+        lo |= (static_cast<uint32_t>(ql) & 0xFFu) << (8 * b);
+        hi |= (static_cast<uint32_t>(qh) & 0xFFu) << (8 * b);
+      }
+      w[i] = lo;
+      w[8 + i] = hi;
     }
-    w[i] = lo;
-    w[8 + i] = hi;
-  }
-  uint4* d = reinterpret_cast<uint4*>(dst);
+    uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+    for (int i = 0; i < 4; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  }
 }
 
 template <bool F16>
 __global__ void __launch_bounds__(kThreadsHbm)
-    k_quant_int8_token(const uint8_t* __restrict__ x, int64_t M, int32_t K, int hadamard,
-                       uint8_t* __restrict__ codes, float* __restrict__ scales) {
-  extern __shared__ __align__(128) uint8_t s_rows[];
+    k_quant_int8_token(const __grid_constant__ CUtensorMap tm_x, int64_t M, int32_t K, int hadamard,
+                       int32_t buf_bytes, int32_t box_rows, uint8_t* __restrict__ codes,
+                       float* __restrict__ scales, int* status) {
+  extern __shared__ uint8_t s_raw[];
+  __shared__ uint64_t bars[2 * (kThreadsHbm / 32)];
+  uint8_t* s_rows = ring_base(s_raw);
   const uint32_t lane = lane_id();
   const int wid = threadIdx.x >> 5;
-  const int32_t row_bytes = 2 * K;
-  const int32_t halves = K >> 6;                 // 64-element half blocks per row
+  const int32_t halves = K >> 6;                 // 64-element half blocks (128-byte rows) per token row
   const int32_t passes = (halves + 31) >> 5;
-  uint8_t* rows[2] = {s_rows + (2 * wid) * row_bytes, s_rows + (2 * wid + 1) * row_bytes};
+  uint8_t* rows[2] = {s_rows + (2 * wid) * buf_bytes, s_rows + (2 * wid + 1) * buf_bytes};
+  uint64_t* bar = bars + 2 * wid;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + wid;
   const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
-  auto issue_row = [&](int64_t r, uint8_t* dst) {
-    const uint8_t* src = x + r * row_bytes;
-    const uint32_t d = smem_u32(dst);
-    for (int32_t o = 16 * static_cast<int32_t>(lane); o < row_bytes; o += 512) {
-      const uint32_t owner = static_cast<uint32_t>(o) >> 7, s16 = (static_cast<uint32_t>(o) >> 4) & 7u;
-      const bool ok = r < M;
-      cp_async16(d + owner * kLaneBytes + ((s16 ^ (owner & 7u)) << 4),
-                 ok ? static_cast<const void*>(src + o) : static_cast<const void*>(x), ok ? 16u : 0u);
+  if (lane == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  auto issue_row = [&](int64_t r, int b) {   // token row r into buffer b: halves / box_rows boxes
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bar[b], static_cast<uint32_t>(halves) * kLaneBytes);
+      for (int32_t y = 0; y < halves; y += box_rows)
+        tma_load_2d(rows[b] + y * kLaneBytes, &tm_x, &bar[b], 0, static_cast<int32_t>(r * halves + y));
     }
   };
   auto load_half = [&](const uint8_t* row, int p, float2 (&P)[32]) {
@@ -497,14 +503,14 @@ __global__ void __launch_bounds__(kThreadsHbm)
     }
     if (hadamard) fwht128_half(P);   // all lanes (pair shuffles)
   };
-  issue_row(gw, rows[0]);
-  cp_async_commit();
+  if (gw < M) issue_row(gw, 0);
   int k = 0;
+  bool ok = true;
   for (int64_t r = gw; r < M; r += nw, ++k) {
-    issue_row(r + nw, rows[(k + 1) & 1]);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncwarp();
+    // the buffer refilled here was read in the previous iteration, before its closing __syncwarp
+    if (r + nw < M) issue_row(r + nw, (k + 1) & 1);
+    ok = __all_sync(0xffffffffu, mbar_wait(&bar[k & 1], static_cast<uint32_t>((k >> 1) & 1), kDrainLimit));
+    if (!ok) break;
     const uint8_t* row = rows[k & 1];
     float2 P[32];
     float m = 0.f;
@@ -526,7 +532,13 @@ __global__ void __launch_bounds__(kThreadsHbm)
     }
     __syncwarp();
   }
-  cp_async_wait<0>();
+  if (!ok && lane == 0) {   // timed out at iteration k: let this row's and the next row's loads land
+    record_error(status, QL_ERR_TIMEOUT);
+    const int64_t r = gw + static_cast<int64_t>(k) * nw;
+    (void)mbar_wait(&bar[k & 1], static_cast<uint32_t>((k >> 1) & 1), kDrainLimit);
+    if (r + nw < M) (void)mbar_wait(&bar[(k + 1) & 1], static_cast<uint32_t>(((k + 1) >> 1) & 1), kDrainLimit);
+  }
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------------------
@@ -640,10 +652,10 @@ __global__ void k_debug_div_check(float d, uint32_t a_begin, uint64_t count,
 // The streaming kernels' view of a contiguous bf16 tensor: rows of 128 bytes
 // (half a Hadamard block), a box of 32 rows (one warp's 4 KB chunk), 128-byte
 // swizzle.  total_bytes is a multiple of 256.
-static bool make_stream_tmap(CUtensorMap* tm, const void* x, int64_t total_bytes) {
+static bool make_stream_tmap(CUtensorMap* tm, const void* x, int64_t total_bytes, uint32_t box_rows = 32) {
   if (total_bytes / kLaneBytes >= (int64_t(1) << 31)) return false;   // row coordinates are 32-bit
   return make_tmap_2d(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, x, kLaneBytes, total_bytes / kLaneBytes, kLaneBytes,
-                      kLaneBytes, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+                      kLaneBytes, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 ql_status launch_debug_div_check(float d, uint32_t a_begin, uint64_t count, unsigned long long* mismatches,
@@ -709,16 +721,24 @@ ql_status launch_expand_nvfp4_f16(const void* codes, const void* sf, int32_t N, 
 ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadamard, void* codes,
                                   float* scales, cudaStream_t st, int f16_codes) {
   if (M == 0) return QL_OK;
-  const int64_t per_warp = 4 * static_cast<int64_t>(K);   // two bf16 row buffers
-  const int warps = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kThreadsHbm / 32, (200 * 1024) / per_warp)));
+  // a token row is K/64 rows of 128 bytes; TMA boxes of at most 256 rows that tile it exactly
+  const int32_t halves = K / 64;
+  int32_t box_rows = std::min<int32_t>(halves, 256);
+  while (halves % box_rows != 0) --box_rows;
+  const int64_t buf = (static_cast<int64_t>(halves) * kLaneBytes + 1023) / 1024 * 1024;   // 1024-byte aligned
+  const int64_t per_warp = 2 * buf;                                                        // two row buffers
   if (per_warp > 200 * 1024) return QL_ERR_UNSUPPORTED_SHAPE;
-  const size_t smem = static_cast<size_t>(warps) * per_warp;
+  const int warps = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(kThreadsHbm / 32, (200 * 1024) / per_warp)));
+  const size_t smem = static_cast<size_t>(warps) * per_warp + kRingAlignPad;
+  const int per_sm = std::max(1, std::min(4, static_cast<int>((227 * 1024) / smem)));
   const int64_t want = (M + warps - 1) / warps;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, 2 * num_sms())));
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, static_cast<int64_t>(per_sm) * num_sms())));
+  CUtensorMap tm;
+  if (!make_stream_tmap(&tm, x, M * K * 2, static_cast<uint32_t>(box_rows))) return QL_ERR_CUDA;
   auto kern = f16_codes ? k_quant_int8_token<true> : k_quant_int8_token<false>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), static_cast<int>(smem))) return QL_ERR_CUDA;
-  kern<<<grid, 32 * warps, smem, st>>>(static_cast<const uint8_t*>(x), M, K, hadamard,
-                                       static_cast<uint8_t*>(codes), scales);
+  kern<<<grid, 32 * warps, smem, st>>>(tm, M, K, hadamard, static_cast<int32_t>(buf), box_rows,
+                                       static_cast<uint8_t*>(codes), scales, status_word());
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
