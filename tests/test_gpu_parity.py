@@ -181,6 +181,9 @@ W4A4_CASES = [
     (129, 640, 384),     # N not a multiple of 192 -> 128-wide tiles
     (1, 192, 128),
     (1000, 5760, 1920),  # many tiles per CTA (persistent loop, both accumulators)
+    (300, 1040, 640),    # ragged last 192-wide tile, N not a multiple of 128 (padded scale rows)
+    (520, 5120, 2048),   # ragged 192-wide tiles with streamed scales (the Wan-14B FFN-down form)
+    (100, 1040, 2048),   # one SM per tile (M <= 128), ragged, streamed scales
 ]
 
 
