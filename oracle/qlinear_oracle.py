@@ -275,31 +275,41 @@ def decompose_weights(wq: dict) -> dict:
 # details: per-tensor activation quantisation).
 # ---------------------------------------------------------------------------
 
-def _int8_from_amax(x: np.ndarray, amax: np.ndarray):
+def _int8_from_amax(x: np.ndarray, amax: np.ndarray, qmax: int = INT8_QMAX):
+    """Symmetric integer codes in [-qmax, qmax] (int8 containers): scale =
+    RN(amax / qmax), q = clamp(rint(RN(x * RN(qmax / amax)))), 0 where amax = 0."""
     amax = np.asarray(amax, dtype=np.float32)
     nz = amax != 0
-    scale = np.where(nz, (amax / np.float32(INT8_QMAX)).astype(np.float32), np.float32(0))
+    scale = np.where(nz, (amax / np.float32(qmax)).astype(np.float32), np.float32(0))
     inv = np.zeros_like(amax)
-    inv[nz] = np.float32(INT8_QMAX) / amax[nz]                  # RN(127 / amax)
+    inv[nz] = np.float32(qmax) / amax[nz]                       # RN(qmax / amax)
     y = (x * inv).astype(np.float32)                            # RN(x * inv)
-    q = np.clip(np.rint(y), -INT8_QMAX, INT8_QMAX).astype(np.int8)   # ties to even
+    q = np.clip(np.rint(y), -qmax, qmax).astype(np.int8)        # ties to even
     return q, scale.astype(np.float32)
 
 
-def int8_per_token(h: np.ndarray):
-    """h: fp32 [R, K] -> (int8 [R, K], fp32 [R] scales s_m = amax_m / 127)."""
+def int8_per_token(h: np.ndarray, qmax: int = INT8_QMAX):
+    """h: fp32 [R, K] -> (int8 [R, K], fp32 [R] scales s_m = amax_m / qmax)."""
     h = np.asarray(h, dtype=np.float32)
     amax = np.max(np.abs(h), axis=1) if h.shape[1] else np.zeros(h.shape[0], np.float32)
-    q, s = _int8_from_amax(h, amax[:, None])
+    q, s = _int8_from_amax(h, amax[:, None], qmax)
     return q, s[:, 0]
 
 
-def int8_per_tensor(x: np.ndarray):
-    """x: fp32 [R, K] -> (int8 [R, K], fp32 scale s = amax / 127)."""
+def int8_per_tensor(x: np.ndarray, qmax: int = INT8_QMAX):
+    """x: fp32 [R, K] -> (int8 [R, K], fp32 scale s = amax / qmax)."""
     x = np.asarray(x, dtype=np.float32)
     amax = np.float32(np.max(np.abs(x))) if x.size else np.float32(0)
-    q, s = _int8_from_amax(x, np.array([[amax]], dtype=np.float32))
+    q, s = _int8_from_amax(x, np.array([[amax]], dtype=np.float32), qmax)
     return q, np.float32(s[0, 0])
+
+
+# W4A6 (S2Q-VDiT and Q-ARVD report W4A6 results; 6Bit-Diffusion's average
+# activation width is about 6 bits).  Reading: 6-bit signed integer
+# activations, symmetric [-31, 31], the same per-token / per-tensor recipes
+# as INT8 with 31 in place of 127, carried in int8 containers so the exact
+# integer products of the existing GEMMs apply unchanged.
+INT6_QMAX = 31
 
 
 # ---------------------------------------------------------------------------

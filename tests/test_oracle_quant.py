@@ -153,6 +153,31 @@ def test_int8_per_tensor():
     assert q.tolist() == [[0, -1], [0, 127]]             # 0.5 and -1 -> ties to even 0, -1
 
 
+def test_int6_brute_force_and_range():
+    """W4A6: the INT8 recipe with qmax = 31 (codes within [-31, 31])."""
+    rng = np.random.default_rng(8)
+    h = rng.standard_normal((5, 40)).astype(np.float32)
+    h[2, 7] = 40.0
+    q, s = O.int8_per_token(h, O.INT6_QMAX)
+    assert np.abs(q.astype(int)).max() == 31
+    for r in range(5):
+        a = max(abs(float(v)) for v in h[r])
+        assert s[r] == np.float32(np.float32(a) / np.float32(31))
+        inv = np.float32(np.float32(31) / np.float32(a))
+        for j in range(40):
+            assert q[r, j] == max(-31, min(31, round(float(np.float32(h[r, j] * inv)))))
+    qt, st = O.int8_per_tensor(np.array([[1.0, -62.0], [0.5, 31.0]], np.float32), O.INT6_QMAX)
+    assert st == np.float32(2.0) and qt.tolist() == [[0, -31], [0, 16]]   # 0.5 -> 0 and 15.5 -> 16 (ties to even)
+
+
+def test_int6_integer_rows_roundtrip():
+    rng = np.random.default_rng(9)
+    q = rng.integers(-31, 32, size=(4, 64)).astype(np.float32)
+    q[:, 5] = -31
+    got, s = O.int8_per_token(q, O.INT6_QMAX)
+    assert np.all(s == 1.0) and np.array_equal(got.astype(np.float32), q)
+
+
 # ---- a7 Q-ARVD ---------------------------------------------------------------
 
 def test_qarvd_golden_zscore_cases(golden):
