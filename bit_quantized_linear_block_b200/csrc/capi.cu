@@ -201,6 +201,16 @@ struct Carver {  // sequential 256-byte aligned sub-buffers of one allocation
   }
 };
 
+// W4A6: the INT6 formats are the INT8 formats with codes in [-31, 31].
+int32_t int_base_fmt(int32_t f) {
+  return f == QL_ROUTE_INT6 ? int32_t(QL_ROUTE_INT8)
+         : f == QL_ACT_INT6_F16 ? int32_t(QL_ACT_INT8_F16)
+         : f == QL_ACT_INT6_TENSOR ? int32_t(QL_ACT_INT8_TENSOR) : f;
+}
+int act_qmax(int32_t f) {
+  return (f == QL_ROUTE_INT6 || f == QL_ACT_INT6_F16 || f == QL_ACT_INT6_TENSOR) ? 31 : 127;
+}
+
 // f16_codes: the INT8 route keeps its codes as f16 values (weights with an
 // f16 copy), 2 bytes per element.
 size_t forward_act_bytes(int64_t M, int32_t K, int32_t Kp, int32_t fmt, bool f16_codes = false) {
@@ -445,6 +455,7 @@ ql_status qlinear_tdc_skip(const void* in, int64_t numel, const void* delta0, co
 // ---------------------------------------------------------------- activations
 size_t qlinear_quantize_ws_bytes(int64_t M, int32_t K, int32_t act_fmt) {
   if (M < 0 || check_k(K) != QL_OK) return 0;
+  act_fmt = int_base_fmt(act_fmt);
   if (act_fmt != QL_ROUTE_NVFP4 && act_fmt != QL_ROUTE_INT8 && act_fmt != QL_ACT_INT8_TENSOR &&
       act_fmt != QL_ACT_INT8_F16 && act_fmt != QL_ACT_NVFP4_DECOMP)
     return 0;
@@ -472,6 +483,8 @@ ql_status qlinear_quantize_act(const void* X, int64_t M, int32_t K, int32_t act_
   QL_TRY(check_mk(M, K));
   if (codes == nullptr || scales == nullptr || ws == nullptr || (M > 0 && X == nullptr))
     return QL_ERR_INVALID_ARG;
+  const int qmax = act_qmax(act_fmt);
+  act_fmt = int_base_fmt(act_fmt);
   if (act_fmt == QL_ROUTE_NVFP4 || act_fmt == QL_ACT_NVFP4_DECOMP) {
     if (sf_mma == nullptr) return QL_ERR_INVALID_ARG;
   } else if (act_fmt == QL_ACT_INT8_TENSOR) {
@@ -487,8 +500,8 @@ ql_status qlinear_quantize_act(const void* X, int64_t M, int32_t K, int32_t act_
   QL_TRY(device_ready());
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int had = hadamard ? 1 : 0;
-  if (act_fmt == QL_ROUTE_INT8) return launch_quant_int8_token(X, M, K, had, codes, scales, st);
-  if (act_fmt == QL_ACT_INT8_F16) return launch_quant_int8_token(X, M, K, had, codes, scales, st, 1);
+  if (act_fmt == QL_ROUTE_INT8) return launch_quant_int8_token(X, M, K, had, codes, scales, st, 0, qmax);
+  if (act_fmt == QL_ACT_INT8_F16) return launch_quant_int8_token(X, M, K, had, codes, scales, st, 1, qmax);
   const float* amax = amax_in;
   if (amax == nullptr) {
     float* slot = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kAmaxWsBytes);
@@ -498,7 +511,7 @@ ql_status qlinear_quantize_act(const void* X, int64_t M, int32_t K, int32_t act_
   if (act_fmt == QL_ROUTE_NVFP4 || act_fmt == QL_ACT_NVFP4_DECOMP)
     return launch_quant_nvfp4(X, M, K, had, amax, codes, sf_mma, sf_rowmajor, scales, st,
                               act_fmt == QL_ACT_NVFP4_DECOMP ? 1 : 0);
-  return launch_quant_int8_tensor_perm(X, M, K, w->Kp, w->gather, amax, codes, scales, st);
+  return launch_quant_int8_tensor_perm(X, M, K, w->Kp, w->gather, amax, codes, scales, st, qmax);
 }
 
 // ---------------------------------------------------------------- GEMM
@@ -507,6 +520,7 @@ ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf, c
   QL_TRY(check_m(M));
   QL_TRY(check_w(w));
   if (M > 0 && (a_codes == nullptr || a_scales == nullptr || Y == nullptr)) return QL_ERR_INVALID_ARG;
+  act_fmt = int_base_fmt(act_fmt);   // INT6 codes run through the INT8 GEMMs unchanged
   if (act_fmt == QL_ROUTE_NVFP4 || act_fmt == QL_ROUTE_INT8 || act_fmt == QL_ACT_INT8_F16) {
     if (w->fmt != QL_W_NVFP4) return QL_ERR_INVALID_ARG;
     if (act_fmt == QL_ACT_INT8_F16 && w->w16 == nullptr) return QL_ERR_INVALID_ARG;
@@ -542,6 +556,7 @@ size_t qlinear_forward_ws_bytes(int64_t M, const ql_weights* w, int32_t route) {
   if (w->fmt == QL_W_QARVD_INT4) return forward_act_bytes(M, w->K, w->Kp, QL_ACT_INT8_TENSOR);
   if (w->fmt == QL_W_NVFP4_DECOMP)
     return route == QL_ROUTE_NVFP4 ? forward_act_bytes(M, w->K, 0, QL_ACT_NVFP4_DECOMP) : 0;
+  route = int_base_fmt(route);
   if (route != QL_ROUTE_NVFP4 && route != QL_ROUTE_INT8) return 0;
   return forward_act_bytes(M, w->K, 0, route, w->w16 != nullptr);
 }
@@ -553,9 +568,12 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
   QL_TRY(check_mk(M, w->K));
   if (ws == nullptr || (M > 0 && (X == nullptr || Y == nullptr))) return QL_ERR_INVALID_ARG;
   if (w->fmt == QL_W_NVFP4_DECOMP && route != QL_ROUTE_NVFP4) return QL_ERR_INVALID_ARG;
+  // W4A6: route QL_ROUTE_INT6 (or QL_ACT_INT6_TENSOR for Q-ARVD weights)
+  const int qmax = (route == QL_ROUTE_INT6 || route == QL_ACT_INT6_TENSOR) ? 31 : 127;
+  if (w->fmt == QL_W_NVFP4 && route == QL_ACT_INT6_TENSOR) return QL_ERR_INVALID_ARG;
   const int32_t fmt = (w->fmt == QL_W_QARVD_INT4)     ? int32_t(QL_ACT_INT8_TENSOR)
                       : (w->fmt == QL_W_NVFP4_DECOMP) ? int32_t(QL_ACT_NVFP4_DECOMP)
-                                                      : route;
+                                                      : int_base_fmt(route);
   if (fmt != QL_ROUTE_NVFP4 && fmt != QL_ROUTE_INT8 && fmt != QL_ACT_INT8_TENSOR && fmt != QL_ACT_NVFP4_DECOMP)
     return QL_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256)) return QL_ERR_ALIGNMENT;
@@ -586,7 +604,7 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
     const int f16 = w->w16 != nullptr ? 1 : 0;
     uint8_t* codes = c.take<uint8_t>(static_cast<size_t>(M) * K * (f16 ? 2 : 1));
     float* s = c.take<float>(4 * static_cast<size_t>(M));
-    QL_TRY(launch_quant_int8_token(X, M, K, w->hadamard, codes, s, st, f16));
+    QL_TRY(launch_quant_int8_token(X, M, K, w->hadamard, codes, s, st, f16, qmax));
     return launch_gemm_w4a8(codes, s, M, w, Y, st, status, f16);
   }
   void* aws = c.take<uint8_t>(kAmaxWsBytes);
@@ -594,7 +612,7 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
   float* sx = c.take<float>(256);
   int8_t* codes = c.take<int8_t>(static_cast<size_t>(M) * w->Kp);
   QL_TRY(launch_amax(X, M, K, 0, amax, aws, st));
-  QL_TRY(launch_quant_int8_tensor_perm(X, M, K, w->Kp, w->gather, amax, codes, sx, st));
+  QL_TRY(launch_quant_int8_tensor_perm(X, M, K, w->Kp, w->gather, amax, codes, sx, st, qmax));
   return launch_gemm_qarvd(codes, sx, M, w, Y, st, status);
 }
 

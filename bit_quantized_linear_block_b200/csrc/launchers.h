@@ -36,11 +36,12 @@ ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, 
 ql_status launch_expand_nvfp4_f16(const void* codes, const void* sf, int32_t N, int32_t K, void* out,
                                   cudaStream_t st);
 // f16_codes = 1 writes each INT8 code as the equal f16 value ([M, K] f16).
+// qmax: 127 (INT8) or 31 (INT6 codes in int8 / f16 containers).
 ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadamard, void* codes,
-                                  float* scales, cudaStream_t st, int f16_codes = 0);
+                                  float* scales, cudaStream_t st, int f16_codes = 0, int qmax = 127);
 ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int32_t Kp,
                                         const int32_t* gather, const float* amax_in, void* codes,
-                                        float* scale_out, cudaStream_t st);
+                                        float* scale_out, cudaStream_t st, int qmax = 127);
 ql_status launch_gamma_route(const void* in, const void* out, int64_t numel, float threshold,
                              double* gamma, int32_t* route, void* ws, cudaStream_t st);
 ql_status launch_qarvd_prepare(const void* W, int32_t N, int32_t K, float tau, float alpha,

@@ -427,15 +427,15 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
 // F16 = true writes each code as the equal f16 value (an integer in
 // [-127, 127], exact), the operand layout of the f16 MMA.
 template <bool F16>
-__device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv, uint8_t* dst) {
+__device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv, int qmax, uint8_t* dst) {
   if constexpr (F16) {
     uint32_t w[32];   // element pairs (4i+b) and (32+4i+b) -> f16 words
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int ql0 = max(-127, min(127, __float2int_rn(__fmul_rn(P[2 * i].x, inv))));
-      const int ql1 = max(-127, min(127, __float2int_rn(__fmul_rn(P[2 * i + 1].x, inv))));
-      const int qh0 = max(-127, min(127, __float2int_rn(__fmul_rn(P[2 * i].y, inv))));
-      const int qh1 = max(-127, min(127, __float2int_rn(__fmul_rn(P[2 * i + 1].y, inv))));
+      const int ql0 = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[2 * i].x, inv))));
+      const int ql1 = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[2 * i + 1].x, inv))));
+      const int qh0 = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[2 * i].y, inv))));
+      const int qh1 = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[2 * i + 1].y, inv))));
       const __half2 lo = __halves2half2(__int2half_rn(ql0), __int2half_rn(ql1));
       const __half2 hi = __halves2half2(__int2half_rn(qh0), __int2half_rn(qh1));
       w[i] = *reinterpret_cast<const uint32_t*>(&lo);          // elements 2i, 2i+1
@@ -451,8 +451,8 @@ __device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv
       uint32_t lo = 0, hi = 0;
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        const int ql = max(-127, min(127, __float2int_rn(__fmul_rn(P[4 * i + b].x, inv))));
-        const int qh = max(-127, min(127, __float2int_rn(__fmul_rn(P[4 * i + b].y, inv))));
+        const int ql = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[4 * i + b].x, inv))));
+        const int qh = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[4 * i + b].y, inv))));
         lo |= (static_cast<uint32_t>(ql) & 0xFFu) << (8 * b);
         hi |= (static_cast<uint32_t>(qh) & 0xFFu) << (8 * b);
       }
@@ -468,7 +468,7 @@ __device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv
 template <bool F16>
 __global__ void __launch_bounds__(kThreadsHbm)
     k_quant_int8_token(const __grid_constant__ CUtensorMap tm_x, int64_t M, int32_t K, int hadamard,
-                       int32_t buf_bytes, int32_t box_rows, uint8_t* __restrict__ codes,
+                       int32_t buf_bytes, int32_t box_rows, int qmax, uint8_t* __restrict__ codes,
                        float* __restrict__ scales, int* status) {
   extern __shared__ uint8_t s_raw[];
   __shared__ uint64_t bars[2 * (kThreadsHbm / 32)];
@@ -521,14 +521,15 @@ __global__ void __launch_bounds__(kThreadsHbm)
         m = fmax3(m, fmax3(fabsf(P[j].x), fabsf(P[j].y), fabsf(P[j + 1].x)), fabsf(P[j + 1].y));
     }
     m = warp_max(m);
-    const float inv = (m == 0.f) ? 0.f : __fdiv_rn(127.f, m);
-    if (lane == 0) scales[r] = (m == 0.f) ? 0.f : __fdiv_rn(m, 127.f);
+    const float fq = static_cast<float>(qmax);
+    const float inv = (m == 0.f) ? 0.f : __fdiv_rn(fq, m);
+    if (lane == 0) scales[r] = (m == 0.f) ? 0.f : __fdiv_rn(m, fq);
     constexpr int kElemBytes = F16 ? 2 : 1;
     uint8_t* crow = codes + r * K * kElemBytes;
     for (int p = 0; p < passes; ++p) {
       if (passes > 1) load_half(row, p, P);    // one pass: P still holds the rotated half
       const int32_t hb = 32 * p + static_cast<int32_t>(lane);
-      if (hb < halves) quant_int8_half<F16>(P, inv, crow + 64 * kElemBytes * hb);
+      if (hb < halves) quant_int8_half<F16>(P, inv, qmax, crow + 64 * kElemBytes * hb);
     }
     __syncwarp();
   }
@@ -562,7 +563,7 @@ constexpr int kPermThreads = 256;
 
 __global__ void __launch_bounds__(kPermThreads)
     k_quant_int8_tensor_perm(const uint8_t* __restrict__ x, int64_t M, int32_t K, int32_t Kp,
-                             const int32_t* __restrict__ gather, const float* __restrict__ amax_in,
+                             const int32_t* __restrict__ gather, const float* __restrict__ amax_in, int qmax,
                              int8_t* __restrict__ codes, float* __restrict__ scale_out) {
   extern __shared__ __align__(16) uint8_t s_perm[];
   const PermLayout L(K, Kp);
@@ -571,8 +572,9 @@ __global__ void __launch_bounds__(kPermThreads)
   uint32_t* orow = reinterpret_cast<uint32_t*>(s_perm + L.gather_bytes + 2 * L.row_bytes);
   for (int i = threadIdx.x; i < Kp; i += blockDim.x) s_gather[i] = static_cast<int16_t>(gather[i]);
   const float amax = __ldg(amax_in);
-  const float inv = (amax == 0.f) ? 0.f : __fdiv_rn(127.f, amax);
-  if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = (amax == 0.f) ? 0.f : __fdiv_rn(amax, 127.f);
+  const float fq = static_cast<float>(qmax);
+  const float inv = (amax == 0.f) ? 0.f : __fdiv_rn(fq, amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = (amax == 0.f) ? 0.f : __fdiv_rn(amax, fq);
   auto issue_row = [&](int64_t r, uint8_t* dst) {
     const uint8_t* src = x + r * L.row_bytes;
     const uint32_t d = smem_u32(dst);
@@ -584,7 +586,7 @@ __global__ void __launch_bounds__(kPermThreads)
   auto q8 = [&](const unsigned short* xr, int32_t src) -> uint32_t {
     if (src < 0) return 0u;
     const float v = __uint_as_float(static_cast<uint32_t>(xr[src]) << 16);
-    return static_cast<uint32_t>(max(-127, min(127, __float2int_rn(__fmul_rn(v, inv))))) & 0xFFu;
+    return static_cast<uint32_t>(max(-qmax, min(qmax, __float2int_rn(__fmul_rn(v, inv))))) & 0xFFu;
   };
   issue_row(blockIdx.x, rows[0]);
   cp_async_commit();
@@ -719,7 +721,7 @@ ql_status launch_expand_nvfp4_f16(const void* codes, const void* sf, int32_t N, 
 }
 
 ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadamard, void* codes,
-                                  float* scales, cudaStream_t st, int f16_codes) {
+                                  float* scales, cudaStream_t st, int f16_codes, int qmax) {
   if (M == 0) return QL_OK;
   // a token row is K/64 rows of 128 bytes; TMA boxes of at most 256 rows that tile it exactly
   const int32_t halves = K / 64;
@@ -737,21 +739,21 @@ ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadam
   if (!make_stream_tmap(&tm, x, M * K * 2, static_cast<uint32_t>(box_rows))) return QL_ERR_CUDA;
   auto kern = f16_codes ? k_quant_int8_token<true> : k_quant_int8_token<false>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), static_cast<int>(smem))) return QL_ERR_CUDA;
-  kern<<<grid, 32 * warps, smem, st>>>(tm, M, K, hadamard, static_cast<int32_t>(buf), box_rows,
+  kern<<<grid, 32 * warps, smem, st>>>(tm, M, K, hadamard, static_cast<int32_t>(buf), box_rows, qmax,
                                        static_cast<uint8_t*>(codes), scales, status_word());
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
 ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int32_t Kp,
                                         const int32_t* gather, const float* amax_in, void* codes,
-                                        float* scale_out, cudaStream_t st) {
+                                        float* scale_out, cudaStream_t st, int qmax) {
   const PermLayout L(K, Kp);
   if (L.total > 200 * 1024) return QL_ERR_UNSUPPORTED_SHAPE;
   const int per_sm = std::max(1, std::min(4, (220 * 1024) / L.total));
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(M, static_cast<int64_t>(per_sm) * num_sms())));
   if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_int8_tensor_perm), L.total)) return QL_ERR_CUDA;
   k_quant_int8_tensor_perm<<<grid, kPermThreads, L.total, st>>>(static_cast<const uint8_t*>(x), M, K, Kp, gather,
-                                                                amax_in, static_cast<int8_t*>(codes), scale_out);
+                                                                amax_in, qmax, static_cast<int8_t*>(codes), scale_out);
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 

@@ -29,6 +29,9 @@ QL_ROUTE_INT8 = 1
 QL_ACT_INT8_TENSOR = 2
 QL_ACT_INT8_F16 = 3
 QL_ACT_NVFP4_DECOMP = 4
+QL_ROUTE_INT6 = 5
+QL_ACT_INT6_F16 = 6
+QL_ACT_INT6_TENSOR = 7
 
 
 class WeightCfg(C.Structure):
@@ -230,10 +233,10 @@ def qlinear_quantize_act(X: torch.Tensor, act_fmt: int, hadamard: bool = True,
         if rowmajor_scales:
             sf_rm = torch.empty((M, kq // 16), dtype=torch.uint8, device=dev)
         scales = torch.empty(1, dtype=torch.float32, device=dev)
-    elif act_fmt == QL_ROUTE_INT8:
+    elif act_fmt in (QL_ROUTE_INT8, QL_ROUTE_INT6):
         codes = torch.empty((M, K), dtype=torch.int8, device=dev)
         scales = torch.empty(max(M, 1), dtype=torch.float32, device=dev)
-    elif act_fmt == QL_ACT_INT8_F16:
+    elif act_fmt in (QL_ACT_INT8_F16, QL_ACT_INT6_F16):
         codes = torch.empty((M, K), dtype=torch.float16, device=dev)
         scales = torch.empty(max(M, 1), dtype=torch.float32, device=dev)
     else:

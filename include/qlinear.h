@@ -96,12 +96,20 @@ typedef enum {
   QL_ACT_INT8_F16 = 3,      /* W4A8: per-token INT8 codes stored as the equal
                                f16 values, f16 [M, K]; the GEMM needs weights
                                prepared with expand_f16                      */
-  QL_ACT_NVFP4_DECOMP = 4   /* activation decomposition (SemanticDialect,
+  QL_ACT_NVFP4_DECOMP = 4,  /* activation decomposition (SemanticDialect,
                                Methodology 2.2): NVFP4 of h, then NVFP4 of the
                                residual r = RN(h - RN(e2m1(q1) RN(sb1 g))) with
                                the same tensor scale g; codes [M, K] bytes =
                                [q1 | q2] per row, scales over K' = 2K (q1's
                                first); the GEMM needs QL_W_NVFP4_DECOMP      */
+  /* W4A6: 6-bit signed integer activations, symmetric [-31, 31], the INT8
+     recipes with 31 in place of 127, in 8-bit (or f16) containers that the
+     integer GEMMs multiply exactly. */
+  QL_ROUTE_INT6 = 5,        /* per-token INT6 (int8 [M, K] + fp32 [M]); also
+                               a qlinear_forward route                        */
+  QL_ACT_INT6_F16 = 6,      /* per-token INT6 codes as f16 values (weights with
+                               expand_f16)                                    */
+  QL_ACT_INT6_TENSOR = 7    /* Q-ARVD per-tensor INT6 in the permuted K order  */
 } ql_act_format;
 
 typedef struct {
@@ -256,15 +264,21 @@ QL_API ql_status qlinear_quantize_act(const void* X_bf16, int64_t M, int32_t K,
                        both operands go straight to the f16 MMA.
    QL_ACT_INT8_TENSOR: INT8 x INT4 integer MMA, two class accumulators;
                        y = s_x (s_norm[n] acc_normal + s_out[n] acc_outlier).
+   QL_ACT_NVFP4_DECOMP: the W4A4 GEMM over K' = 2K ([q1 | q2] x [W | W]).
+   QL_ROUTE_INT6, QL_ACT_INT6_F16, QL_ACT_INT6_TENSOR: as the INT8 formats
+                       (the codes are integers in [-31, 31]).
    Operands are the outputs of qlinear_quantize_act for the same format. */
 QL_API ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf,
                        const float* a_scales, int64_t M, const ql_weights* w,
                        void* Y_bf16, void* stream);
 
 /* ---- forward: quantize + GEMM ----------------------------------------------
-   route: QL_ROUTE_NVFP4 or QL_ROUTE_INT8 for NVFP4 weights (the activation
-   rotation follows w->hadamard); ignored for Q-ARVD weights (per-tensor
-   INT8).  Scratch for the quantized activations lives in `ws`.  On the INT8
+   route: QL_ROUTE_NVFP4, QL_ROUTE_INT8 or QL_ROUTE_INT6 for NVFP4 weights
+   (the activation rotation follows w->hadamard); for Q-ARVD weights
+   QL_ROUTE_INT6 or QL_ACT_INT6_TENSOR selects per-tensor INT6 activations,
+   any other value per-tensor INT8; QL_ROUTE_NVFP4 only for
+   QL_W_NVFP4_DECOMP weights.  Scratch for the quantized activations lives
+   in `ws`.  On the INT8
    route with weights prepared with expand_f16, the INT8 codes are kept as
    the equal f16 values (2 bytes each) so that the GEMM reads both operands
    straight into the f16 MMA. */

@@ -333,3 +333,60 @@ def test_qarvd_activation_quant_and_forward_parity(ql, m, n, k, frac, expand):
     assert np.array_equal(_np(q["codes"]), want)
     ref = O.gemm_qarvd(qxp, sx, pk["codes"], pk["s_norm"], pk["s_out"], pk["k_norm_pad"])
     assert excess_err(_np(y.float()).astype(np.float64), ref) <= 1e-3
+
+
+# ---------------------------------------------------------------- W4A6 (INT6 activations)
+
+@pytest.mark.parametrize("expand", [False, True])
+@pytest.mark.parametrize("m,n,k", [(300, 384, 640), (129, 1920, 1920), (1, 192, 128)])
+def test_w4a6_token_route_parity(ql, m, n, k, expand):
+    """6-bit signed integer activations per token (codes in [-31, 31]) into
+    the INT8-route GEMM: codes and scales bit-exact, product within the INT8
+    tolerance against the oracle's INT6 product."""
+    x = _x(m, k, seed=m + 11 * k)
+    w = S.weights(n, k, 0.02, 7, m + n)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    q6, s6 = O.int8_per_token(O.block_hadamard(O.bf16_bits_to_f32(xb)), O.INT6_QMAX)
+    wq = O.prepare_weights_nvfp4(wb)
+    ref = O.gemm_w4a8_token(q6, s6, wq["packed"], wq["sb"], wq["g"])
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True, expand_f16=expand)
+    xc = x.cuda()
+    q = ql.qlinear_quantize_act(xc, ql.QL_ROUTE_INT6, hadamard=True)
+    y = ql.qlinear_forward(xc, pw, ql.QL_ROUTE_INT6)
+    y2 = ql.qlinear_gemm(ql.QL_ROUTE_INT6, q, m, pw)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    assert np.array_equal(_np(q["codes"]), q6) and np.array_equal(_np(q["scales"])[:m], s6)
+    assert np.abs(q6.astype(int)).max() <= 31
+    assert excess_err(_np(y.float()).astype(np.float64), ref) <= 1e-3
+    assert excess_err(_np(y2.float()).astype(np.float64), ref) <= 1e-3
+    if expand:
+        qf = ql.qlinear_quantize_act(xc, ql.QL_ACT_INT6_F16, hadamard=True)
+        y3 = ql.qlinear_gemm(ql.QL_ACT_INT6_F16, qf, m, pw)
+        torch.cuda.synchronize()
+        assert np.array_equal(_np(qf["codes"].float()), q6.astype(np.float32))
+        assert excess_err(_np(y3.float()).astype(np.float64), ref) <= 1e-3
+
+
+@pytest.mark.parametrize("expand", [False, True])
+@pytest.mark.parametrize("m,n,k", [(300, 384, 640), (77, 128, 128), (600, 576, 1024)])
+def test_w4a6_qarvd_parity(ql, m, n, k, expand):
+    """Q-ARVD with per-tensor INT6 activations (its W4A6 setting)."""
+    w = _qarvd_weights(n, k, seed=m + n + 1)
+    pk = O.qarvd_pack(S.bf16_bits(w), 3.5, 2.0)
+    _assert_guard_band(pk)
+    x = _x(m, k, seed=m + 3 * k)
+    qx, sx = O.int8_per_tensor(O.bf16_bits_to_f32(S.bf16_bits(x)), O.INT6_QMAX)
+    qxp = O.qarvd_permute_activations(qx, pk["perm"], pk["k_norm"], pk["k_norm_pad"], pk["n_out"], pk["k_out_pad"])
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_QARVD_INT4, hadamard=False, expand_i8=expand)
+    xc = x.cuda()
+    q = ql.qlinear_quantize_act(xc, ql.QL_ACT_INT6_TENSOR, hadamard=False, w=pw)
+    y = ql.qlinear_forward(xc, pw, ql.QL_ROUTE_INT6)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    kp = pw.desc.Kp
+    want = np.zeros((m, kp), np.int8)
+    want[:, :qxp.shape[1]] = qxp
+    assert _np(q["scales"])[0] == sx and np.array_equal(_np(q["codes"]), want)
+    ref = O.gemm_qarvd(qxp, sx, pk["codes"], pk["s_norm"], pk["s_out"], pk["k_norm_pad"])
+    assert excess_err(_np(y.float()).astype(np.float64), ref) <= 1e-3
