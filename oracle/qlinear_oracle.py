@@ -470,6 +470,13 @@ def gemm_w4a8_token(q_x, s_x, w_packed, w_sb, g_w, hadamard=True, rows=None) -> 
     return (q @ dq_w.T) * (s[:, None] * np.float64(g_w) / c)
 
 
+def gemm_bf16(x_bits, w_bits, rows=None) -> np.ndarray:
+    """Unquantized product of the bf16 operands, exact in fp64 (PDR's
+    high-precision path): R = X W^T."""
+    x = bf16_bits_to_f32(x_bits if rows is None else x_bits[rows]).astype(np.float64)
+    return x @ bf16_bits_to_f32(w_bits).astype(np.float64).T
+
+
 def gemm_qarvd(q_x_perm, s_x, codes, s_norm, s_out, k_norm_pad, rows=None) -> np.ndarray:
     """Dual-scale integer product: exact int64 class sums, then
     R[m, n] = s_x (s_norm[n] acc_normal + s_out[n] acc_outlier) in fp64."""

@@ -29,8 +29,14 @@ Readings of what the page leaves open (every one listed in the design notes):
   * the route of a computed step is INT8 when the previous step skipped or
     when the block has no Gamma yet (its first step), otherwise Gamma of the
     last computed step > gamma_threshold;
-  * PDR's high-precision refresh on a high input outlier ratio is not part of
-    this (the page does not define the ratio).
+  * PDR's high-precision refresh: the input outlier ratio rho is the
+    fraction of 16-element blocks of the block input (in element order,
+    whole blocks only) dominated by one value: with a = max |x| and s the
+    fp32 sum of |x| over the block (two sequential halves of 8, then their
+    sum), the block counts iff RN(a * 15) > RN(kappa * RN(s - a)), i.e. its
+    largest magnitude exceeds kappa times the mean of the other 15; a
+    computed step whose preceding refresh saw rho > rho_max runs in BF16
+    (this takes precedence over the INT8 / NVFP4 choice).
 """
 from __future__ import annotations
 
@@ -39,6 +45,8 @@ from dataclasses import dataclass, field
 import numpy as np
 
 from .qlinear_oracle import ROUTE_INT8, ROUTE_NVFP4, bf16_bits_to_f32, dmpq_gamma
+
+ROUTE_BF16 = 8   # unquantized bf16 product (PDR's high-precision refresh)
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -71,6 +79,8 @@ class TdcParams:
     eps_threshold: float = 0.1      # skip when the delta change is below this
     acc_max: float = 0.3            # cap on the summed E over a run of skips
     max_skips: int = 3              # cap on consecutive skips
+    kappa: float = 8.0              # outlier block: largest magnitude > kappa x mean of the rest
+    rho_max: float = 1.0            # BF16 when the outlier-block fraction exceeds this
 
 
 @dataclass
@@ -83,6 +93,24 @@ class TdcState:
     acc: float = 0.0
     skips: int = 0
     last_skipped: bool = False
+    rho: float = 0.0
+
+
+def outlier_ratio(inp_bits: np.ndarray, kappa: float) -> float:
+    """Fraction of the 16-element blocks dominated by one value (see the header)."""
+    x = np.abs(bf16_bits_to_f32(inp_bits).ravel())
+    nb = x.size // 16
+    if nb == 0:
+        return 0.0
+    b = x[:nb * 16].reshape(nb, 2, 8)
+    halves = np.zeros((nb, 2), np.float32)
+    for j in range(8):                                           # sequential fp32 sums
+        halves = (halves + b[:, :, j]).astype(np.float32)
+    s = (halves[:, 0] + halves[:, 1]).astype(np.float32)
+    a = b.reshape(nb, 16).max(axis=1)
+    others = (s - a).astype(np.float32)
+    flagged = (a * np.float32(15)).astype(np.float32) > (np.float32(kappa) * others).astype(np.float32)
+    return float(np.count_nonzero(flagged)) / nb
 
 
 def tdc_should_skip(st: TdcState, prm: TdcParams) -> bool:
@@ -91,16 +119,22 @@ def tdc_should_skip(st: TdcState, prm: TdcParams) -> bool:
 
 
 def pdr_route(st: TdcState, prm: TdcParams) -> int:
-    """Route of the next computed step (PDR: INT8 right after a skip)."""
+    """Route of the next computed step (PDR: BF16 after a refresh that saw
+    many outlier blocks, else INT8 right after a skip)."""
+    if st.rho > prm.rho_max:
+        return ROUTE_BF16
     if st.last_skipped:
         return ROUTE_INT8
     return ROUTE_INT8 if st.gamma > prm.gamma_threshold else ROUTE_NVFP4
 
 
-def tdc_after_compute(st: TdcState, inp_bits: np.ndarray, out_bits: np.ndarray) -> None:
+def tdc_after_compute(st: TdcState, inp_bits: np.ndarray, out_bits: np.ndarray,
+                      kappa: float = TdcParams.kappa) -> None:
     """Cache refresh after the block was computed: the new delta, Gamma of
-    this step and E between the new and the previous delta."""
+    this step, E between the new and the previous delta and the input's
+    outlier-block ratio."""
     d = tdc_delta(inp_bits, out_bits)
+    st.rho = outlier_ratio(inp_bits, kappa)
     st.gamma = dmpq_gamma(inp_bits, out_bits)
     st.eps = tdc_delta_error(d, st.deltas[-1]) if st.deltas else float("inf")
     st.deltas = (st.deltas + [d])[-2:]
@@ -124,5 +158,5 @@ def tdc_step(st: TdcState, prm: TdcParams, inp_bits: np.ndarray, block) -> tuple
         return out, True, -1
     route = pdr_route(st, prm)
     out = block(inp_bits, route)
-    tdc_after_compute(st, inp_bits, out)
+    tdc_after_compute(st, inp_bits, out, prm.kappa)
     return out, False, route

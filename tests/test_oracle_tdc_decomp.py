@@ -194,3 +194,49 @@ def test_first_two_steps_always_compute():
     assert st.eps == float("inf") and not T.tdc_should_skip(st, prm)
     T.tdc_after_compute(st, inp, _bf16(np.full(16, 1.5, np.float32)))
     assert st.eps == 0.0 and T.tdc_should_skip(st, prm)
+
+
+# ---------------------------------------------------------------- PDR outlier ratio
+
+def test_outlier_ratio_hand_cases():
+    blocks = np.zeros((4, 16), np.float32)
+    blocks[0] = 1.0                                   # uniform: a*15 = 15, kappa*others = 8*15
+    blocks[1] = 1.0
+    blocks[1, 3] = 9.0                                # 9*15 = 135 > 8*15 = 120: flagged
+    blocks[2] = 1.0
+    blocks[2, 5] = 8.0                                # 8*15 = 120, not > 120: not flagged
+    blocks[3, 0] = -0.5                               # one nonzero value: others = 0, flagged
+    bits = _bf16(blocks.ravel())
+    assert T.outlier_ratio(bits, 8.0) == 0.5
+    assert T.outlier_ratio(bits, 7.0) == 0.75         # 8*15 = 120 > 7*15 = 105
+    assert T.outlier_ratio(_bf16(np.zeros(40, np.float32)), 8.0) == 0.0   # all zero: 0 > 0 is false
+    assert T.outlier_ratio(bits[:15], 8.0) == 0.0     # no whole block
+
+
+def test_outlier_ratio_counts_planted_channels():
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((64, 1920)).astype(np.float32)
+    cols = rng.choice(1920, 19, replace=False)
+    x[:, cols] *= 30.0
+    rho = T.outlier_ratio(_bf16(x), 8.0)
+    blocks_hit = len(set(int(c) // 16 for c in cols))
+    assert abs(rho - blocks_hit / 120) < 0.02          # the blocks holding a planted channel
+    assert T.outlier_ratio(_bf16(rng.standard_normal((64, 1920)).astype(np.float32)), 8.0) < 0.01
+
+
+def test_pdr_bf16_takes_precedence():
+    prm = T.TdcParams(rho_max=0.1)
+    st = T.TdcState(rho=0.2, last_skipped=True, gamma=0.0)
+    assert T.pdr_route(st, prm) == T.ROUTE_BF16
+    st.rho = 0.05
+    assert T.pdr_route(st, prm) == O.ROUTE_INT8
+    st.last_skipped = False
+    assert T.pdr_route(st, prm) == O.ROUTE_NVFP4
+
+
+def test_gemm_bf16_is_the_exact_product():
+    rng = np.random.default_rng(22)
+    xi = rng.integers(-64, 65, (5, 32)).astype(np.float32)
+    wi = rng.integers(-64, 65, (7, 32)).astype(np.float32)
+    r = O.gemm_bf16(_bf16(xi), _bf16(wi))
+    assert np.array_equal(r, (xi.astype(np.int64) @ wi.astype(np.int64).T).astype(np.float64))
