@@ -676,7 +676,13 @@ def run_configs(reps: int = 20):
                                     M_TOKENS * 1920 * (3.0 + 4.0 / 1920)),
         "gemm_w4a8_onchip": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, M_TOKENS, pw, Y=y)),
                                     M_TOKENS, 7680, 1920, 1.0)}
-    del bi, bo, q, q16, y, pw, pwx, wd
+    # PDR's BF16 refresh: the unquantized product of the same FFN-up (bf16
+    # input and kept bf16 weights, kind::f16 with bf16 operands)
+    pwb = ql.qlinear_prepare_weights(wd, ql.QL_W_NVFP4, hadamard=True, keep_bf16=True)
+    out["cfg3_int8_ffn_up"]["gemm_bf16"] = mma_rec(
+        med(lambda: ql.qlinear_gemm(ql.QL_ROUTE_BF16, {"codes": bi, "scales": None}, M_TOKENS, pwb, Y=y)),
+        M_TOKENS, 7680, 1920, 1.0)
+    del bi, bo, q, q16, y, pw, pwx, pwb, wd
     # Temporal delta cache on a sweep block pair [17776, 1920] (6Bit-Diffusion,
     # B.2): the fused refresh reads in, out and the latest delta and writes
     # the new delta (8 B/elem); the skip reads in and the delta and writes

@@ -280,7 +280,8 @@ size_t qlinear_weights_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg) {
   if (cfg == nullptr || N <= 0 || check_k(K) != QL_OK) return 0;
   const size_t n = N, k = K;
   if (cfg->fmt == QL_W_NVFP4)
-    return align256(n * k / 2) + align256(qlinear_sf_bytes(N, K)) + 256 + (cfg->expand_f16 ? align256(n * k * 2) : 0);
+    return align256(n * k / 2) + align256(qlinear_sf_bytes(N, K)) + 256 + (cfg->expand_f16 ? align256(n * k * 2) : 0) +
+           (cfg->keep_bf16 ? align256(n * k * 2) : 0);
   if (cfg->fmt == QL_W_NVFP4_DECOMP) return align256(n * k) + align256(qlinear_sf_bytes(N, 2 * K)) + 256;
   if (cfg->fmt == QL_W_QARVD_INT4) {
     const size_t kp = qarvd_kp(K);
@@ -308,6 +309,7 @@ ql_status qlinear_prepare_weights(const void* W, int32_t N, int32_t K, const ql_
     return QL_ERR_INVALID_ARG;
   if (cfg->fmt != QL_W_NVFP4 && cfg->expand_f16 != 0) return QL_ERR_INVALID_ARG;
   if (cfg->fmt != QL_W_QARVD_INT4 && cfg->expand_i8 != 0) return QL_ERR_INVALID_ARG;
+  if (cfg->fmt != QL_W_NVFP4 && cfg->keep_bf16 != 0) return QL_ERR_INVALID_ARG;
   if (cfg->fmt == QL_W_NVFP4_DECOMP && check_k(2 * K) != QL_OK) return QL_ERR_UNSUPPORTED_SHAPE;
   QL_TRY(check_k(K));
   if (N <= 0 || N % 16 != 0 || N > (1 << 24)) return QL_ERR_UNSUPPORTED_SHAPE;
@@ -361,6 +363,11 @@ ql_status qlinear_prepare_weights(const void* W, int32_t N, int32_t K, const ql_
     if (cfg->expand_f16) {
       w.w16 = c.take<uint16_t>(static_cast<size_t>(N) * K * 2);
       QL_TRY(launch_expand_nvfp4_f16(w.codes, w.sf, N, K, w.w16, st));
+    }
+    if (cfg->keep_bf16) {   // the weights as given, for the unquantized product
+      w.wbf16 = c.take<uint16_t>(static_cast<size_t>(N) * K * 2);
+      if (cudaMemcpyAsync(w.wbf16, W, static_cast<size_t>(N) * K * 2, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return QL_ERR_CUDA;
     }
   } else {
     w.Kp = qarvd_kp(K);
@@ -519,8 +526,15 @@ ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf, c
                        int64_t M, const ql_weights* w, void* Y, void* stream) {
   QL_TRY(check_m(M));
   QL_TRY(check_w(w));
-  if (M > 0 && (a_codes == nullptr || a_scales == nullptr || Y == nullptr)) return QL_ERR_INVALID_ARG;
+  if (M > 0 && (a_codes == nullptr || (a_scales == nullptr && act_fmt != QL_ROUTE_BF16) || Y == nullptr))
+    return QL_ERR_INVALID_ARG;
   act_fmt = int_base_fmt(act_fmt);   // INT6 codes run through the INT8 GEMMs unchanged
+  if (act_fmt == QL_ROUTE_BF16) {      // a_codes: the bf16 input [M, K]; no scales
+    if (w->fmt != QL_W_NVFP4 || w->wbf16 == nullptr || (M > 0 && a_codes == nullptr)) return QL_ERR_INVALID_ARG;
+    if (!aligned(a_codes, 16) || !aligned(Y, 16)) return QL_ERR_ALIGNMENT;
+    QL_TRY(device_ready());
+    return launch_gemm_bf16(a_codes, M, w, Y, static_cast<cudaStream_t>(stream), status_word());
+  }
   if (act_fmt == QL_ROUTE_NVFP4 || act_fmt == QL_ROUTE_INT8 || act_fmt == QL_ACT_INT8_F16) {
     if (w->fmt != QL_W_NVFP4) return QL_ERR_INVALID_ARG;
     if (act_fmt == QL_ACT_INT8_F16 && w->w16 == nullptr) return QL_ERR_INVALID_ARG;
@@ -556,6 +570,7 @@ size_t qlinear_forward_ws_bytes(int64_t M, const ql_weights* w, int32_t route) {
   if (w->fmt == QL_W_QARVD_INT4) return forward_act_bytes(M, w->K, w->Kp, QL_ACT_INT8_TENSOR);
   if (w->fmt == QL_W_NVFP4_DECOMP)
     return route == QL_ROUTE_NVFP4 ? forward_act_bytes(M, w->K, 0, QL_ACT_NVFP4_DECOMP) : 0;
+  if (route == QL_ROUTE_BF16) return w->wbf16 != nullptr ? 256 : 0;
   route = int_base_fmt(route);
   if (route != QL_ROUTE_NVFP4 && route != QL_ROUTE_INT8) return 0;
   return forward_act_bytes(M, w->K, 0, route, w->w16 != nullptr);
@@ -568,6 +583,12 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
   QL_TRY(check_mk(M, w->K));
   if (ws == nullptr || (M > 0 && (X == nullptr || Y == nullptr))) return QL_ERR_INVALID_ARG;
   if (w->fmt == QL_W_NVFP4_DECOMP && route != QL_ROUTE_NVFP4) return QL_ERR_INVALID_ARG;
+  if (route == QL_ROUTE_BF16) {   // PDR's high-precision refresh: the input as it is
+    if (w->fmt != QL_W_NVFP4 || w->wbf16 == nullptr) return QL_ERR_INVALID_ARG;
+    if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256)) return QL_ERR_ALIGNMENT;
+    QL_TRY(device_ready());
+    return launch_gemm_bf16(X, M, w, Y, static_cast<cudaStream_t>(stream), status_word());
+  }
   // W4A6: route QL_ROUTE_INT6 (or QL_ACT_INT6_TENSOR for Q-ARVD weights)
   const int qmax = (route == QL_ROUTE_INT6 || route == QL_ACT_INT6_TENSOR) ? 31 : 127;
   if (w->fmt == QL_W_NVFP4 && route == QL_ACT_INT6_TENSOR) return QL_ERR_INVALID_ARG;

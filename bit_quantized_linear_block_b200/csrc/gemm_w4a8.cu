@@ -26,7 +26,7 @@
 
 namespace ql {
 
-template <int BN, int S, int RS, bool PRE, bool A16>
+template <int BN, int S, int RS, bool PRE, bool A16, bool BF16 = false>
 struct W4A8Cfg {
   static_assert(!A16 || PRE, "f16 activations need pre-expanded weights");
   static constexpr bool XFORM = !(PRE && A16);   // any operand expanded on chip
@@ -54,9 +54,12 @@ struct W4A8Cfg {
   static_assert(BN * 8 % XFORM_THREADS == 0, "B chunks per transform thread");
   static_assert(SMEM <= 232448, "shared memory budget");
   static_assert(2 * BN <= 512, "tensor memory budget");
-  // kind::f16 descriptor: D = F32 (bit 4), A = B = F16 (0), K-major,
-  // N >> 3 at bit 17, M >> 4 at bit 24.
-  static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+  static_assert(!BF16 || (PRE && A16), "the bf16 product takes both operands by TMA");
+  // kind::f16 descriptor: D = F32 (bit 4), A = B = F16 (0) or BF16 (1 at
+  // bits 7 and 10; both operands always the same type), K-major, N >> 3 at
+  // bit 17, M >> 4 at bit 24.
+  static constexpr uint32_t IDESC = (1u << 4) | (BF16 ? ((1u << 7) | (1u << 10)) : 0u) |
+                                    (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 };
 
 // int8 x4 -> two f16x2 words holding the exact values (byte permute builds
@@ -86,11 +89,11 @@ __device__ __forceinline__ bool warp_wait2(uint64_t* a, uint32_t pa, uint64_t* b
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-template <int BN, int S, int RS, bool PRE, bool A16>
+template <int BN, int S, int RS, bool PRE, bool A16, bool BF16>
 __global__ void __launch_bounds__(512, 1)
     k_gemm_w4a8(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
-  using C = W4A8Cfg<BN, S, RS, PRE, A16>;
+  using C = W4A8Cfg<BN, S, RS, PRE, A16, BF16>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -266,7 +269,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp >= 12) {
     // ------------------------------------------------------------ epilogue
-    const float alpha = __fmul_rn(*p.g_w, p.alpha_mul);
+    const float alpha = BF16 ? 1.f : __fmul_rn(*p.g_w, p.alpha_mul);   // the bf16 product is unscaled
     EpilogueState es{};
     int local = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
@@ -288,17 +291,18 @@ __global__ void __launch_bounds__(512, 1)
   if (warp == 10) tmem_dealloc(tmem, 512);
 }
 
-template <int BN, int S, int RS, bool PRE, bool A16>
+template <int BN, int S, int RS, bool PRE, bool A16, bool BF16 = false>
 static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int64_t M,
                                  const ql_weights* w, void* Y, cudaStream_t st, int* status) {
-  using C = W4A8Cfg<BN, S, RS, PRE, A16>;
+  using C = W4A8Cfg<BN, S, RS, PRE, A16, BF16>;
   const int N = w->N, K = w->K;
+  const CUtensorMapDataType t16 = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUtensorMap ta, tb, ty;
-  if (!(A16 ? make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a_codes, K, M, static_cast<int64_t>(K) * 2, C::BK,
+  if (!(A16 ? make_tmap_2d(&ta, t16, a_codes, K, M, static_cast<int64_t>(K) * 2, C::BK,
                            C::BM, CU_TENSOR_MAP_SWIZZLE_128B)
              : make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, K, M, K, C::BK, C::BM,
                             CU_TENSOR_MAP_SWIZZLE_NONE)) ||
-      !(PRE ? make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w->w16, K, N, static_cast<int64_t>(K) * 2, C::BK,
+      !(PRE ? make_tmap_2d(&tb, t16, BF16 ? w->wbf16 : w->w16, K, N, static_cast<int64_t>(K) * 2, C::BK,
                            BN, CU_TENSOR_MAP_SWIZZLE_128B)
             : make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, C::BK / 2, BN,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) ||
@@ -314,7 +318,7 @@ static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int
   p.g_w = w->gscale;
   p.row_scale = a_scales;
   p.alpha_mul = w->hadamard ? (1.0f / 128.0f) : 1.0f;
-  auto kern = k_gemm_w4a8<BN, S, RS, PRE, A16>;
+  auto kern = k_gemm_w4a8<BN, S, RS, PRE, A16, BF16>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int grid = std::min(p.num_tiles, num_sms());
   kern<<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, ty, p);
@@ -336,6 +340,16 @@ ql_status launch_gemm_w4a8(const void* a_codes, const float* a_scales, int64_t M
   }
   if (n192) return launch_w4a8_cfg<192, 2, 6, false, false>(a_codes, a_scales, M, w, Y, st, status);
   return launch_w4a8_cfg<128, 2, 8, false, false>(a_codes, a_scales, M, w, Y, st, status);
+}
+
+// Unquantized bf16 product Y = X W^T (fp32 accumulation) from the bf16 input
+// and the kept bf16 weights: the same kernel with bf16 operand types, both
+// operands by TMA, no scales.
+ql_status launch_gemm_bf16(const void* X, int64_t M, const ql_weights* w, void* Y, cudaStream_t st, int* status) {
+  if (M == 0) return QL_OK;
+  if (w->wbf16 == nullptr) return QL_ERR_UNSUPPORTED_SHAPE;
+  if (w->N % 192 == 0) return launch_w4a8_cfg<192, 1, 4, true, true, true>(X, nullptr, M, w, Y, st, status);
+  return launch_w4a8_cfg<128, 1, 5, true, true, true>(X, nullptr, M, w, Y, st, status);
 }
 
 }  // namespace ql

@@ -15,7 +15,7 @@ constexpr int kMaxPartials = 4096;               // upper bound of any streaming
 constexpr size_t kAmaxPartialBytes = kMaxPartials * sizeof(float);
 constexpr size_t kAmaxWsBytes = kAmaxPartialBytes + 256;   // partials + ticket
 constexpr size_t kRoutePartialBytes = 2 * kMaxPartials * sizeof(double);
-constexpr size_t kTdcPartialBytes = 4 * kMaxPartials * sizeof(double);
+constexpr size_t kTdcPartialBytes = 5 * kMaxPartials * sizeof(double);
 
 int num_sms();
 int* status_word();   // device status word of the current device (see qlinear_device_status)
@@ -64,6 +64,8 @@ ql_status launch_gemm_w4a8(const void* a_codes, const float* a_scales, int64_t M
 // int8 copy [N, Kp] of the Q-ARVD INT4 codes (sign-extended).
 ql_status launch_expand_int4_i8(const void* codes, int32_t N, int32_t Kp, void* out, cudaStream_t st);
 // Uses the int8 weight copy (w->w8) when the weights carry one.
+// Unquantized bf16 product from weights prepared with keep_bf16.
+ql_status launch_gemm_bf16(const void* X, int64_t M, const ql_weights* w, void* Y, cudaStream_t st, int* status);
 ql_status launch_gemm_qarvd(const void* a_codes, const float* s_x, int64_t M, const ql_weights* w,
                             void* Y, cudaStream_t st, int* status);
 

@@ -1,5 +1,6 @@
 // Temporal delta cache ("6Bit-Diffusion", Methodology A.2 and B.2 TDC) with
-// PDR's forced INT8 after a skip (B.3).
+// PDR's forced INT8 after a skip and its BF16 refresh on an outlier-heavy
+// input (B.3).
 //
 // A transformer block's residual delta Delta_t = output - input changes
 // little between adjacent timesteps.  The cache keeps the block's latest two
@@ -17,8 +18,15 @@
 // device state:
 //   skip  iff two deltas are cached, E < eps_threshold,
 //         acc + E <= acc_max and skips < max_skips
-//   route INT8 when the step just taken was a skip (no fresh Gamma: PDR) or
-//         Gamma > gamma_threshold, else NVFP4.
+//   route BF16 when the last refresh saw an outlier-block ratio rho >
+//         rho_max (PDR's high-precision refresh), else INT8 when the step
+//         just taken was a skip (no fresh Gamma: PDR) or Gamma >
+//         gamma_threshold, else NVFP4.
+// rho is the fraction of the input's whole 16-element blocks whose largest
+// magnitude a exceeds kappa times the mean of the other 15 elements:
+// RN(15 a) > RN(kappa RN(s - a)), s the fp32 sum of |x| taken as two
+// sequential halves of 8 and then their sum.  The refresh walks the tensors
+// a block (two 16-byte vectors of each) at a time so one thread sees it all.
 // Arithmetic: fp32 differences of the bf16 values (RN), bf16 rounding RN-even,
 // fp64 sums (their order differs from a sequential sum only by rounding).
 #include "ql_common.cuh"
@@ -27,10 +35,9 @@
 
 namespace ql {
 
-constexpr int kTdcUnroll = 2;   // 16-byte vectors of each tensor in flight per thread
-
 struct TdcSums {
   double d, x, e, p;   // sum |out - in|, sum |in|, sum |D_new - D_prev|, sum |D_prev|
+  unsigned long long nflag;   // outlier blocks of the input
 };
 
 __device__ __forceinline__ uint32_t bf16x2_rn(float lo, float hi) {
@@ -70,52 +77,106 @@ __device__ __forceinline__ uint4 tdc_vec(const uint4& xi, const uint4& yo, const
   return r;
 }
 
-// This thread's share: grid-stride over 16-byte vectors, kTdcUnroll vectors
-// of every tensor loaded before any is used; the < 8-element tail by the
-// first threads (bf16 scalars).
+// |x| of one 16-byte vector in element order: sequential fp32 sum and max.
+__device__ __forceinline__ void abs_half(const uint4& v, float& sum, float& mx) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float a0 = fabsf(bf16_lo(w[k])), a1 = fabsf(bf16_hi(w[k]));
+    sum = __fadd_rn(__fadd_rn(sum, a0), a1);
+    mx = fmax3(mx, a0, a1);
+  }
+}
+
+// One 16-element block: the new delta's two vectors, the sums and the
+// outlier test on the input.
+template <bool PREV>
+__device__ __forceinline__ void tdc_block(const uint4 (&xi)[2], const uint4 (&yo)[2], const uint4 (&pv)[2],
+                                          uint4 (&dn)[2], float kappa, TdcSums& s) {
+  float h0 = 0.f, h1 = 0.f, a = 0.f;
+  dn[0] = tdc_vec<PREV>(xi[0], yo[0], pv[0], s);
+  dn[1] = tdc_vec<PREV>(xi[1], yo[1], pv[1], s);
+  abs_half(xi[0], h0, a);
+  abs_half(xi[1], h1, a);
+  const float others = __fsub_rn(__fadd_rn(h0, h1), a);
+  s.nflag += (__fmul_rn(a, 15.f) > __fmul_rn(kappa, others)) ? 1ull : 0ull;
+}
+
+// This thread's share: grid-stride over 16-element blocks, two blocks of
+// every tensor loaded before either is used; the < 16-element tail (outside
+// the outlier test) by the first threads as bf16 scalars.
 template <bool PREV>
 __device__ __forceinline__ void tdc_thread(const uint4* __restrict__ in, const uint4* __restrict__ out,
                                            const uint4* __restrict__ prev, uint4* __restrict__ dst,
-                                           int64_t numel, TdcSums& s) {
-  const int64_t nvec = numel >> 3;
+                                           int64_t numel, float kappa, TdcSums& s) {
+  const int64_t nblk = numel >> 4;
   const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nthr = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  int64_t i = tid;
-  for (; i + (kTdcUnroll - 1) * nthr < nvec; i += kTdcUnroll * nthr) {
-    uint4 a[kTdcUnroll], b[kTdcUnroll], c[kTdcUnroll];
+  const uint4 z = make_uint4(0, 0, 0, 0);
+  int64_t b = tid;
+  for (; b + nthr < nblk; b += 2 * nthr) {
+    uint4 x[2][2], y[2][2], p[2][2], d[2][2];
 #pragma unroll
-    for (int u = 0; u < kTdcUnroll; ++u) {
-      a[u] = __ldcs(in + i + u * nthr);
-      b[u] = __ldcs(out + i + u * nthr);
-      c[u] = PREV ? __ldcs(prev + i + u * nthr) : make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < 2; ++u) {
+      const int64_t v = 2 * (b + u * nthr);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        x[u][h] = __ldcs(in + v + h);
+        y[u][h] = __ldcs(out + v + h);
+        p[u][h] = PREV ? __ldcs(prev + v + h) : z;
+      }
     }
 #pragma unroll
-    for (int u = 0; u < kTdcUnroll; ++u) dst[i + u * nthr] = tdc_vec<PREV>(a[u], b[u], c[u], s);
+    for (int u = 0; u < 2; ++u) {
+      tdc_block<PREV>(x[u], y[u], p[u], d[u], kappa, s);
+      const int64_t v = 2 * (b + u * nthr);
+      dst[v] = d[u][0];
+      dst[v + 1] = d[u][1];
+    }
   }
-  for (; i < nvec; i += nthr)
-    dst[i] = tdc_vec<PREV>(__ldcs(in + i), __ldcs(out + i), PREV ? __ldcs(prev + i) : make_uint4(0, 0, 0, 0), s);
-  if (tid < (numel & 7)) {
-    const int64_t e = (nvec << 3) + tid;
-    const uint32_t x = reinterpret_cast<const unsigned short*>(in)[e];
-    const uint32_t y = reinterpret_cast<const unsigned short*>(out)[e];
-    const uint32_t p = PREV ? reinterpret_cast<const unsigned short*>(prev)[e] : 0u;
-    const uint32_t dn = tdc_pair<PREV>(x, y, p, s);   // low halves carry the element; the high halves are 0
+  for (; b < nblk; b += nthr) {
+    uint4 x[2], y[2], p[2], d[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      x[h] = __ldcs(in + 2 * b + h);
+      y[h] = __ldcs(out + 2 * b + h);
+      p[h] = PREV ? __ldcs(prev + 2 * b + h) : z;
+    }
+    tdc_block<PREV>(x, y, p, d, kappa, s);
+    dst[2 * b] = d[0];
+    dst[2 * b + 1] = d[1];
+  }
+  if (tid < (numel & 15)) {
+    const int64_t e = (nblk << 4) + tid;
+    const uint32_t xv = reinterpret_cast<const unsigned short*>(in)[e];
+    const uint32_t yv = reinterpret_cast<const unsigned short*>(out)[e];
+    const uint32_t pv = PREV ? reinterpret_cast<const unsigned short*>(prev)[e] : 0u;
+    const uint32_t dn = tdc_pair<PREV>(xv, yv, pv, s);   // low halves carry the element; the high halves are 0
     reinterpret_cast<unsigned short*>(dst)[e] = static_cast<unsigned short>(dn & 0xFFFFu);
   }
 }
 
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
 __device__ __forceinline__ void block_sum4(TdcSums& s) {
   __shared__ double red[4][32];
+  __shared__ unsigned long long redn[32];
   s.d = warp_sum_f64(s.d);
   s.x = warp_sum_f64(s.x);
   s.e = warp_sum_f64(s.e);
   s.p = warp_sum_f64(s.p);
+  s.nflag = warp_sum_u64(s.nflag);
   const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
   if (lane_id() == 0) {
     red[0][w] = s.d;
     red[1][w] = s.x;
     red[2][w] = s.e;
     red[3][w] = s.p;
+    redn[w] = s.nflag;
   }
   __syncthreads();
   if (w == 0) {
@@ -124,6 +185,7 @@ __device__ __forceinline__ void block_sum4(TdcSums& s) {
     s.x = warp_sum_f64(in ? red[1][lane_id()] : 0.0);
     s.e = warp_sum_f64(in ? red[2][lane_id()] : 0.0);
     s.p = warp_sum_f64(in ? red[3][lane_id()] : 0.0);
+    s.nflag = warp_sum_u64(in ? redn[lane_id()] : 0ull);
   }
   __syncthreads();
 }
@@ -134,7 +196,8 @@ __device__ __forceinline__ void tdc_decide(ql_tdc_state* st, const ql_tdc_params
                    st->acc + st->eps <= static_cast<double>(prm.acc_max) && st->skips < prm.max_skips)
                       ? 1
                       : 0;
-  st->next_route = (st->last_skipped != 0 || st->gamma > static_cast<double>(prm.gamma_threshold))
+  st->next_route = (st->rho > static_cast<double>(prm.rho_max)) ? QL_ROUTE_BF16
+                   : (st->last_skipped != 0 || st->gamma > static_cast<double>(prm.gamma_threshold))
                        ? QL_ROUTE_INT8
                        : QL_ROUTE_NVFP4;
 }
@@ -143,6 +206,7 @@ __global__ void k_tdc_init(ql_tdc_state* st) {
   st->gamma = inf_f64();   // no Gamma yet: the first step runs INT8
   st->eps = inf_f64();
   st->acc = 0.0;
+  st->rho = 0.0;
   st->n_delta = 0;
   st->cur = 1;             // the first delta goes to slot 0
   st->skips = 0;
@@ -164,36 +228,40 @@ __global__ void __launch_bounds__(kThreadsHbm)
   const bool has_prev = n_delta >= 1;
   const uint4* prev = cur ? slot1 : slot0;
   uint4* dst = cur ? slot0 : slot1;
-  TdcSums s{0.0, 0.0, 0.0, 0.0};
+  TdcSums s{0.0, 0.0, 0.0, 0.0, 0ull};
   if (has_prev)
-    tdc_thread<true>(in, out, prev, dst, numel, s);
+    tdc_thread<true>(in, out, prev, dst, numel, prm.kappa, s);
   else
-    tdc_thread<false>(in, out, prev, dst, numel, s);
+    tdc_thread<false>(in, out, prev, dst, numel, prm.kappa, s);
   __shared__ bool s_last;
   block_sum4(s);
   if (threadIdx.x == 0) {
-    partials[4 * blockIdx.x + 0] = s.d;
-    partials[4 * blockIdx.x + 1] = s.x;
-    partials[4 * blockIdx.x + 2] = s.e;
-    partials[4 * blockIdx.x + 3] = s.p;
+    partials[5 * blockIdx.x + 0] = s.d;
+    partials[5 * blockIdx.x + 1] = s.x;
+    partials[5 * blockIdx.x + 2] = s.e;
+    partials[5 * blockIdx.x + 3] = s.p;
+    partials[5 * blockIdx.x + 4] = __longlong_as_double(static_cast<long long>(s.nflag));   // bit pattern
     __threadfence();
     s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  TdcSums t{0.0, 0.0, 0.0, 0.0};
+  TdcSums t{0.0, 0.0, 0.0, 0.0, 0ull};
   const volatile double* pp = partials;
   for (unsigned int b = threadIdx.x; b < gridDim.x; b += blockDim.x) {
-    t.d += pp[4 * b + 0];
-    t.x += pp[4 * b + 1];
-    t.e += pp[4 * b + 2];
-    t.p += pp[4 * b + 3];
+    t.d += pp[5 * b + 0];
+    t.x += pp[5 * b + 1];
+    t.e += pp[5 * b + 2];
+    t.p += pp[5 * b + 3];
+    t.nflag += static_cast<unsigned long long>(__double_as_longlong(pp[5 * b + 4]));
   }
   block_sum4(t);
   if (threadIdx.x == 0) {
     st->gamma = (t.x == 0.0) ? inf_f64() : t.d / t.x;
     st->eps = (!has_prev || t.p == 0.0) ? inf_f64() : t.e / t.p;
+    const int64_t nblk = numel >> 4;
+    st->rho = nblk ? static_cast<double>(t.nflag) / static_cast<double>(nblk) : 0.0;
     st->n_delta = min(n_delta + 1, 2);
     st->cur = 1 - cur;
     st->acc = 0.0;
@@ -253,7 +321,7 @@ ql_status launch_tdc_init(ql_tdc_state* st, cudaStream_t s) {
 
 ql_status launch_tdc_refresh(const void* in, const void* out, int64_t numel, void* slot0, void* slot1,
                              ql_tdc_state* st, const ql_tdc_params& prm, void* ws, cudaStream_t s) {
-  const int grid = hbm_grid(std::max<int64_t>(1, (numel / 8 + kThreadsHbm - 1) / kThreadsHbm), 1);
+  const int grid = hbm_grid(std::max<int64_t>(1, (numel / 16 + kThreadsHbm - 1) / kThreadsHbm), 1);
   double* partials = static_cast<double*>(ws);
   unsigned int* ticket = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + kTdcPartialBytes);
   k_tdc_refresh<<<grid, kThreadsHbm, 0, s>>>(static_cast<const uint4*>(in), static_cast<const uint4*>(out),

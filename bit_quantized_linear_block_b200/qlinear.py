@@ -32,11 +32,13 @@ QL_ACT_NVFP4_DECOMP = 4
 QL_ROUTE_INT6 = 5
 QL_ACT_INT6_F16 = 6
 QL_ACT_INT6_TENSOR = 7
+QL_ROUTE_BF16 = 8
 
 
 class WeightCfg(C.Structure):
     _fields_ = [("fmt", C.c_int32), ("hadamard", C.c_int32), ("tau", C.c_float), ("alpha", C.c_float),
-                ("expand_f16", C.c_int32), ("expand_i8", C.c_int32)]
+                ("expand_f16", C.c_int32), ("expand_i8", C.c_int32), ("keep_bf16", C.c_int32),
+                ("reserved", C.c_int32)]
 
 
 class Weights(C.Structure):
@@ -45,11 +47,11 @@ class Weights(C.Structure):
                 ("codes", C.c_void_p), ("sf", C.c_void_p), ("gscale", C.c_void_p),
                 ("outlier_mask", C.c_void_p), ("perm", C.c_void_p), ("gather", C.c_void_p),
                 ("kinfo", C.c_void_p), ("s_norm", C.c_void_p), ("s_out", C.c_void_p),
-                ("norms", C.c_void_p), ("w16", C.c_void_p), ("w8", C.c_void_p)]
+                ("norms", C.c_void_p), ("w16", C.c_void_p), ("w8", C.c_void_p), ("wbf16", C.c_void_p)]
 
 
 class TdcState(C.Structure):
-    _fields_ = [("gamma", C.c_double), ("eps", C.c_double), ("acc", C.c_double),
+    _fields_ = [("gamma", C.c_double), ("eps", C.c_double), ("acc", C.c_double), ("rho", C.c_double),
                 ("n_delta", C.c_int32), ("cur", C.c_int32), ("skips", C.c_int32), ("last_skipped", C.c_int32),
                 ("next_skip", C.c_int32), ("next_route", C.c_int32), ("steps", C.c_int32),
                 ("reserved", C.c_int32)]
@@ -57,7 +59,7 @@ class TdcState(C.Structure):
 
 class TdcParams(C.Structure):
     _fields_ = [("gamma_threshold", C.c_float), ("eps_threshold", C.c_float), ("acc_max", C.c_float),
-                ("max_skips", C.c_int32)]
+                ("max_skips", C.c_int32), ("kappa", C.c_float), ("rho_max", C.c_float)]
 
 
 class QLinearError(RuntimeError):
@@ -150,15 +152,16 @@ class PackedWeights:
 
 def qlinear_prepare_weights(W: torch.Tensor, fmt: int = QL_W_NVFP4, hadamard: bool = True,
                             tau: float = 3.5, alpha: float = 2.0, stream=None,
-                            expand_f16: bool = False, expand_i8: bool = False) -> PackedWeights:
+                            expand_f16: bool = False, expand_i8: bool = False,
+                            keep_bf16: bool = False) -> PackedWeights:
     """expand_f16 (NVFP4 only) also keeps an f16 copy of the dequantized
     weights for the INT8 route's GEMM; expand_i8 (Q-ARVD only) keeps the
-    INT4 codes sign-extended to int8 for the Q-ARVD GEMM."""
+    INT4 codes sign-extended to int8 for the Q-ARVD GEMM; keep_bf16 (NVFP4
+    only) keeps the bf16 weights for the unquantized QL_ROUTE_BF16 product."""
     assert W.dtype == torch.bfloat16 and W.is_cuda and W.dim() == 2 and W.is_contiguous()
     N, K = W.shape
     cfg = WeightCfg(fmt, int(bool(hadamard)) if fmt in (QL_W_NVFP4, QL_W_NVFP4_DECOMP) else 0, tau, alpha,
-                    int(bool(expand_f16)),
-                    int(bool(expand_i8)))
+                    int(bool(expand_f16)), int(bool(expand_i8)), int(bool(keep_bf16)), 0)
     wbytes = lib.qlinear_weights_bytes(N, K, C.byref(cfg))
     wsbytes = lib.qlinear_prepare_ws_bytes(N, K, C.byref(cfg))
     if wbytes == 0:
@@ -297,13 +300,13 @@ class TdcCache:
     state (read with ``state()``) and the refresh workspace."""
 
     def __init__(self, numel: int, device, gamma_threshold=0.05, eps_threshold=0.1, acc_max=0.3,
-                 max_skips=3, stream=None):
+                 max_skips=3, kappa=8.0, rho_max=1.0, stream=None):
         self.numel = int(numel)
         # each slot starts on a 16-byte boundary
         self.slots = torch.empty(2, max(8, (self.numel + 7) // 8 * 8), dtype=torch.bfloat16, device=device)
         self.state_buf = torch.zeros(C.sizeof(TdcState), dtype=torch.uint8, device=device)
         self.ws = _bytes(lib.qlinear_tdc_ws_bytes(self.numel), device)
-        self.params = TdcParams(gamma_threshold, eps_threshold, acc_max, int(max_skips))
+        self.params = TdcParams(gamma_threshold, eps_threshold, acc_max, int(max_skips), kappa, rho_max)
         qlinear_tdc_init(self, stream)
 
     def state(self) -> TdcState:

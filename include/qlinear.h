@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define QLINEAR_ABI_VERSION 4
+#define QLINEAR_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define QL_API __attribute__((visibility("default")))
@@ -109,7 +109,11 @@ typedef enum {
                                a qlinear_forward route                        */
   QL_ACT_INT6_F16 = 6,      /* per-token INT6 codes as f16 values (weights with
                                expand_f16)                                    */
-  QL_ACT_INT6_TENSOR = 7    /* Q-ARVD per-tensor INT6 in the permuted K order  */
+  QL_ACT_INT6_TENSOR = 7,   /* Q-ARVD per-tensor INT6 in the permuted K order  */
+  QL_ROUTE_BF16 = 8         /* unquantized bf16 product X W^T (PDR's
+                               high-precision refresh); the activations are
+                               the bf16 input itself; needs weights prepared
+                               with keep_bf16                                 */
 } ql_act_format;
 
 typedef struct {
@@ -127,6 +131,9 @@ typedef struct {
                         int8 ([N, Kp], exact) for the GEMM, which then loads
                         both operands by TMA instead of widening the weights
                         on chip.  Costs 1 byte per code in the weight buffer. */
+  int32_t keep_bf16; /* NVFP4: 1 = also keep the bf16 weights [N, K] for the
+                        QL_ROUTE_BF16 product.  2 bytes per weight.          */
+  int32_t reserved;  /* 0                                                      */
 } ql_weight_cfg;
 
 /* Packed weights.  Filled by qlinear_prepare_weights(); every pointer points
@@ -149,6 +156,8 @@ typedef struct {
                             (no g_w); NULL otherwise                            */
   void* w8;              /* Q-ARVD with expand_i8: int8 [N, Kp] = the INT4
                             codes sign-extended; NULL otherwise                 */
+  void* wbf16;           /* NVFP4 with keep_bf16: the bf16 weights [N, K] as
+                            given (not rotated); NULL otherwise                 */
 } ql_weights;
 
 /* ---- library ------------------------------------------------------------ */
@@ -303,12 +312,18 @@ QL_API ql_status qlinear_forward(const void* X_bf16, int64_t M, const ql_weights
                                                           or sum |D_prev| = 0)
      skip next   iff n_delta == 2, E < eps_threshold, acc + E <= acc_max and
                  skips < max_skips  (acc sums E over the current run of skips)
-     next_route  INT8 if the step just taken was a skip or Gamma >
-                 gamma_threshold (strict), else NVFP4; INT8 before any Gamma. */
+     next_route  BF16 if the last refresh saw rho > rho_max; else INT8 if
+                 the step just taken was a skip or Gamma > gamma_threshold
+                 (strict), else NVFP4; INT8 before any Gamma.
+     rho         (PDR) fraction of the input's whole 16-element blocks whose
+                 largest magnitude a exceeds kappa times the mean of the
+                 other 15: RN(a 15) > RN(kappa RN(s - a)), s the fp32 sum
+                 of |x| (two sequential halves of 8, then their sum).       */
 typedef struct {
   double gamma;          /* Gamma of the last computed step                   */
   double eps;            /* E between the two cached deltas                   */
   double acc;            /* summed E over the current run of skips            */
+  double rho;            /* outlier-block ratio of the last refreshed input   */
   int32_t n_delta;       /* cached deltas, 0..2                               */
   int32_t cur;           /* slot (0 or 1) holding the latest delta            */
   int32_t skips;         /* consecutive skips so far                          */
@@ -324,6 +339,9 @@ typedef struct {
   float eps_threshold;   /* skip while E is below this                        */
   float acc_max;         /* cap on the summed E of one run of skips           */
   int32_t max_skips;     /* cap on consecutive skips (>= 0)                   */
+  float kappa;           /* outlier block: largest magnitude > kappa x mean of
+                            the rest (8)                                       */
+  float rho_max;         /* BF16 when rho exceeds this (>= 1: never)           */
 } ql_tdc_params;
 
 /* Reset a block's cache state (device pointer, 8-byte aligned): no deltas,

@@ -63,6 +63,9 @@ def test_size_queries(ql):
             == ql.lib.qlinear_weights_bytes(1920, 1920, C.byref(cfg)) + 1920 * 1920 * 2)
     cq = ql.WeightCfg(ql.QL_W_QARVD_INT4, 0, 3.5, 2.0)
     assert ql.lib.qlinear_weights_bytes(384, 640, C.byref(cq)) >= 384 * (640 + 64) // 2
+    cb = ql.WeightCfg(ql.QL_W_NVFP4, 1, 3.5, 2.0, 0, 0, 1)                        # + bf16 weights
+    assert (ql.lib.qlinear_weights_bytes(1920, 1920, C.byref(cb))
+            == ql.lib.qlinear_weights_bytes(1920, 1920, C.byref(cfg)) + 1920 * 1920 * 2)
     cq8 = ql.WeightCfg(ql.QL_W_QARVD_INT4, 0, 3.5, 2.0, 0, 1)                     # + int8 copy
     assert (ql.lib.qlinear_weights_bytes(384, 640, C.byref(cq8))
             == ql.lib.qlinear_weights_bytes(384, 640, C.byref(cq)) + 384 * 672)    # Kp = 640 + 32

@@ -390,3 +390,34 @@ def test_w4a6_qarvd_parity(ql, m, n, k, expand):
     assert _np(q["scales"])[0] == sx and np.array_equal(_np(q["codes"]), want)
     ref = O.gemm_qarvd(qxp, sx, pk["codes"], pk["s_norm"], pk["s_out"], pk["k_norm_pad"])
     assert excess_err(_np(y.float()).astype(np.float64), ref) <= 1e-3
+
+
+
+# ---------------------------------------------------------------- BF16 (PDR's refresh)
+
+@pytest.mark.parametrize("m,n,k", [(300, 384, 640), (129, 1920, 1920), (1, 640, 128), (1000, 5760, 1920)])
+def test_bf16_route_parity(ql, m, n, k):
+    """The unquantized product X W^T from the kept bf16 weights (fp32
+    accumulation, bf16 out) against the exact fp64 product."""
+    x = _x(m, k, seed=m + 13 * k)
+    w = S.weights(n, k, 0.02, 9, m + n)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    rows = np.arange(m) if m <= 512 else np.unique(np.r_[np.random.default_rng(2).choice(m, 256, replace=False), m - 1])
+    ref = O.gemm_bf16(xb, wb, rows=rows)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True, keep_bf16=True)
+    xc = x.cuda()
+    y = ql.qlinear_forward(xc, pw, ql.QL_ROUTE_BF16)
+    y2 = ql.qlinear_gemm(ql.QL_ROUTE_BF16, {"codes": xc, "scales": None}, m, pw)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    assert torch.equal(pw.view("wbf16", torch.bfloat16, n * k).reshape(n, k).cpu(), w)   # kept as given
+    yn = _np(y.float())[rows].astype(np.float64)
+    assert excess_err(yn, ref) <= 1e-3
+    assert torch.equal(y, y2)
+
+
+def test_bf16_route_needs_kept_weights(ql):
+    w = S.weights(64, 128, 0.02, 9, 3)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True)
+    with pytest.raises(ql.QLinearError):
+        ql.qlinear_forward(_x(8, 128, seed=1).cuda(), pw, ql.QL_ROUTE_BF16)

@@ -37,7 +37,7 @@ def _close(a, b):
 
 def _params(**kw):
     # the device holds the thresholds as fp32: give the oracle the same values
-    p = dict(gamma_threshold=0.05, eps_threshold=0.1, acc_max=0.25, max_skips=3)
+    p = dict(gamma_threshold=0.05, eps_threshold=0.1, acc_max=0.25, max_skips=3, kappa=8.0, rho_max=1.0)
     p.update(kw)
     f = {k: (float(np.float32(v)) if k != "max_skips" else int(v)) for k, v in p.items()}
     return f, T.TdcParams(**f)
@@ -48,6 +48,7 @@ def _params(**kw):
     (8 * 40000 + 3, dict(acc_max=1.0)),            # several CTAs; the skip count caps the runs
     (17776 * 1920 // 8, dict(max_skips=1)),
     (4096, dict(eps_threshold=0.0)),               # never skips
+    (5000 * 16 + 9, dict(rho_max=0.05)),           # outlier-heavy inputs every third step -> BF16 route
 ])
 def test_tdc_sequence_matches_oracle(ql, numel, kw):
     f, prm = _params(**kw)
@@ -56,11 +57,15 @@ def test_tdc_sequence_matches_oracle(ql, numel, kw):
     rng = np.random.default_rng(numel)
     base = rng.standard_normal(numel).astype(np.float32) * 0.1
     pattern = ""
+    seen_bf16 = False
     for step in range(14):
         dev = cache.state()
         want_skip = T.tdc_should_skip(st, prm)
         assert bool(dev.next_skip) == want_skip, step
-        inp_bits = S.bf16_bits(S.to_bf16(rng.standard_normal(numel).astype(np.float32)))
+        xin = rng.standard_normal(numel).astype(np.float32)
+        if step % 3 == 1:
+            xin[::61] *= 40.0          # one dominating value in about a quarter of the 16-blocks
+        inp_bits = S.bf16_bits(S.to_bf16(xin))
         inp = _from_bits(inp_bits).cuda()
         if want_skip:
             out = ql.qlinear_tdc_skip(inp, cache)
@@ -70,6 +75,7 @@ def test_tdc_sequence_matches_oracle(ql, numel, kw):
             pattern += "S"
         else:
             assert dev.next_route == T.pdr_route(st, prm), step
+            seen_bf16 = seen_bf16 or dev.next_route == T.ROUTE_BF16
             # block output: in + a slowly drifting delta, with a jump at step 9
             drift = 1.0 + 0.02 * step + (0.5 if step == 9 else 0.0)
             out_bits = S.bf16_bits(S.to_bf16(
@@ -80,6 +86,7 @@ def test_tdc_sequence_matches_oracle(ql, numel, kw):
             pattern += "C"
         dev = cache.state()
         assert _close(dev.gamma, st.gamma) and _close(dev.eps, st.eps), step
+        assert dev.rho == st.rho, step                 # exact: a ratio of block counts
         assert dev.n_delta == len(st.deltas) and dev.skips == st.skips
         assert bool(dev.last_skipped) == st.last_skipped and dev.steps == step + 1
         assert _close(dev.acc, st.acc) or (dev.acc == 0 and st.acc == 0)
@@ -88,6 +95,8 @@ def test_tdc_sequence_matches_oracle(ql, numel, kw):
         assert "S" in pattern and pattern.count("C") >= 3, pattern
     else:
         assert pattern == "C" * 14
+    if kw.get("rho_max", 1.0) < 1.0:
+        assert seen_bf16, pattern
 
 
 def test_tdc_skip_without_delta_reports(ql):
