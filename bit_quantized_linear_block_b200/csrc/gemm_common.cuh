@@ -3,6 +3,7 @@
 #pragma once
 
 #include <algorithm>
+#include <utility>
 #include "ql_common.cuh"
 
 namespace ql {
@@ -268,6 +269,34 @@ bool make_tmap_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
 bool make_sf_tmap(CUtensorMap* map, const void* base, int64_t rows, int K, uint32_t box_k);
 int num_sms();
 bool set_smem_attr(const void* kernel, int bytes);
+
+// Launch with programmatic stream serialization (the kernel calls
+// pdl_wait_then_release before touching global memory) and, when
+// cluster_x > 1, a cluster of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 void fill_gemm_args(GemmArgs& p, int64_t M, int N, int K, int BN, int* status);
 
 }  // namespace ql

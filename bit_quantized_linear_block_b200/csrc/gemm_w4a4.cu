@@ -192,6 +192,7 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait_then_release();   // everything above touched only shared and tensor memory
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -445,19 +446,8 @@ static ql_status launch_w4a4_cfg(const void* a_codes, const uint8_t* a_sf, const
   auto kern = k_gemm_w4a4<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int units = std::min(p.num_tiles, num_sms() / C::CTAS);
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(units * C::CTAS));
-  cfg.blockDim = dim3(384);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C::CTAS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, tsa, tsb, ty, p) != cudaSuccess) {
+  if (launch_pdl(kern, dim3(static_cast<unsigned>(units * C::CTAS)), dim3(384), C::SMEM, st, C::CTAS, ta, tb,
+                 tsa, tsb, ty, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return QL_ERR_CUDA;
   }

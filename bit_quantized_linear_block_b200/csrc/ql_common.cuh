@@ -300,6 +300,18 @@ __device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t adesc, 
       : "memory");
 }
 
+// ---- programmatic dependent launch -------------------------------------------
+// A kernel launched with the programmatic-stream-serialization attribute may
+// start while its predecessor in the stream is still running.  It calls this
+// before its first access to global memory (read or write): the wait returns
+// once the predecessor has completed and its writes are visible; only then
+// may this kernel's own dependents launch, so every kernel further back has
+// completed too.  Without the attribute both instructions are no-ops.
+__device__ __forceinline__ void pdl_wait_then_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- UMMA descriptors --------------------------------------------------------
 // Shared-memory matrix descriptor (sm_100 "version 1"): start address,
 // leading / stride byte offsets (>> 4), swizzle mode in bits 61-63.

@@ -186,6 +186,7 @@ __global__ void __launch_bounds__(kThreadsHbm, kRingCtasPerSm)
   __shared__ uint64_t bars[kWarpsPerCta * kRing];
   uint8_t* ring_all = ring_base(ring_raw);
   const uint32_t lane = lane_id();
+  pdl_wait_then_release();
   float m = 0.f;
   stream_blocks<kWarpsPerCta>(&tm_x, total_bytes, hadamard, ring_all, bars, status, [&](float2 (&P)[32], int64_t) {
     float2 mm = make_float2(0.f, 0.f);
@@ -349,6 +350,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   __shared__ Nvfp4Tables tab;
   __shared__ uint64_t bars[kQuantWarps * kRing];
   uint8_t* ring_all = ring_base(ring_raw);
+  pdl_wait_then_release();
   const float amax_t = __ldg(amax_in);
   const float g = (amax_t == 0.f) ? 1.f : __fdiv_rn(amax_t, 2688.f);
   if (blockIdx.x == 0 && threadIdx.x == 0 && g_out != nullptr) *g_out = g;
@@ -691,9 +693,12 @@ ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* 
   CUtensorMap tm;
   if (!make_stream_tmap(&tm, x, units * 256)) return QL_ERR_CUDA;
   if (!set_smem_attr(reinterpret_cast<const void*>(k_amax), kRingBytesPerCta + kRingAlignPad)) return QL_ERR_CUDA;
-  k_amax<<<grid, kThreadsHbm, kRingBytesPerCta + kRingAlignPad, st>>>(tm, units * 256, hadamard, partials, ticket,
-                                                                      amax_out, status_word());
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  if (launch_pdl(k_amax, dim3(grid), dim3(kThreadsHbm), kRingBytesPerCta + kRingAlignPad, st, 1, tm, units * 256,
+                 hadamard, partials, ticket, amax_out, status_word()) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
 }
 
 ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, const float* amax_in,
@@ -706,10 +711,13 @@ ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, 
   CUtensorMap tm;
   if (!make_stream_tmap(&tm, x, M * K * 2)) return QL_ERR_CUDA;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), kQuantRingBytes + kRingAlignPad)) return QL_ERR_CUDA;
-  kern<<<grid, kQuantThreads, kQuantRingBytes + kRingAlignPad, st>>>(
-      tm, M, K, hadamard, amax_in, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf_mma),
-      static_cast<uint8_t*>(sf_rm), g_out, status_word());
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  if (launch_pdl(kern, dim3(grid), dim3(kQuantThreads), kQuantRingBytes + kRingAlignPad, st, 1, tm, M, K, hadamard,
+                 amax_in, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf_mma), static_cast<uint8_t*>(sf_rm),
+                 g_out, status_word()) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
 }
 
 ql_status launch_expand_nvfp4_f16(const void* codes, const void* sf, int32_t N, int32_t K, void* out,

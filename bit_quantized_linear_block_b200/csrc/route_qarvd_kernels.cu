@@ -14,6 +14,7 @@
 // class.
 #include "ql_common.cuh"
 #include "route_common.cuh"
+#include "gemm_common.cuh"
 #include "launchers.h"
 
 namespace ql {
@@ -26,6 +27,7 @@ __global__ void __launch_bounds__(kThreadsHbm)
     k_gamma_route(const uint4* __restrict__ in, const uint4* __restrict__ out, int64_t numel,
                   double* __restrict__ partials, unsigned int* __restrict__ ticket, float threshold,
                   double* __restrict__ gamma_out, int32_t* __restrict__ route_out) {
+  pdl_wait_then_release();
   double s1, s0;
   gamma_thread_sums(in, out, numel, s1, s0);
   gamma_finish(s1, s0, partials, ticket, threshold, gamma_out, route_out);
@@ -219,10 +221,12 @@ ql_status launch_gamma_route(const void* in, const void* out, int64_t numel, flo
   const int grid = hbm_grid(std::max<int64_t>(1, (numel / 8 + kThreadsHbm - 1) / kThreadsHbm), 1);
   double* partials = static_cast<double*>(ws);
   unsigned int* ticket = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + kRoutePartialBytes);
-  k_gamma_route<<<grid, kThreadsHbm, 0, st>>>(static_cast<const uint4*>(in),
-                                              static_cast<const uint4*>(out), numel, partials,
-                                              ticket, threshold, gamma, route);
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  if (launch_pdl(k_gamma_route, dim3(grid), dim3(kThreadsHbm), 0, st, 1, static_cast<const uint4*>(in),
+                 static_cast<const uint4*>(out), numel, partials, ticket, threshold, gamma, route) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
 }
 
 int qarvd_slices(int32_t N) { return std::max(1, std::min(64, N / 64)); }
