@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(512, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
+  pdl_wait();   // before the first global access
   // Class sizes (device-resident, written by the weight preparation).
   const int k_norm_pad = p.kinfo[1];
   const int k_out_pad = p.kinfo[3];
@@ -281,6 +282,7 @@ __global__ void __launch_bounds__(512, 1)
     epilogue_finish(es);
   }
 
+  pdl_release();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -354,6 +356,7 @@ __global__ void __launch_bounds__(384, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
+  pdl_wait();   // before the first global access
   const int k_norm_pad = p.kinfo[1];
   const int k_out_pad = p.kinfo[3];
   const int k_used = k_norm_pad + k_out_pad;
@@ -590,6 +593,7 @@ __global__ void __launch_bounds__(384, 1)
     epilogue_warp_finish();
   }
 
+  pdl_release();
   tc_fence_before();
   __syncthreads();
   if constexpr (PAIR) cluster_sync();   // no CTA leaves while its peer may still signal it
@@ -626,19 +630,8 @@ static ql_status launch_qarvd_pre(const void* a_codes, const float* s_x, int64_t
   auto kern = k_gemm_qarvd_pre<PAIR, STAGES, BN_, BK_>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int units = std::min(p.num_tiles, num_sms() / C::CTAS);
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(units * C::CTAS));
-  cfg.blockDim = dim3(384);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = C::CTAS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, p) != cudaSuccess) {
+  if (launch_pdl(kern, dim3(static_cast<unsigned>(units * C::CTAS)), dim3(384), C::SMEM, st, C::CTAS, ta, tb, ty,
+                 p) != cudaSuccess) {
     (void)cudaGetLastError();
     return QL_ERR_CUDA;
   }
@@ -691,8 +684,11 @@ ql_status launch_gemm_qarvd(const void* a_codes, const float* s_x, int64_t M, co
   auto kern = k_gemm_qarvd<S>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int grid = std::min(p.num_tiles, num_sms());
-  kern<<<grid, 512, C::SMEM, st>>>(ta, tb, ty, p);
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  if (launch_pdl(kern, dim3(grid), dim3(512), C::SMEM, st, 1, ta, tb, ty, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
 }
 
 }  // namespace ql

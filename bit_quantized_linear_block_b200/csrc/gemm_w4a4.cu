@@ -192,7 +192,7 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait_then_release();   // everything above touched only shared and tensor memory
+  pdl_wait();   // everything above touched only shared and tensor memory
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -402,6 +402,7 @@ __global__ void __launch_bounds__(384, 1)
     epilogue_warp_finish();
   }
 
+  pdl_release();
   tc_fence_before();
   __syncthreads();
   if constexpr (PAIR) cluster_sync();   // no CTA leaves while its peer may still signal it

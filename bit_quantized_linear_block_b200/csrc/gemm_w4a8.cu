@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();   // everything above touched only shared and tensor memory
 
   if (warp < 8 && C::XFORM) {
     // ------------------------------------------------------------ transform
@@ -285,6 +286,7 @@ __global__ void __launch_bounds__(512, 1)
     epilogue_finish(es);
   }
 
+  pdl_release();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -321,8 +323,11 @@ static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int
   auto kern = k_gemm_w4a8<BN, S, RS, PRE, A16, BF16>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int grid = std::min(p.num_tiles, num_sms());
-  kern<<<grid, C::THREADS, C::SMEM, st>>>(ta, tb, ty, p);
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  if (launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, ta, tb, ty, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
 }
 
 ql_status launch_gemm_w4a8(const void* a_codes, const float* a_scales, int64_t M, const ql_weights* w,

@@ -302,15 +302,16 @@ __device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t adesc, 
 
 // ---- programmatic dependent launch -------------------------------------------
 // A kernel launched with the programmatic-stream-serialization attribute may
-// start while its predecessor in the stream is still running.  It calls this
-// before its first access to global memory (read or write): the wait returns
-// once the predecessor has completed and its writes are visible; only then
-// may this kernel's own dependents launch, so every kernel further back has
-// completed too.  Without the attribute both instructions are no-ops.
-__device__ __forceinline__ void pdl_wait_then_release() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
+// start while its predecessor in the stream is still running.  It calls
+// pdl_wait() before its first access to global memory (read or write): the
+// wait returns once the predecessor has completed and its writes are
+// visible.  pdl_release(), called after the wait once a CTA's main work is
+// done, lets the dependents launch when every CTA has released or exited; a
+// kernel further back has then always completed, and no dependent CTA sits
+// waiting on an SM while this kernel still runs there.  Without the
+// attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---- UMMA descriptors --------------------------------------------------------
 // Shared-memory matrix descriptor (sm_100 "version 1"): start address,

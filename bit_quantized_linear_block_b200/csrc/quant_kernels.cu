@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(kThreadsHbm, kRingCtasPerSm)
   __shared__ uint64_t bars[kWarpsPerCta * kRing];
   uint8_t* ring_all = ring_base(ring_raw);
   const uint32_t lane = lane_id();
-  pdl_wait_then_release();
+  pdl_wait();
   float m = 0.f;
   stream_blocks<kWarpsPerCta>(&tm_x, total_bytes, hadamard, ring_all, bars, status, [&](float2 (&P)[32], int64_t) {
     float2 mm = make_float2(0.f, 0.f);
@@ -197,6 +197,7 @@ __global__ void __launch_bounds__(kThreadsHbm, kRingCtasPerSm)
     }
     m = fmax3(m, mm.x, mm.y);   // blocks past the end hold zeros
   });
+  pdl_release();
   m = warp_max(m);
   __shared__ float red[kWarpsPerCta];
   __shared__ bool s_last;
@@ -350,7 +351,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   __shared__ Nvfp4Tables tab;
   __shared__ uint64_t bars[kQuantWarps * kRing];
   uint8_t* ring_all = ring_base(ring_raw);
-  pdl_wait_then_release();
+  pdl_wait();
   const float amax_t = __ldg(amax_in);
   const float g = (amax_t == 0.f) ? 1.f : __fdiv_rn(amax_t, 2688.f);
   if (blockIdx.x == 0 && threadIdx.x == 0 && g_out != nullptr) *g_out = g;
@@ -405,6 +406,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
       store(1);
     }
   });
+  pdl_release();
   // zero scales of the padding rows of the last 128-row atom
   const int64_t mpad = (M + 127) & ~int64_t(127);
   const int64_t pad_words = (mpad - M) * k_atoms;
@@ -475,6 +477,7 @@ __global__ void __launch_bounds__(kThreadsHbm)
   extern __shared__ uint8_t s_raw[];
   __shared__ uint64_t bars[2 * (kThreadsHbm / 32)];
   uint8_t* s_rows = ring_base(s_raw);
+  pdl_wait();
   const uint32_t lane = lane_id();
   const int wid = threadIdx.x >> 5;
   const int32_t halves = K >> 6;                 // 64-element half blocks (128-byte rows) per token row
@@ -535,6 +538,7 @@ __global__ void __launch_bounds__(kThreadsHbm)
     }
     __syncwarp();
   }
+  pdl_release();
   if (!ok && lane == 0) {   // timed out at iteration k: let this row's and the next row's loads land
     record_error(status, QL_ERR_TIMEOUT);
     const int64_t r = gw + static_cast<int64_t>(k) * nw;
@@ -568,6 +572,7 @@ __global__ void __launch_bounds__(kPermThreads)
                              const int32_t* __restrict__ gather, const float* __restrict__ amax_in, int qmax,
                              int8_t* __restrict__ codes, float* __restrict__ scale_out) {
   extern __shared__ __align__(16) uint8_t s_perm[];
+  pdl_wait();
   const PermLayout L(K, Kp);
   int16_t* s_gather = reinterpret_cast<int16_t*>(s_perm);
   uint8_t* rows[2] = {s_perm + L.gather_bytes, s_perm + L.gather_bytes + L.row_bytes};
@@ -610,6 +615,7 @@ __global__ void __launch_bounds__(kPermThreads)
     for (int32_t o = 16 * static_cast<int32_t>(threadIdx.x); o < Kp; o += 16 * kPermThreads)
       *reinterpret_cast<uint4*>(dst + o) = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(orow) + o);
   }
+  pdl_release();
   cp_async_wait<0>();
 }
 
@@ -747,9 +753,12 @@ ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadam
   if (!make_stream_tmap(&tm, x, M * K * 2, static_cast<uint32_t>(box_rows))) return QL_ERR_CUDA;
   auto kern = f16_codes ? k_quant_int8_token<true> : k_quant_int8_token<false>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), static_cast<int>(smem))) return QL_ERR_CUDA;
-  kern<<<grid, 32 * warps, smem, st>>>(tm, M, K, hadamard, static_cast<int32_t>(buf), box_rows, qmax,
-                                       static_cast<uint8_t*>(codes), scales, status_word());
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  if (launch_pdl(kern, dim3(grid), dim3(32 * warps), smem, st, 1, tm, M, K, hadamard, static_cast<int32_t>(buf),
+                 box_rows, qmax, static_cast<uint8_t*>(codes), scales, status_word()) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
 }
 
 ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int32_t Kp,
@@ -760,9 +769,13 @@ ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int
   const int per_sm = std::max(1, std::min(4, (220 * 1024) / L.total));
   const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(M, static_cast<int64_t>(per_sm) * num_sms())));
   if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_int8_tensor_perm), L.total)) return QL_ERR_CUDA;
-  k_quant_int8_tensor_perm<<<grid, kPermThreads, L.total, st>>>(static_cast<const uint8_t*>(x), M, K, Kp, gather,
-                                                                amax_in, qmax, static_cast<int8_t*>(codes), scale_out);
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  if (launch_pdl(k_quant_int8_tensor_perm, dim3(grid), dim3(kPermThreads), L.total, st, 1,
+                 static_cast<const uint8_t*>(x), M, K, Kp, gather, amax_in, qmax, static_cast<int8_t*>(codes),
+                 scale_out) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
 }
 
 }  // namespace ql

@@ -27,9 +27,10 @@ __global__ void __launch_bounds__(kThreadsHbm)
     k_gamma_route(const uint4* __restrict__ in, const uint4* __restrict__ out, int64_t numel,
                   double* __restrict__ partials, unsigned int* __restrict__ ticket, float threshold,
                   double* __restrict__ gamma_out, int32_t* __restrict__ route_out) {
-  pdl_wait_then_release();
+  pdl_wait();
   double s1, s0;
   gamma_thread_sums(in, out, numel, s1, s0);
+  pdl_release();
   gamma_finish(s1, s0, partials, ticket, threshold, gamma_out, route_out);
 }
 

@@ -31,6 +31,7 @@
 // fp64 sums (their order differs from a sequential sum only by rounding).
 #include "ql_common.cuh"
 #include "route_common.cuh"
+#include "gemm_common.cuh"
 #include "launchers.h"
 
 namespace ql {
@@ -223,6 +224,7 @@ __global__ void __launch_bounds__(kThreadsHbm)
     k_tdc_refresh(const uint4* __restrict__ in, const uint4* __restrict__ out, int64_t numel, uint4* slot0,
                   uint4* slot1, ql_tdc_state* st, const ql_tdc_params prm, double* __restrict__ partials,
                   unsigned int* __restrict__ ticket) {
+  pdl_wait();
   const int cur = st->cur;
   const int n_delta = st->n_delta;
   const bool has_prev = n_delta >= 1;
@@ -233,6 +235,7 @@ __global__ void __launch_bounds__(kThreadsHbm)
     tdc_thread<true>(in, out, prev, dst, numel, prm.kappa, s);
   else
     tdc_thread<false>(in, out, prev, dst, numel, prm.kappa, s);
+  pdl_release();
   __shared__ bool s_last;
   block_sum4(s);
   if (threadIdx.x == 0) {
@@ -278,6 +281,7 @@ __global__ void __launch_bounds__(kThreadsHbm)
 __global__ void __launch_bounds__(kThreadsHbm)
     k_tdc_skip(const uint4* __restrict__ in, int64_t numel, const uint4* slot0, const uint4* slot1,
                ql_tdc_state* st, const ql_tdc_params prm, uint4* __restrict__ out, int* status) {
+  pdl_wait();
   const int cur = st->cur;
   if (st->n_delta < 1) {   // nothing cached: the caller skipped without a delta
     if (blockIdx.x == 0 && threadIdx.x == 0) record_error(status, QL_ERR_INVALID_ARG);
@@ -302,6 +306,7 @@ __global__ void __launch_bounds__(kThreadsHbm)
     const float d = __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const unsigned short*>(dl)[e]) << 16);
     reinterpret_cast<unsigned short*>(out)[e] = static_cast<unsigned short>(bf16x2_rn(__fadd_rn(x, d), 0.f) & 0xFFFFu);
   }
+  pdl_release();
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     st->acc += st->eps;
     st->skips += 1;
@@ -324,19 +329,25 @@ ql_status launch_tdc_refresh(const void* in, const void* out, int64_t numel, voi
   const int grid = hbm_grid(std::max<int64_t>(1, (numel / 16 + kThreadsHbm - 1) / kThreadsHbm), 1);
   double* partials = static_cast<double*>(ws);
   unsigned int* ticket = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + kTdcPartialBytes);
-  k_tdc_refresh<<<grid, kThreadsHbm, 0, s>>>(static_cast<const uint4*>(in), static_cast<const uint4*>(out),
-                                             numel, static_cast<uint4*>(slot0), static_cast<uint4*>(slot1), st,
-                                             prm, partials, ticket);
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  if (launch_pdl(k_tdc_refresh, dim3(grid), dim3(kThreadsHbm), 0, s, 1, static_cast<const uint4*>(in),
+                 static_cast<const uint4*>(out), numel, static_cast<uint4*>(slot0), static_cast<uint4*>(slot1), st, prm,
+                 partials, ticket) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
 }
 
 ql_status launch_tdc_skip(const void* in, int64_t numel, const void* slot0, const void* slot1,
                           ql_tdc_state* st, const ql_tdc_params& prm, void* out, int* status, cudaStream_t s) {
   const int grid = hbm_grid(std::max<int64_t>(1, (numel / 8 + kThreadsHbm - 1) / kThreadsHbm), 1);
-  k_tdc_skip<<<grid, kThreadsHbm, 0, s>>>(static_cast<const uint4*>(in), numel, static_cast<const uint4*>(slot0),
-                                          static_cast<const uint4*>(slot1), st, prm, static_cast<uint4*>(out),
-                                          status);
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  if (launch_pdl(k_tdc_skip, dim3(grid), dim3(kThreadsHbm), 0, s, 1, static_cast<const uint4*>(in), numel,
+                 static_cast<const uint4*>(slot0), static_cast<const uint4*>(slot1), st, prm, static_cast<uint4*>(out),
+                 status) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
 }
 
 }  // namespace ql
