@@ -122,3 +122,48 @@ def test_valid_call_without_a_device_reports_no_device(ql):
     w = ql.Weights(fmt=ql.QL_W_NVFP4, N=1920, K=1920, hadamard=1, codes=FAKE, sf=FAKE, gscale=FAKE)
     assert ql.lib.qlinear_forward(FAKE, 10, C.byref(w), 0, FAKE, FAKE, 1 << 30, None) == 7
 
+
+
+def test_new_entry_points_validate_on_the_host(ql):
+    """TDC, BF16 route, INT6 and decomposition arguments are checked before
+    any CUDA call (no device needed)."""
+    L = ql.lib
+    prm = ql.TdcParams(0.05, 0.1, 0.3, 3, 8.0, 1.0)
+    assert L.qlinear_tdc_init(None, None) == 1
+    assert L.qlinear_tdc_init(FAKE + 4, None) == 3                                   # state not 8-aligned
+    assert L.qlinear_tdc_refresh(FAKE, FAKE, 100, FAKE, FAKE, None, C.byref(prm), FAKE, 1 << 20, None) == 1
+    assert L.qlinear_tdc_refresh(FAKE, FAKE, 100, FAKE, FAKE + 8, FAKE, C.byref(prm), FAKE, 1 << 20, None) == 3
+    assert L.qlinear_tdc_refresh(FAKE, FAKE, 100, FAKE, FAKE, FAKE, C.byref(prm), FAKE, 16, None) == 6
+    nan = ql.TdcParams(0.05, float("nan"), 0.3, 3, 8.0, 1.0)
+    assert L.qlinear_tdc_refresh(FAKE, FAKE, 100, FAKE, FAKE, FAKE, C.byref(nan), FAKE, 1 << 20, None) == 1
+    neg = ql.TdcParams(0.05, 0.1, 0.3, -1, 8.0, 1.0)
+    assert L.qlinear_tdc_skip(FAKE, 100, FAKE, FAKE, FAKE, C.byref(neg), FAKE, None) == 1
+    assert L.qlinear_tdc_skip(FAKE, 100, FAKE, FAKE, FAKE, None, FAKE, None) == 1
+    assert L.qlinear_tdc_ws_bytes(-1) == 0 and L.qlinear_tdc_ws_bytes(1000) > 0
+    # the BF16 route needs kept bf16 weights; other formats reject it
+    w = ql.Weights(fmt=ql.QL_W_NVFP4, N=1920, K=1920, hadamard=1, codes=FAKE, sf=FAKE, gscale=FAKE)
+    assert L.qlinear_gemm(ql.QL_ROUTE_BF16, FAKE, None, None, 10, C.byref(w), FAKE, None) == 1
+    assert L.qlinear_forward_ws_bytes(10, C.byref(w), ql.QL_ROUTE_BF16) == 0
+    wq = ql.Weights(fmt=ql.QL_W_QARVD_INT4, N=256, K=256, codes=FAKE, Kp=256 + 32, gather=FAKE, kinfo=FAKE,
+                    s_norm=FAKE, s_out=FAKE)
+    assert L.qlinear_gemm(ql.QL_ROUTE_BF16, FAKE, None, None, 10, C.byref(wq), FAKE, None) == 1
+    # INT6 formats size like their INT8 counterparts; unknown formats size to 0
+    assert L.qlinear_quantize_ws_bytes(10, 256, ql.QL_ROUTE_INT6) == L.qlinear_quantize_ws_bytes(10, 256, ql.QL_ROUTE_INT8)
+    assert L.qlinear_quantize_ws_bytes(10, 256, ql.QL_ACT_INT6_TENSOR) > 0
+    assert L.qlinear_quantize_ws_bytes(10, 256, 99) == 0
+    # decomposed weights: twice the codes, scales over 2K; not with an f16 or bf16 copy
+    cd = ql.WeightCfg(ql.QL_W_NVFP4_DECOMP, 1, 3.5, 2.0)
+    cn = ql.WeightCfg(ql.QL_W_NVFP4, 1, 3.5, 2.0)
+    assert L.qlinear_weights_bytes(640, 1920, C.byref(cd)) > L.qlinear_weights_bytes(640, 1920, C.byref(cn))
+    desc = ql.Weights()
+    for bad in (ql.WeightCfg(ql.QL_W_NVFP4_DECOMP, 1, 3.5, 2.0, 1, 0, 0), ql.WeightCfg(ql.QL_W_NVFP4_DECOMP, 1, 3.5, 2.0, 0, 0, 1)):
+        assert L.qlinear_prepare_weights(FAKE, 256, 256, C.byref(bad), FAKE, 1 << 30, C.byref(desc),
+                                         FAKE, 1 << 30, None) == 1
+    # decomposed weights run the decomposed NVFP4 route only
+    wd = ql.Weights(fmt=ql.QL_W_NVFP4_DECOMP, N=1920, K=1920, hadamard=1, codes=FAKE, sf=FAKE, gscale=FAKE)
+    assert L.qlinear_forward_ws_bytes(10, C.byref(wd), ql.QL_ROUTE_INT8) == 0
+    assert L.qlinear_forward(FAKE, 10, C.byref(wd), ql.QL_ROUTE_INT8, FAKE, FAKE, 1 << 30, None) == 1
+    # the division test hook
+    assert L.qlinear_debug_div_check(0.0, 0, 10, FAKE, None) == 1
+    assert L.qlinear_debug_div_check(1.0, 0x7F800000, 1, FAKE, None) == 1
+    assert L.qlinear_debug_div_check(1.0, 0, 10, None, None) == 1
