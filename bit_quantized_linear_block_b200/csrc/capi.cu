@@ -637,4 +637,47 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
   return launch_gemm_qarvd(codes, sx, M, w, Y, st, status);
 }
 
+// ---------------------------------------------------------------- forward, device route
+size_t qlinear_forward_routed_ws_bytes(int64_t M, const ql_weights* w) {
+  if (M < 0 || check_w(w) != QL_OK || w->fmt != QL_W_NVFP4) return 0;
+  return forward_act_bytes(M, w->K, 0, QL_ROUTE_NVFP4) +
+         forward_act_bytes(M, w->K, 0, QL_ROUTE_INT8, w->w16 != nullptr);
+}
+
+ql_status qlinear_forward_routed(const void* X, int64_t M, const ql_weights* w, const int32_t* route_dev, void* Y,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  QL_TRY(check_m(M));
+  QL_TRY(check_w(w));
+  QL_TRY(check_mk(M, w->K));
+  if (w->fmt != QL_W_NVFP4 || route_dev == nullptr || ws == nullptr || (M > 0 && (X == nullptr || Y == nullptr)))
+    return QL_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256) || !aligned(route_dev, 4)) return QL_ERR_ALIGNMENT;
+  if (ws_bytes < qlinear_forward_routed_ws_bytes(M, w)) return QL_ERR_WORKSPACE;
+  QL_TRY(device_ready());
+  if (M == 0) return QL_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int K = w->K;
+  Carver c{static_cast<uint8_t*>(ws)};
+  int* status = status_word();
+  const Gate g_fp4{route_dev, QL_ROUTE_NVFP4}, g_int8{route_dev, QL_ROUTE_INT8}, g_bf16{route_dev, QL_ROUTE_BF16};
+  // NVFP4 route
+  void* aws = c.take<uint8_t>(kAmaxWsBytes);
+  float* amax = c.take<float>(256);
+  float* g = c.take<float>(256);
+  uint8_t* codes4 = c.take<uint8_t>(static_cast<size_t>(M) * K / 2);
+  uint8_t* sf = c.take<uint8_t>(qlinear_sf_bytes(M, K));
+  QL_TRY(launch_amax(X, M, K, w->hadamard, amax, aws, st, g_fp4));
+  QL_TRY(launch_quant_nvfp4(X, M, K, w->hadamard, amax, codes4, sf, nullptr, g, st, 0, g_fp4));
+  QL_TRY(launch_gemm_w4a4(codes4, sf, g, M, w, Y, st, status, g_fp4));
+  // INT8 route
+  const int f16 = w->w16 != nullptr ? 1 : 0;
+  uint8_t* codes8 = c.take<uint8_t>(static_cast<size_t>(M) * K * (f16 ? 2 : 1));
+  float* s8 = c.take<float>(4 * static_cast<size_t>(M));
+  QL_TRY(launch_quant_int8_token(X, M, K, w->hadamard, codes8, s8, st, f16, 127, g_int8));
+  QL_TRY(launch_gemm_w4a8(codes8, s8, M, w, Y, st, status, f16, g_int8));
+  // BF16 (PDR's refresh) when the weights were kept
+  if (w->wbf16 != nullptr) QL_TRY(launch_gemm_bf16(X, M, w, Y, st, status, g_bf16));
+  return QL_OK;
+}
+
 }  // extern "C"

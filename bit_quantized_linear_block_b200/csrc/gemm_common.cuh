@@ -30,6 +30,8 @@ struct GemmArgs {
   float alpha_mul;
   long long wait_limit;
   int* status;             // device status word
+  const int32_t* gate;     // device-routed forward: the route in device memory (or null)
+  int32_t gate_value;      // this launch's route
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {

@@ -142,6 +142,13 @@ __global__ void __launch_bounds__(384, 1)
                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                 const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
   using C = W4A4Cfg<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_>;
+  if (p.gate != nullptr) {   // device-routed forward: both CTAs of a pair read the same route
+    pdl_wait();
+    if (gated_off(p.gate, p.gate_value)) {
+      pdl_release();
+      return;
+    }
+  }
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);   // pair: the leader's is used
@@ -421,7 +428,7 @@ __global__ void __launch_bounds__(384, 1)
 template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES, int BKB_ = 128>
 static ql_status launch_w4a4_cfg(const void* a_codes, const uint8_t* a_sf, const float* g_a,
                                  int64_t M, const ql_weights* w, void* Y, cudaStream_t st,
-                                 int* status) {
+                                 int* status, Gate gate) {
   using C = W4A4Cfg<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_>;
   const int N = w->N, K = w->K;
   if (RES && K / 64 > kResKSteps) return QL_ERR_UNSUPPORTED_SHAPE;
@@ -444,6 +451,8 @@ static ql_status launch_w4a4_cfg(const void* a_codes, const uint8_t* a_sf, const
   p.g_a = g_a;
   p.g_w = w->gscale;
   p.alpha_mul = w->hadamard ? (1.0f / 128.0f) : 1.0f;
+  p.gate = gate.route;
+  p.gate_value = gate.value;
   auto kern = k_gemm_w4a4<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int units = std::min(p.num_tiles, num_sms() / C::CTAS);
@@ -456,7 +465,7 @@ static ql_status launch_w4a4_cfg(const void* a_codes, const uint8_t* a_sf, const
 }
 
 ql_status launch_gemm_w4a4(const void* a_codes, const uint8_t* a_sf, const float* g_a, int64_t M,
-                           const ql_weights* w, void* Y, cudaStream_t st, int* status) {
+                           const ql_weights* w, void* Y, cudaStream_t st, int* status, Gate gate) {
   if (M == 0) return QL_OK;
   const bool res = w->K / 64 <= kResKSteps;
   // 192-wide tiles spend fewer tensor-pipe instructions per output column
@@ -469,18 +478,18 @@ ql_status launch_gemm_w4a4(const void* a_codes, const uint8_t* a_sf, const float
   const bool wide = w->N > 128 && 10 * n192 <= 13 * static_cast<int64_t>(w->N);
   if (M > 128) {   // CTA pairs on 256-row tiles
     if (wide) {
-      if (res) return launch_w4a4_cfg<192, 5, true, 2, 3, true>(a_codes, a_sf, g_a, M, w, Y, st, status);
-      return launch_w4a4_cfg<192, 5, true, 2, 3, false>(a_codes, a_sf, g_a, M, w, Y, st, status);
+      if (res) return launch_w4a4_cfg<192, 5, true, 2, 3, true>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
+      return launch_w4a4_cfg<192, 5, true, 2, 3, false>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
     }
-    if (res) return launch_w4a4_cfg<128, 6, true, 2, 2, true>(a_codes, a_sf, g_a, M, w, Y, st, status);
-    return launch_w4a4_cfg<128, 6, true, 2, 2, false>(a_codes, a_sf, g_a, M, w, Y, st, status);
+    if (res) return launch_w4a4_cfg<128, 6, true, 2, 2, true>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
+    return launch_w4a4_cfg<128, 6, true, 2, 2, false>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
   }
   if (wide) {
-    if (res) return launch_w4a4_cfg<192, 4, false, 2, 2, true>(a_codes, a_sf, g_a, M, w, Y, st, status);
-    return launch_w4a4_cfg<192, 4, false, 2, 2, false>(a_codes, a_sf, g_a, M, w, Y, st, status);
+    if (res) return launch_w4a4_cfg<192, 4, false, 2, 2, true>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
+    return launch_w4a4_cfg<192, 4, false, 2, 2, false>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
   }
-  if (res) return launch_w4a4_cfg<128, 5, false, 2, 2, true>(a_codes, a_sf, g_a, M, w, Y, st, status);
-  return launch_w4a4_cfg<128, 5, false, 2, 2, false>(a_codes, a_sf, g_a, M, w, Y, st, status);
+  if (res) return launch_w4a4_cfg<128, 5, false, 2, 2, true>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
+  return launch_w4a4_cfg<128, 5, false, 2, 2, false>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
 }
 
 }  // namespace ql

@@ -94,6 +94,13 @@ __global__ void __launch_bounds__(512, 1)
     k_gemm_w4a8(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
   using C = W4A8Cfg<BN, S, RS, PRE, A16, BF16>;
+  if (p.gate != nullptr) {   // device-routed forward
+    pdl_wait();
+    if (gated_off(p.gate, p.gate_value)) {
+      pdl_release();
+      return;
+    }
+  }
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
@@ -295,7 +302,7 @@ __global__ void __launch_bounds__(512, 1)
 
 template <int BN, int S, int RS, bool PRE, bool A16, bool BF16 = false>
 static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int64_t M,
-                                 const ql_weights* w, void* Y, cudaStream_t st, int* status) {
+                                 const ql_weights* w, void* Y, cudaStream_t st, int* status, Gate gate) {
   using C = W4A8Cfg<BN, S, RS, PRE, A16, BF16>;
   const int N = w->N, K = w->K;
   const CUtensorMapDataType t16 = BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -320,6 +327,8 @@ static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int
   p.g_w = w->gscale;
   p.row_scale = a_scales;
   p.alpha_mul = w->hadamard ? (1.0f / 128.0f) : 1.0f;
+  p.gate = gate.route;
+  p.gate_value = gate.value;
   auto kern = k_gemm_w4a8<BN, S, RS, PRE, A16, BF16>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int grid = std::min(p.num_tiles, num_sms());
@@ -331,30 +340,31 @@ static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int
 }
 
 ql_status launch_gemm_w4a8(const void* a_codes, const float* a_scales, int64_t M, const ql_weights* w,
-                           void* Y, cudaStream_t st, int* status, int a_f16) {
+                           void* Y, cudaStream_t st, int* status, int a_f16, Gate gate) {
   if (M == 0) return QL_OK;
   const bool n192 = w->N % 192 == 0;
   if (a_f16) {   // f16 activations and pre-expanded weights: both operands by TMA
     if (w->w16 == nullptr) return QL_ERR_UNSUPPORTED_SHAPE;
-    if (n192) return launch_w4a8_cfg<192, 1, 4, true, true>(a_codes, a_scales, M, w, Y, st, status);
-    return launch_w4a8_cfg<128, 1, 5, true, true>(a_codes, a_scales, M, w, Y, st, status);
+    if (n192) return launch_w4a8_cfg<192, 1, 4, true, true>(a_codes, a_scales, M, w, Y, st, status, gate);
+    return launch_w4a8_cfg<128, 1, 5, true, true>(a_codes, a_scales, M, w, Y, st, status, gate);
   }
   if (w->w16 != nullptr) {   // weights pre-expanded to f16 at preparation
-    if (n192) return launch_w4a8_cfg<192, 2, 4, true, false>(a_codes, a_scales, M, w, Y, st, status);
-    return launch_w4a8_cfg<128, 2, 5, true, false>(a_codes, a_scales, M, w, Y, st, status);
+    if (n192) return launch_w4a8_cfg<192, 2, 4, true, false>(a_codes, a_scales, M, w, Y, st, status, gate);
+    return launch_w4a8_cfg<128, 2, 5, true, false>(a_codes, a_scales, M, w, Y, st, status, gate);
   }
-  if (n192) return launch_w4a8_cfg<192, 2, 6, false, false>(a_codes, a_scales, M, w, Y, st, status);
-  return launch_w4a8_cfg<128, 2, 8, false, false>(a_codes, a_scales, M, w, Y, st, status);
+  if (n192) return launch_w4a8_cfg<192, 2, 6, false, false>(a_codes, a_scales, M, w, Y, st, status, gate);
+  return launch_w4a8_cfg<128, 2, 8, false, false>(a_codes, a_scales, M, w, Y, st, status, gate);
 }
 
 // Unquantized bf16 product Y = X W^T (fp32 accumulation) from the bf16 input
 // and the kept bf16 weights: the same kernel with bf16 operand types, both
 // operands by TMA, no scales.
-ql_status launch_gemm_bf16(const void* X, int64_t M, const ql_weights* w, void* Y, cudaStream_t st, int* status) {
+ql_status launch_gemm_bf16(const void* X, int64_t M, const ql_weights* w, void* Y, cudaStream_t st, int* status,
+                           Gate gate) {
   if (M == 0) return QL_OK;
   if (w->wbf16 == nullptr) return QL_ERR_UNSUPPORTED_SHAPE;
-  if (w->N % 192 == 0) return launch_w4a8_cfg<192, 1, 4, true, true, true>(X, nullptr, M, w, Y, st, status);
-  return launch_w4a8_cfg<128, 1, 5, true, true, true>(X, nullptr, M, w, Y, st, status);
+  if (w->N % 192 == 0) return launch_w4a8_cfg<192, 1, 4, true, true, true>(X, nullptr, M, w, Y, st, status, gate);
+  return launch_w4a8_cfg<128, 1, 5, true, true, true>(X, nullptr, M, w, Y, st, status, gate);
 }
 
 }  // namespace ql

@@ -313,6 +313,13 @@ __device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t adesc, 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Route gate of the device-routed forward: a launch of one route's kernel
+// returns at once when the route in device memory is another one.  Read
+// after pdl_wait() (an earlier kernel of the stream may have written it).
+__device__ __forceinline__ bool gated_off(const int32_t* route, int32_t value) {
+  return route != nullptr && *reinterpret_cast<const volatile int32_t*>(route) != value;
+}
+
 // ---- UMMA descriptors --------------------------------------------------------
 // Shared-memory matrix descriptor (sm_100 "version 1"): start address,
 // leading / stride byte offsets (>> 4), swizzle mode in bits 61-63.

@@ -181,12 +181,16 @@ __device__ __forceinline__ void stream_blocks(const CUtensorMap* tm, int64_t tot
 __global__ void __launch_bounds__(kThreadsHbm, kRingCtasPerSm)
     k_amax(const __grid_constant__ CUtensorMap tm_x, int64_t total_bytes, int hadamard,
            float* __restrict__ partials, unsigned int* __restrict__ ticket, float* __restrict__ amax_out,
-           int* status) {
+           int* status, const int32_t* gate, int32_t gate_value) {
   extern __shared__ uint8_t ring_raw[];
   __shared__ uint64_t bars[kWarpsPerCta * kRing];
   uint8_t* ring_all = ring_base(ring_raw);
   const uint32_t lane = lane_id();
   pdl_wait();
+  if (gated_off(gate, gate_value)) {
+    pdl_release();
+    return;
+  }
   float m = 0.f;
   stream_blocks<kWarpsPerCta>(&tm_x, total_bytes, hadamard, ring_all, bars, status, [&](float2 (&P)[32], int64_t) {
     float2 mm = make_float2(0.f, 0.f);
@@ -346,12 +350,16 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     k_quant_nvfp4(const __grid_constant__ CUtensorMap tm_x, int64_t M, int32_t K, int hadamard,
                   const float* __restrict__ amax_in, uint8_t* __restrict__ codes,
                   uint8_t* __restrict__ sf_mma, uint8_t* __restrict__ sf_rm,
-                  float* __restrict__ g_out, int* status) {
+                  float* __restrict__ g_out, int* status, const int32_t* gate, int32_t gate_value) {
   extern __shared__ uint8_t ring_raw[];
   __shared__ Nvfp4Tables tab;
   __shared__ uint64_t bars[kQuantWarps * kRing];
   uint8_t* ring_all = ring_base(ring_raw);
   pdl_wait();
+  if (gated_off(gate, gate_value)) {
+    pdl_release();
+    return;
+  }
   const float amax_t = __ldg(amax_in);
   const float g = (amax_t == 0.f) ? 1.f : __fdiv_rn(amax_t, 2688.f);
   if (blockIdx.x == 0 && threadIdx.x == 0 && g_out != nullptr) *g_out = g;
@@ -473,11 +481,15 @@ template <bool F16>
 __global__ void __launch_bounds__(kThreadsHbm)
     k_quant_int8_token(const __grid_constant__ CUtensorMap tm_x, int64_t M, int32_t K, int hadamard,
                        int32_t buf_bytes, int32_t box_rows, int qmax, uint8_t* __restrict__ codes,
-                       float* __restrict__ scales, int* status) {
+                       float* __restrict__ scales, int* status, const int32_t* gate, int32_t gate_value) {
   extern __shared__ uint8_t s_raw[];
   __shared__ uint64_t bars[2 * (kThreadsHbm / 32)];
   uint8_t* s_rows = ring_base(s_raw);
   pdl_wait();
+  if (gated_off(gate, gate_value)) {
+    pdl_release();
+    return;
+  }
   const uint32_t lane = lane_id();
   const int wid = threadIdx.x >> 5;
   const int32_t halves = K >> 6;                 // 64-element half blocks (128-byte rows) per token row
@@ -690,7 +702,7 @@ static int ring_grid(int64_t nchunks) {
 }
 
 ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* amax_out, void* ws,
-                      cudaStream_t st) {
+                      cudaStream_t st, Gate gate) {
   const int64_t units = M * (K / 128);
   if (units == 0) return cudaMemsetAsync(amax_out, 0, sizeof(float), st) == cudaSuccess ? QL_OK : QL_ERR_CUDA;
   const int grid = ring_grid((units * 256 + kChunkBytes - 1) / kChunkBytes);
@@ -700,7 +712,7 @@ ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* 
   if (!make_stream_tmap(&tm, x, units * 256)) return QL_ERR_CUDA;
   if (!set_smem_attr(reinterpret_cast<const void*>(k_amax), kRingBytesPerCta + kRingAlignPad)) return QL_ERR_CUDA;
   if (launch_pdl(k_amax, dim3(grid), dim3(kThreadsHbm), kRingBytesPerCta + kRingAlignPad, st, 1, tm, units * 256,
-                 hadamard, partials, ticket, amax_out, status_word()) != cudaSuccess) {
+                 hadamard, partials, ticket, amax_out, status_word(), gate.route, gate.value) != cudaSuccess) {
     (void)cudaGetLastError();
     return QL_ERR_CUDA;
   }
@@ -708,7 +720,8 @@ ql_status launch_amax(const void* x, int64_t M, int32_t K, int hadamard, float* 
 }
 
 ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, const float* amax_in,
-                             void* codes, void* sf_mma, void* sf_rm, float* g_out, cudaStream_t st, int decomp) {
+                             void* codes, void* sf_mma, void* sf_rm, float* g_out, cudaStream_t st, int decomp,
+                             Gate gate) {
   if (M == 0) return QL_OK;
   const int64_t nchunks = (M * K * 2 + kChunkBytes - 1) / kChunkBytes;
   const int grid = static_cast<int>(std::max<int64_t>(
@@ -719,7 +732,7 @@ ql_status launch_quant_nvfp4(const void* x, int64_t M, int32_t K, int hadamard, 
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), kQuantRingBytes + kRingAlignPad)) return QL_ERR_CUDA;
   if (launch_pdl(kern, dim3(grid), dim3(kQuantThreads), kQuantRingBytes + kRingAlignPad, st, 1, tm, M, K, hadamard,
                  amax_in, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf_mma), static_cast<uint8_t*>(sf_rm),
-                 g_out, status_word()) != cudaSuccess) {
+                 g_out, status_word(), gate.route, gate.value) != cudaSuccess) {
     (void)cudaGetLastError();
     return QL_ERR_CUDA;
   }
@@ -735,7 +748,7 @@ ql_status launch_expand_nvfp4_f16(const void* codes, const void* sf, int32_t N, 
 }
 
 ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadamard, void* codes,
-                                  float* scales, cudaStream_t st, int f16_codes, int qmax) {
+                                  float* scales, cudaStream_t st, int f16_codes, int qmax, Gate gate) {
   if (M == 0) return QL_OK;
   // a token row is K/64 rows of 128 bytes; TMA boxes of at most 256 rows that tile it exactly
   const int32_t halves = K / 64;
@@ -754,7 +767,8 @@ ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadam
   auto kern = f16_codes ? k_quant_int8_token<true> : k_quant_int8_token<false>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), static_cast<int>(smem))) return QL_ERR_CUDA;
   if (launch_pdl(kern, dim3(grid), dim3(32 * warps), smem, st, 1, tm, M, K, hadamard, static_cast<int32_t>(buf),
-                 box_rows, qmax, static_cast<uint8_t*>(codes), scales, status_word()) != cudaSuccess) {
+                 box_rows, qmax, static_cast<uint8_t*>(codes), scales, status_word(), gate.route,
+                 gate.value) != cudaSuccess) {
     (void)cudaGetLastError();
     return QL_ERR_CUDA;
   }

@@ -94,6 +94,8 @@ def _load() -> C.CDLL:
         "qlinear_gemm": (C.c_int, [i32, vp, vp, vp, i64, C.POINTER(Weights), vp, vp]),
         "qlinear_forward_ws_bytes": (sz, [i64, C.POINTER(Weights), i32]),
         "qlinear_forward": (C.c_int, [vp, i64, C.POINTER(Weights), i32, vp, vp, sz, vp]),
+        "qlinear_forward_routed_ws_bytes": (sz, [i64, C.POINTER(Weights)]),
+        "qlinear_forward_routed": (C.c_int, [vp, i64, C.POINTER(Weights), vp, vp, vp, sz, vp]),
         "qlinear_tdc_init": (C.c_int, [vp, vp]),
         "qlinear_tdc_ws_bytes": (sz, [i64]),
         "qlinear_tdc_refresh": (C.c_int, [vp, vp, i64, vp, vp, vp, C.POINTER(TdcParams), vp, sz, vp]),
@@ -288,6 +290,24 @@ def qlinear_forward(X: torch.Tensor, w: PackedWeights, route: int = QL_ROUTE_NVF
     _check("qlinear_forward",
            lib.qlinear_forward(_ptr(X), M, C.byref(w.desc), route, _ptr(Y), _ptr(plan.ws),
                                plan.ws.numel(), _stream(stream)))
+    return Y
+
+
+def qlinear_forward_routed(X: torch.Tensor, w: PackedWeights, route: torch.Tensor, Y: torch.Tensor | None = None,
+                           ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Forward with the route read on the device (int32 [1] tensor, e.g. the
+    router's output or a TDC state's next_route): no host synchronization."""
+    assert X.dtype == torch.bfloat16 and X.is_cuda and X.dim() == 2 and X.is_contiguous()
+    assert route.dtype == torch.int32 and route.is_cuda
+    M, K = X.shape
+    assert K == w.K
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+    if ws is None:
+        ws = _bytes(lib.qlinear_forward_routed_ws_bytes(M, C.byref(w.desc)), X.device)
+    _check("qlinear_forward_routed",
+           lib.qlinear_forward_routed(_ptr(X), M, C.byref(w.desc), _ptr(route), _ptr(Y), _ptr(ws), ws.numel(),
+                                      _stream(stream)))
     return Y
 
 

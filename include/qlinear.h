@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define QLINEAR_ABI_VERSION 5
+#define QLINEAR_ABI_VERSION 6
 
 #if defined(__GNUC__)
 #define QL_API __attribute__((visibility("default")))
@@ -295,6 +295,22 @@ QL_API size_t qlinear_forward_ws_bytes(int64_t M, const ql_weights* w, int32_t r
 QL_API ql_status qlinear_forward(const void* X_bf16, int64_t M, const ql_weights* w,
                           int32_t route, void* Y_bf16,
                           void* ws, size_t ws_bytes, void* stream);
+
+/* ---- forward with the route in device memory ----------------------------
+   DMPQ routes a block from the previous step's Gamma, which the router (or
+   a TDC state's next_route) leaves in device memory.  This forward enqueues
+   the kernels of every route the weights support -- NVFP4, INT8 (f16-coded
+   with an f16 weight copy) and, with keep_bf16, BF16 -- and each kernel
+   waits for its predecessor, reads *route_dev and returns at once unless
+   the route is its own.  So the call never synchronizes with the host and
+   a whole step can be captured in one CUDA graph.  Weights: QL_W_NVFP4.
+   route_dev: device int32, 4-byte aligned, written earlier in the same
+   stream; a value no enqueued route has leaves Y unwritten.  ws:
+   qlinear_forward_routed_ws_bytes bytes, 256-byte aligned. */
+QL_API size_t qlinear_forward_routed_ws_bytes(int64_t M, const ql_weights* w);
+QL_API ql_status qlinear_forward_routed(const void* X_bf16, int64_t M, const ql_weights* w,
+                                        const int32_t* route_dev, void* Y_bf16, void* ws,
+                                        size_t ws_bytes, void* stream);
 
 /* ---- temporal delta cache ------------------------------------------------
    "6Bit-Diffusion", Methodology A.2 / B.2 (TDC) and B.3 (PDR).  A block's
