@@ -5,14 +5,19 @@
 //  * tensor amax pre-pass for the dynamic NVFP4 tensor scale;
 //  * NVFP4 quantizer (E2M1 codes, E4M3 scale per 16 elements, fp32 tensor
 //    scale), writing the block scales straight into the MMA atom layout;
-//  * per-token INT8 quantizer (the route DMPQ takes for sensitive blocks);
-//  * per-tensor INT8 quantizer with Q-ARVD's channel permutation
+//  * the NVFP4 activation decomposition (SemanticDialect, Methodology 2.2):
+//    NVFP4 of h and of its residual in one pass;
+//  * per-token INT8 quantizer (the route DMPQ takes for sensitive blocks),
+//    also with 6-bit codes (W4A6);
+//  * per-tensor INT8 / INT6 quantizer with Q-ARVD's channel permutation
 //    (Q-ARVD, Technical details: per-tensor activation quantization).
 //
-// Work decomposition shared by all of them: a 128-element Hadamard block is
-// held by 4 consecutive lanes, 32 contiguous elements each (four 16-byte
-// loads).  Butterfly distances 1..16 stay inside a lane, 32 and 64 are one
-// shuffle each.  A warp covers 8 blocks = 1024 contiguous elements.
+// Work decomposition of the rotated kernels: a 128-element Hadamard block is
+// held by 2 lanes, 64 contiguous elements (one 128-byte row) each, in pair
+// registers (x_j, x_{j+32}).  Butterfly distances 1..16 are packed f32x2
+// operations inside a lane, 32 is inside each pair, 64 is one shuffle
+// between the two lanes.  A warp covers 16 blocks = 2048 contiguous
+// elements per chunk.
 #include "ql_common.cuh"
 #include "gemm_common.cuh"
 #include "launchers.h"
