@@ -7,9 +7,13 @@
 // zero padding to 32, outlier channels, zero padding to 32), so each class
 // is a contiguous, MMA-aligned K range and gets its own int32 accumulator:
 //   Y[m, n] = bf16(s_x * (s_norm[n] * acc_normal[m, n] + s_out[n] * acc_outlier[m, n])).
-// The MMA is tcgen05 kind::i8 (128 x 128 x 32, int32 accumulation, exact).
+// The MMA is tcgen05 kind::i8 (int32 accumulation, exact).  Two kernels:
+//   k_gemm_qarvd_pre  weights kept as int8 (expand_i8): CTA pairs, both
+//                     operands by TMA (described further down);
+//   k_gemm_qarvd      INT4 weights widened on chip, below.
+// Activations may carry INT8 or INT6 codes (W4A6); the product is the same.
 //
-// Persistent, warp-specialized, one CTA (512 threads) per SM:
+// k_gemm_qarvd: persistent, warp-specialized, one CTA (512 threads) per SM:
 //   warps 0-7   transform: INT4 nibbles -> sign-extended int8 in the
 //               128-byte-swizzled K-major layout;
 //   warp 8      TMA producer: int8 activations straight into the MMA layout

@@ -3,10 +3,17 @@
 // activations while all weights stay NVFP4).
 //
 // Y[m, n] = bf16(s_m * g_w * alpha_mul * sum_k q[m,k] * (e2m1[n,k] * sb[n,k/16]))
-// with fp32 accumulation in tensor memory.  Both operands are expanded on
-// chip to f16, where every value is exact: int8 codes (|q| <= 127) and every
-// E2M1 x E4M3 product (at most 6 significant bits, magnitudes 2^-10 .. 2688).
-// The MMA is tcgen05 kind::f16 (128 x BN x 16).
+// with fp32 accumulation in tensor memory.  Both operands are f16, where
+// every value is exact: int8 codes (|q| <= 127) and every E2M1 x E4M3
+// product (at most 6 significant bits, magnitudes 2^-10 .. 2688).  The MMA
+// is tcgen05 kind::f16 (128 x BN x 16).  Three forms (template flags):
+//   PRE + A16  f16 weight copy (expand_f16) and f16-coded activations, both
+//              by TMA straight into the MMA layout, no transform warps (the
+//              form qlinear_forward takes when the copy exists);
+//   PRE        f16 weight copy by TMA, int8 activations widened on chip;
+//   neither    both operands widened on chip (below).
+// BF16 instantiates the PRE + A16 form with bf16 operand types and no scales:
+// the unquantized product X W^T of PDR's high-precision refresh.
 //
 // Persistent, warp-specialized, one CTA (512 threads) per SM:
 //   warps 0-7   transform: raw int8 / FP4 + scale tiles -> f16 tiles in the
