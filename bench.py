@@ -48,9 +48,9 @@ NVFP4_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # bf16 in, E2M1 out, E4M3 per 16
 # DRAM bytes per launch of the W4A4 GEMM from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of the GEMM sources).
 GEMM_TRAFFIC = {
-    # ncu dram__bytes_read.sum + dram__bytes_write.sum: 590.8 MB over the 4
+    # ncu dram__bytes_read.sum + dram__bytes_write.sum: 591.0 MB over the 4
     # GEMM launches of one step of this workload
-    "b683ace5ad6f035b": 590.8e6 / 4,
+    "9530880a77d1f62c": 591.0e6 / 4,
 }
 
 
