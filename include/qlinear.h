@@ -237,8 +237,9 @@ QL_API ql_status qlinear_route_noalloc(const void* in_bf16, const void* out_bf16
 /* ---- tensor amax ------------------------------------------------------------
    *amax_out (device fp32) = max |H x| over the whole [M, K] tensor (|x| when
    hadamard is 0): the input of the dynamic NVFP4 tensor scale
-   g = amax / (6 * 448) and of the per-tensor INT8 scale amax / 127.  One
-   launch; ws needs qlinear_quantize_ws_bytes(M, K, QL_ROUTE_NVFP4) bytes. */
+   g = amax / (6 * 448) and of the per-tensor INT8 / INT6 scale amax / 127
+   (amax / 31).  One launch; ws needs qlinear_quantize_ws_bytes(M, K,
+   QL_ROUTE_NVFP4) bytes. */
 QL_API ql_status qlinear_tensor_amax(const void* X_bf16, int64_t M, int32_t K, int32_t hadamard,
                                      float* amax_out, void* ws, size_t ws_bytes, void* stream);
 
@@ -251,6 +252,11 @@ QL_API ql_status qlinear_tensor_amax(const void* X_bf16, int64_t M, int32_t K, i
    QL_ACT_INT8_TENSOR: needs Q-ARVD weights `w`; codes int8 [M, w->Kp] in the
                        weights' channel order with zero padding; scales =
                        fp32[1]; hadamard must be 0.
+   QL_ACT_NVFP4_DECOMP: codes uint8 [M, K] = [q1 | q2] per row; sf_mma over
+                       2K (q1's scales first, required); sf_rowmajor [M, K/8]
+                       (optional); scales = fp32[1] tensor scale g_x.
+   QL_ROUTE_INT6, QL_ACT_INT6_F16, QL_ACT_INT6_TENSOR: as the INT8 formats,
+                       codes in [-31, 31], scales amax / 31.
    `hadamard` = 1 rotates each 128-block of K first (NVFP4 / INT8 routes).
    amax_in: optional device fp32 tensor amax (NVFP4 and per-tensor INT8),
    e.g. from qlinear_tensor_amax or a calibrated static value; NULL makes the
