@@ -92,6 +92,19 @@ def test_nvfp4_subnormal_block_scale():
     assert dq[0, 16] == x[0, 16] and dq[0, 17] == x[0, 17]
 
 
+def test_nvfp4_tensor_scale_takes_the_largest_magnitude():
+    """The tensor scale follows the largest MAGNITUDE, here a negative
+    value: g = 5376 / (6 * 448) = 2 exactly, its block scale is 448 and the
+    element itself is the code for -6."""
+    x = np.zeros((1, 32), np.float32)
+    x[0, 3] = -5376.0
+    x[0, 20] = 1.0
+    packed, sb, g = O.nvfp4_quantize(x)
+    assert g == np.float32(2.0)
+    assert sb[0, 0] == 0x7E
+    assert O.unpack_nibbles(packed)[0, 3] == 0xF
+
+
 def test_nvfp4_static_scale_saturates():
     x = np.full((1, 16), 100.0, np.float32)
     packed, sb, g = O.nvfp4_quantize(x, g=np.float32(0.01))
@@ -197,6 +210,14 @@ def test_median_matches_numpy_and_selection():
         assert O.median_sorted(v) == pytest.approx(float(np.median(v)), abs=0, rel=1e-15)
         if n % 2:
             assert O.median_sorted(v) == np.partition(v, n // 2)[n // 2]
+
+
+def test_qarvd_channel_norms_closed_form():
+    """v_k is the L2 norm of input channel k (a column of W [N, K]):
+    columns (3, 4), (1, 0), (0, 2) give 5, 1, 2."""
+    w = np.array([[3.0, 1.0, 0.0], [4.0, 0.0, 2.0]], np.float32)
+    bits = (w.view(np.uint32) >> 16).astype(np.uint16)        # exact in bf16
+    assert O.qarvd_channel_norms(bits).tolist() == [5.0, 1.0, 2.0]
 
 
 def test_qarvd_layout_and_int4():

@@ -85,17 +85,22 @@ def test_w4a4_gemm_equals_exact_rational_sum():
     assert np.array_equal(got, want)
 
 
-def test_w4a8_token_gemm_brute_force():
+@pytest.mark.parametrize("hadamard", [True, False])
+def test_w4a8_token_gemm_brute_force(hadamard):
+    """With rotated operands the product carries the 1/128 of H H^T = 128 I;
+    without rotation it does not."""
     rng = np.random.default_rng(3)
-    h = O.block_hadamard((rng.standard_normal((2, 128)) * 2).astype(np.float32))
+    rot = O.block_hadamard if hadamard else (lambda v: v)
+    h = rot((rng.standard_normal((2, 128)) * 2).astype(np.float32))
     q, s = O.int8_per_token(h)
-    wp, wsb, gw = O.nvfp4_quantize(O.block_hadamard(rng.standard_normal((3, 128)).astype(np.float32)))
-    got = O.gemm_w4a8_token(q, s, wp, wsb, gw, hadamard=True)
+    wp, wsb, gw = O.nvfp4_quantize(rot(rng.standard_normal((3, 128)).astype(np.float32)))
+    got = O.gemm_w4a8_token(q, s, wp, wsb, gw, hadamard=hadamard)
     dq = O.nvfp4_dequantize(wp, wsb)
+    c = 128 if hadamard else 1
     for i in range(2):
         for j in range(3):
             acc = sum(Fraction(int(q[i, t])) * Fraction(float(dq[j, t])) for t in range(128))
-            want = acc * Fraction(float(s[i])) * Fraction(float(gw)) / 128
+            want = acc * Fraction(float(s[i])) * Fraction(float(gw)) / c
             assert got[i, j] == pytest.approx(float(want), rel=1e-15)
 
 

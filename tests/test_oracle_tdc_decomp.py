@@ -185,6 +185,26 @@ def test_policy_traces(acc_max, max_skips, pattern):
     assert "".join(seq) == "".join(want)
 
 
+@pytest.mark.parametrize("eps_threshold,pattern", [
+    # deltas alternate 0.5, 0.625: E is 0.25 after the second computation and
+    # 0.2 after the third (0.125 / 0.625); both are at or above 0.1
+    (0.1, "CCCCCCC"),
+    # E = 0.25 is not below 0.25 (strict), E = 0.2 is: three skips, then the
+    # skip count forces a computation
+    (0.25, "CCCSSSC"),
+])
+def test_error_threshold_gates_skips(eps_threshold, pattern):
+    prm = T.TdcParams(gamma_threshold=0.05, eps_threshold=eps_threshold, acc_max=1.0, max_skips=3)
+    st = T.TdcState()
+    block, _ = _block_with_deltas([0.5, 0.625] * 4)
+    inp = _bf16(np.ones(64, np.float32))
+    got = ""
+    for _ in range(len(pattern)):
+        _, skipped, _ = T.tdc_step(st, prm, inp, block)
+        got += "S" if skipped else "C"
+    assert got == pattern
+
+
 def test_first_two_steps_always_compute():
     st = T.TdcState()
     prm = T.TdcParams()
