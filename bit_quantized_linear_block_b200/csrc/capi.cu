@@ -415,7 +415,7 @@ ql_status qlinear_route(const void* in, const void* out, int64_t numel, float th
 namespace {
 bool tdc_params_ok(const ql_tdc_params* p) {
   return p != nullptr && p->gamma_threshold == p->gamma_threshold && p->eps_threshold == p->eps_threshold &&
-         p->acc_max == p->acc_max && p->max_skips >= 0;
+         p->acc_max == p->acc_max && p->kappa == p->kappa && p->rho_max == p->rho_max && p->max_skips >= 0;
 }
 }  // namespace
 

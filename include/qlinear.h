@@ -365,6 +365,8 @@ typedef struct {
                             the rest (8)                                       */
   float rho_max;         /* BF16 when rho exceeds this (>= 1: never)           */
 } ql_tdc_params;
+/* A NaN in any float field of ql_tdc_params, or max_skips < 0, makes the
+   TDC calls return QL_ERR_INVALID_ARG before any CUDA call. */
 
 /* Reset a block's cache state (device pointer, 8-byte aligned): no deltas,
    Gamma = E = +inf, next step computed on the INT8 route. */

@@ -134,8 +134,11 @@ def test_new_entry_points_validate_on_the_host(ql):
     assert L.qlinear_tdc_refresh(FAKE, FAKE, 100, FAKE, FAKE, None, C.byref(prm), FAKE, 1 << 20, None) == 1
     assert L.qlinear_tdc_refresh(FAKE, FAKE, 100, FAKE, FAKE + 8, FAKE, C.byref(prm), FAKE, 1 << 20, None) == 3
     assert L.qlinear_tdc_refresh(FAKE, FAKE, 100, FAKE, FAKE, FAKE, C.byref(prm), FAKE, 16, None) == 6
-    nan = ql.TdcParams(0.05, float("nan"), 0.3, 3, 8.0, 1.0)
-    assert L.qlinear_tdc_refresh(FAKE, FAKE, 100, FAKE, FAKE, FAKE, C.byref(nan), FAKE, 1 << 20, None) == 1
+    for fields in [(0.05, float("nan"), 0.3, 3, 8.0, 1.0), (0.05, 0.1, 0.3, 3, float("nan"), 1.0),
+                   (0.05, 0.1, 0.3, 3, 8.0, float("nan"))]:
+        nan = ql.TdcParams(*fields)
+        assert L.qlinear_tdc_refresh(FAKE, FAKE, 100, FAKE, FAKE, FAKE, C.byref(nan), FAKE, 1 << 20, None) == 1
+        assert L.qlinear_tdc_skip(FAKE, 100, FAKE, FAKE, FAKE, C.byref(nan), FAKE, None) == 1
     neg = ql.TdcParams(0.05, 0.1, 0.3, -1, 8.0, 1.0)
     assert L.qlinear_tdc_skip(FAKE, 100, FAKE, FAKE, FAKE, C.byref(neg), FAKE, None) == 1
     assert L.qlinear_tdc_skip(FAKE, 100, FAKE, FAKE, FAKE, None, FAKE, None) == 1
