@@ -411,6 +411,26 @@ ql_status qlinear_route(const void* in, const void* out, int64_t numel, float th
                             static_cast<cudaStream_t>(stream));
 }
 
+ql_status qlinear_gamma_sums(const void* in, const void* out, int64_t numel, double* sums_dev, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (numel < 0 || sums_dev == nullptr || ws == nullptr) return QL_ERR_INVALID_ARG;
+  if (numel > 0 && (in == nullptr || out == nullptr)) return QL_ERR_INVALID_ARG;
+  if (!aligned(in, 16) || !aligned(out, 16) || !aligned(ws, 256) || !aligned(sums_dev, 8))
+    return QL_ERR_ALIGNMENT;
+  if (ws_bytes < qlinear_route_ws_bytes(numel)) return QL_ERR_WORKSPACE;
+  QL_TRY(device_ready());
+  return launch_gamma_sums(in, out, numel, sums_dev, ws, static_cast<cudaStream_t>(stream));
+}
+
+ql_status qlinear_route_from_sums(const double* sums_dev, float threshold, double* gamma_dev, int32_t* route_dev,
+                                  void* stream) {
+  if (sums_dev == nullptr || gamma_dev == nullptr || route_dev == nullptr) return QL_ERR_INVALID_ARG;
+  if (!(threshold == threshold)) return QL_ERR_INVALID_ARG;
+  if (!aligned(sums_dev, 8) || !aligned(gamma_dev, 8) || !aligned(route_dev, 4)) return QL_ERR_ALIGNMENT;
+  QL_TRY(device_ready());
+  return launch_route_from_sums(sums_dev, threshold, gamma_dev, route_dev, static_cast<cudaStream_t>(stream));
+}
+
 // ---------------------------------------------------------------- temporal delta cache
 namespace {
 bool tdc_params_ok(const ql_tdc_params* p) {

@@ -52,6 +52,11 @@ ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int
                                         float* scale_out, cudaStream_t st, int qmax = 127);
 ql_status launch_gamma_route(const void* in, const void* out, int64_t numel, float threshold,
                              double* gamma, int32_t* route, void* ws, cudaStream_t st);
+// sums[0] = sum |out - in|, sums[1] = sum |in| (fp64); ws as for launch_gamma_route.
+ql_status launch_gamma_sums(const void* in, const void* out, int64_t numel, double* sums, void* ws,
+                            cudaStream_t st);
+ql_status launch_route_from_sums(const double* sums, float threshold, double* gamma, int32_t* route,
+                                 cudaStream_t st);
 ql_status launch_qarvd_prepare(const void* W, int32_t N, int32_t K, float tau, float alpha,
                                const ql_weights* w, void* ws, cudaStream_t st);
 

@@ -1,5 +1,6 @@
-// Device pieces of the DMPQ router shared by qlinear_route and
-// qlinear_route_noalloc (6Bit-Diffusion, Methodology A.1 / B.1):
+// Device pieces of the DMPQ router shared by qlinear_route,
+// qlinear_route_noalloc and the token-split form (qlinear_gamma_sums,
+// qlinear_route_from_sums) (6Bit-Diffusion, Methodology A.1 / B.1):
 // Gamma = sum |out - in| / sum |in| with fp32 differences and fp64 sums.
 #pragma once
 
@@ -90,11 +91,9 @@ __device__ __forceinline__ void gamma_block_sums(double& s1, double& s0) {
 }
 
 // Per-CTA partials, then the last CTA to finish (atomic ticket) adds all
-// partials with the whole block and writes Gamma and the route:
-// route = 1 (INT8) if Gamma > threshold, Gamma = +inf when sum |in| is 0.
-// The ticket is reset for the next call.
-__device__ __forceinline__ void gamma_finish(double s1, double s0, double* partials, unsigned int* ticket,
-                                             float threshold, double* gamma_out, int32_t* route_out) {
+// partials with the whole block.  Returns true in thread 0 of that CTA only,
+// with the totals in (s1, s0); the ticket is reset for the next call.
+__device__ __forceinline__ bool gamma_total(double& s1, double& s0, double* partials, unsigned int* ticket) {
   __shared__ bool s_last;
   gamma_block_sums(s1, s0);
   if (threadIdx.x == 0) {
@@ -104,7 +103,7 @@ __device__ __forceinline__ void gamma_finish(double s1, double s0, double* parti
     s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
   }
   __syncthreads();
-  if (!s_last) return;
+  if (!s_last) return false;
   __threadfence();
   double a = 0.0, b = 0.0;
   const volatile double* p = partials;
@@ -113,12 +112,24 @@ __device__ __forceinline__ void gamma_finish(double s1, double s0, double* parti
     b += p[2 * i + 1];
   }
   gamma_block_sums(a, b);
-  if (threadIdx.x == 0) {
-    const double gamma = (b == 0.0) ? __longlong_as_double(0x7ff0000000000000ll) : a / b;
-    *gamma_out = gamma;
-    *route_out = (gamma > static_cast<double>(threshold)) ? 1 : 0;
-    *ticket = 0u;
-  }
+  if (threadIdx.x != 0) return false;
+  s1 = a;
+  s0 = b;
+  *ticket = 0u;
+  return true;
+}
+
+// Gamma = s1 / s0 (+inf when s0 is 0); route = 1 (INT8) if Gamma > threshold.
+__device__ __forceinline__ void gamma_decide(double s1, double s0, float threshold, double* gamma_out,
+                                             int32_t* route_out) {
+  const double gamma = (s0 == 0.0) ? __longlong_as_double(0x7ff0000000000000ll) : s1 / s0;
+  *gamma_out = gamma;
+  *route_out = (gamma > static_cast<double>(threshold)) ? 1 : 0;
+}
+
+__device__ __forceinline__ void gamma_finish(double s1, double s0, double* partials, unsigned int* ticket,
+                                             float threshold, double* gamma_out, int32_t* route_out) {
+  if (gamma_total(s1, s0, partials, ticket)) gamma_decide(s1, s0, threshold, gamma_out, route_out);
 }
 
 }  // namespace ql

@@ -5,7 +5,9 @@
 // the threshold, NVFP4 otherwise.  One launch: grid-stride 16-byte loads of
 // both tensors, fp32 differences, fp64 per-thread sums, per-CTA partials,
 // and the last CTA to finish (atomic ticket) adds the partials and writes
-// Gamma and the route.
+// Gamma and the route.  With the block's tokens split across ranks, each
+// rank writes its two sums instead (k_gamma_sums), the ranks add them, and
+// a one-thread kernel (k_route_from_sums) makes the same decision.
 //
 // Q-ARVD (Methodology / Formula and operation flow): input-channel L2 norms
 // of W, median and MAD, modified z-score M_k = (v_k - median)/MAD, outlier
@@ -32,6 +34,27 @@ __global__ void __launch_bounds__(kThreadsHbm)
   gamma_thread_sums(in, out, numel, s1, s0);
   pdl_release();
   gamma_finish(s1, s0, partials, ticket, threshold, gamma_out, route_out);
+}
+
+// Token-split form: this rank's two sums only (sums_out[0] = sum |out - in|,
+// sums_out[1] = sum |in|); the ranks add them and k_route_from_sums decides.
+__global__ void __launch_bounds__(kThreadsHbm)
+    k_gamma_sums(const uint4* __restrict__ in, const uint4* __restrict__ out, int64_t numel,
+                 double* __restrict__ partials, unsigned int* __restrict__ ticket, double* __restrict__ sums_out) {
+  pdl_wait();
+  double s1, s0;
+  gamma_thread_sums(in, out, numel, s1, s0);
+  pdl_release();
+  if (gamma_total(s1, s0, partials, ticket)) {
+    sums_out[0] = s1;
+    sums_out[1] = s0;
+  }
+}
+
+__global__ void k_route_from_sums(const double* __restrict__ sums, float threshold, double* __restrict__ gamma_out,
+                                  int32_t* __restrict__ route_out) {
+  pdl_wait();
+  if (threadIdx.x == 0) gamma_decide(sums[0], sums[1], threshold, gamma_out, route_out);
 }
 
 // ---------------------------------------------------------------------------
@@ -224,6 +247,28 @@ ql_status launch_gamma_route(const void* in, const void* out, int64_t numel, flo
   unsigned int* ticket = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + kRoutePartialBytes);
   if (launch_pdl(k_gamma_route, dim3(grid), dim3(kThreadsHbm), 0, st, 1, static_cast<const uint4*>(in),
                  static_cast<const uint4*>(out), numel, partials, ticket, threshold, gamma, route) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
+}
+
+ql_status launch_gamma_sums(const void* in, const void* out, int64_t numel, double* sums, void* ws,
+                            cudaStream_t st) {
+  const int grid = hbm_grid(std::max<int64_t>(1, (numel / 8 + kThreadsHbm - 1) / kThreadsHbm), 1);
+  double* partials = static_cast<double*>(ws);
+  unsigned int* ticket = reinterpret_cast<unsigned int*>(static_cast<uint8_t*>(ws) + kRoutePartialBytes);
+  if (launch_pdl(k_gamma_sums, dim3(grid), dim3(kThreadsHbm), 0, st, 1, static_cast<const uint4*>(in),
+                 static_cast<const uint4*>(out), numel, partials, ticket, sums) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
+}
+
+ql_status launch_route_from_sums(const double* sums, float threshold, double* gamma, int32_t* route,
+                                 cudaStream_t st) {
+  if (launch_pdl(k_route_from_sums, dim3(1), dim3(32), 0, st, 1, sums, threshold, gamma, route) != cudaSuccess) {
     (void)cudaGetLastError();
     return QL_ERR_CUDA;
   }

@@ -87,6 +87,8 @@ def _load() -> C.CDLL:
                                               C.POINTER(Weights), vp, sz, vp]),
         "qlinear_route_ws_bytes": (sz, [i64]),
         "qlinear_route": (C.c_int, [vp, vp, i64, f32, vp, vp, vp, sz, vp]),
+        "qlinear_gamma_sums": (C.c_int, [vp, vp, i64, vp, vp, sz, vp]),
+        "qlinear_route_from_sums": (C.c_int, [vp, f32, vp, vp, vp]),
         "qlinear_quantize_ws_bytes": (sz, [i64, i32, i32]),
         "qlinear_tensor_amax": (C.c_int, [vp, i64, i32, i32, vp, vp, sz, vp]),
         "qlinear_quantize_act": (C.c_int, [vp, i64, i32, i32, i32, C.POINTER(Weights), vp, vp, vp,
@@ -196,6 +198,36 @@ def qlinear_route(inp: torch.Tensor, out: torch.Tensor, threshold: float = 0.05,
         ws = _bytes(lib.qlinear_route_ws_bytes(n), inp.device)
     _check("qlinear_route", lib.qlinear_route(_ptr(inp), _ptr(out), n, threshold, _ptr(gamma),
                                               _ptr(route), _ptr(ws), ws.numel(), _stream(stream)))
+    return gamma, route
+
+
+def qlinear_gamma_sums(inp: torch.Tensor, out: torch.Tensor, sums: torch.Tensor | None = None,
+                       ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Device float64 [2]: (sum |out - in|, sum |in|) over these elements,
+    this rank's share of Gamma when a block's tokens are split across ranks."""
+    assert inp.dtype == torch.bfloat16 and out.dtype == torch.bfloat16
+    assert inp.shape == out.shape and inp.is_contiguous() and out.is_contiguous()
+    n = inp.numel()
+    if sums is None:
+        sums = torch.empty(2, dtype=torch.float64, device=inp.device)
+    if ws is None:
+        ws = _bytes(lib.qlinear_route_ws_bytes(n), inp.device)
+    _check("qlinear_gamma_sums", lib.qlinear_gamma_sums(_ptr(inp), _ptr(out), n, _ptr(sums), _ptr(ws),
+                                                        ws.numel(), _stream(stream)))
+    return sums
+
+
+def qlinear_route_from_sums(sums: torch.Tensor, threshold: float = 0.05, gamma: torch.Tensor | None = None,
+                            route: torch.Tensor | None = None, stream=None):
+    """Device tensors (gamma float64 [1], route int32 [1]) from the summed
+    (sum |out - in|, sum |in|) of all ranks."""
+    assert sums.dtype == torch.float64 and sums.is_cuda and sums.numel() == 2 and sums.is_contiguous()
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float64, device=sums.device)
+    if route is None:
+        route = torch.empty(1, dtype=torch.int32, device=sums.device)
+    _check("qlinear_route_from_sums", lib.qlinear_route_from_sums(_ptr(sums), threshold, _ptr(gamma), _ptr(route),
+                                                                  _stream(stream)))
     return gamma, route
 
 

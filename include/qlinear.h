@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define QLINEAR_ABI_VERSION 6
+#define QLINEAR_ABI_VERSION 7
 
 #if defined(__GNUC__)
 #define QL_API __attribute__((visibility("default")))
@@ -212,6 +212,23 @@ QL_API size_t qlinear_route_ws_bytes(int64_t numel);
 QL_API ql_status qlinear_route(const void* in_bf16, const void* out_bf16, int64_t numel,
                         float threshold, double* gamma_dev, int32_t* route_dev,
                         void* ws, size_t ws_bytes, void* stream);
+
+/* ---- router with the block's tokens split across ranks -----------------------
+   The same Gamma when each rank holds some rows of the block: each rank
+   calls qlinear_gamma_sums on its own rows, the ranks add the two sums
+   (one all-reduce of 2 doubles), and each calls qlinear_route_from_sums.
+   Only the order of the fp64 additions differs from qlinear_route on the
+   whole block.
+   qlinear_gamma_sums: sums_dev[0] = sum|out - in|, sums_dev[1] = sum|in|
+   over this rank's numel elements (fp64, device, 8-byte aligned).  ws as
+   for qlinear_route (qlinear_route_ws_bytes(numel) bytes, 256-byte aligned,
+   zero-filled before its first use; calls sharing one must not overlap).
+   qlinear_route_from_sums: *gamma_dev = sums_dev[0] / sums_dev[1] (+inf
+   when sums_dev[1] is 0), *route_dev = 1 (INT8) if Gamma > threshold. */
+QL_API ql_status qlinear_gamma_sums(const void* in_bf16, const void* out_bf16, int64_t numel,
+                                    double* sums_dev, void* ws, size_t ws_bytes, void* stream);
+QL_API ql_status qlinear_route_from_sums(const double* sums_dev, float threshold, double* gamma_dev,
+                                         int32_t* route_dev, void* stream);
 
 /* ---- router without a workspace (no counterpart on the pages) --------------
    Same Gamma and route as qlinear_route, for callers that cannot allocate

@@ -96,6 +96,15 @@ def test_other_entry_points_reject_bad_arguments(ql):
     assert L.qlinear_route(FAKE + 4, FAKE, 100, 0.05, FAKE, FAKE, FAKE, 1 << 20, None) == 3
     assert L.qlinear_route(FAKE, FAKE, 100, 0.05, FAKE, FAKE, FAKE, 8, None) == 6
     assert L.qlinear_route(FAKE, FAKE, 100, float("nan"), FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    # token-split router
+    assert L.qlinear_gamma_sums(FAKE, FAKE, 100, None, FAKE, 1 << 20, None) == 1
+    assert L.qlinear_gamma_sums(FAKE, FAKE, -1, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.qlinear_gamma_sums(FAKE, FAKE + 8, 100, FAKE, FAKE, 1 << 20, None) == 3
+    assert L.qlinear_gamma_sums(FAKE, FAKE, 100, FAKE + 4, FAKE, 1 << 20, None) == 3
+    assert L.qlinear_gamma_sums(FAKE, FAKE, 100, FAKE, FAKE, 8, None) == 6
+    assert L.qlinear_route_from_sums(None, 0.05, FAKE, FAKE, None) == 1
+    assert L.qlinear_route_from_sums(FAKE, float("nan"), FAKE, FAKE, None) == 1
+    assert L.qlinear_route_from_sums(FAKE, 0.05, FAKE + 4, FAKE, None) == 3
     na = L.qlinear_route_noalloc
     na.restype = C.c_int
     na.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_float, C.c_void_p, C.c_void_p, C.c_void_p]
