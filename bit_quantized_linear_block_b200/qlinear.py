@@ -122,9 +122,61 @@ def _ptr(t: torch.Tensor | None):
     return None if t is None else C.c_void_p(t.data_ptr())
 
 
-def _stream(stream=None):
-    s = torch.cuda.current_stream() if stream is None else stream
-    return C.c_void_p(s.cuda_stream)
+def _stream(stream, device):
+    """The stream handle to launch on: the given one (which must belong to
+    `device`) or the current stream of `device`."""
+    if stream is None:
+        return C.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    if stream.device != device:
+        raise ValueError(f"stream is on {stream.device}, the call runs on {device}")
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _tensor(t, name: str, dtype=None, device=None, min_bytes: int | None = None, dim: int | None = None):
+    """Checks one tensor argument before anything reaches CUDA: a contiguous
+    CUDA tensor, of `dtype` and on `device` when given, holding at least
+    `min_bytes` bytes.  Raises TypeError or ValueError."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor, got one on {t.device}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call runs on {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dimensions, got {t.dim()}")
+    if min_bytes is not None and t.numel() * t.element_size() < min_bytes:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, the call needs {min_bytes}")
+    return t
+
+
+def _weights(w) -> "PackedWeights":
+    if not isinstance(w, PackedWeights):
+        raise TypeError(f"w must be PackedWeights (from qlinear_prepare_weights), got {type(w).__name__}")
+    return w
+
+
+def _act_bytes(M: int, K: int, act_fmt: int, w=None) -> dict:
+    """Bytes of each buffer of quantized activations [M, K] in `act_fmt`
+    (K: the layer's input width; the Q-ARVD formats need their weights for
+    the padded width Kp).  None: the format has no such buffer."""
+    if act_fmt in (QL_ROUTE_NVFP4, QL_ACT_NVFP4_DECOMP):
+        kq = 2 * K if act_fmt == QL_ACT_NVFP4_DECOMP else K      # decomposed: [q1 | q2] per row
+        return dict(codes=M * kq // 2, sf_mma=lib.qlinear_sf_bytes(M, kq), sf_rowmajor=M * kq // 16, scales=4)
+    if act_fmt in (QL_ROUTE_INT8, QL_ROUTE_INT6):
+        return dict(codes=M * K, sf_mma=None, sf_rowmajor=None, scales=4 * max(M, 1))
+    if act_fmt in (QL_ACT_INT8_F16, QL_ACT_INT6_F16):
+        return dict(codes=2 * M * K, sf_mma=None, sf_rowmajor=None, scales=4 * max(M, 1))
+    if act_fmt in (QL_ACT_INT8_TENSOR, QL_ACT_INT6_TENSOR):
+        if w is None or w.fmt != QL_W_QARVD_INT4:
+            raise ValueError("the per-tensor Q-ARVD formats need the Q-ARVD weights (w)")
+        return dict(codes=M * w.desc.Kp, sf_mma=None, sf_rowmajor=None, scales=4)
+    if act_fmt == QL_ROUTE_BF16:            # the unquantized bf16 input itself
+        return dict(codes=2 * M * K, sf_mma=None, sf_rowmajor=None, scales=None)
+    raise ValueError(f"unknown activation format {act_fmt}")
 
 
 def _bytes(n: int, device) -> torch.Tensor:
@@ -162,7 +214,8 @@ def qlinear_prepare_weights(W: torch.Tensor, fmt: int = QL_W_NVFP4, hadamard: bo
     weights for the INT8 route's GEMM; expand_i8 (Q-ARVD only) keeps the
     INT4 codes sign-extended to int8 for the Q-ARVD GEMM; keep_bf16 (NVFP4
     only) keeps the bf16 weights for the unquantized QL_ROUTE_BF16 product."""
-    assert W.dtype == torch.bfloat16 and W.is_cuda and W.dim() == 2 and W.is_contiguous()
+    _tensor(W, "W", torch.bfloat16, dim=2)
+    dev = W.device
     N, K = W.shape
     cfg = WeightCfg(fmt, int(bool(hadamard)) if fmt in (QL_W_NVFP4, QL_W_NVFP4_DECOMP) else 0, tau, alpha,
                     int(bool(expand_f16)), int(bool(expand_i8)), int(bool(keep_bf16)), 0)
@@ -170,15 +223,25 @@ def qlinear_prepare_weights(W: torch.Tensor, fmt: int = QL_W_NVFP4, hadamard: bo
     wsbytes = lib.qlinear_prepare_ws_bytes(N, K, C.byref(cfg))
     if wbytes == 0:
         raise QLinearError("qlinear_weights_bytes", 2)
-    buf = _bytes(wbytes, W.device)
-    ws = _bytes(wsbytes, W.device)
-    desc = Weights()
-    _check("qlinear_prepare_weights",
-           lib.qlinear_prepare_weights(_ptr(W), N, K, C.byref(cfg), _ptr(buf), buf.numel(),
-                                       C.byref(desc), _ptr(ws), ws.numel(), _stream(stream)))
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        buf = _bytes(wbytes, dev)
+        ws = _bytes(wsbytes, dev)
+        desc = Weights()
+        _check("qlinear_prepare_weights",
+               lib.qlinear_prepare_weights(_ptr(W), N, K, C.byref(cfg), _ptr(buf), buf.numel(),
+                                           C.byref(desc), _ptr(ws), ws.numel(), st))
     pw = PackedWeights(desc, buf, N, K, fmt)
     pw._ws = ws      # keep the scratch alive until the stream has used it
     return pw
+
+
+def _block_pair(inp, out):
+    _tensor(inp, "inp", torch.bfloat16)
+    _tensor(out, "out", torch.bfloat16, inp.device)
+    if inp.shape != out.shape:
+        raise ValueError(f"inp {tuple(inp.shape)} and out {tuple(out.shape)} differ in shape")
+    return inp.device, inp.numel()
 
 
 def qlinear_route(inp: torch.Tensor, out: torch.Tensor, threshold: float = 0.05, stream=None,
@@ -187,17 +250,23 @@ def qlinear_route(inp: torch.Tensor, out: torch.Tensor, threshold: float = 0.05,
     """Returns device tensors (gamma float64 [1], route int32 [1]); reuses
     the given output and workspace tensors (a workspace stays valid across
     calls on one stream)."""
-    assert inp.dtype == torch.bfloat16 and out.dtype == torch.bfloat16
-    assert inp.shape == out.shape and inp.is_contiguous() and out.is_contiguous()
-    n = inp.numel()
-    if gamma is None:
-        gamma = torch.empty(1, dtype=torch.float64, device=inp.device)
-    if route is None:
-        route = torch.empty(1, dtype=torch.int32, device=inp.device)
-    if ws is None:
-        ws = _bytes(lib.qlinear_route_ws_bytes(n), inp.device)
-    _check("qlinear_route", lib.qlinear_route(_ptr(inp), _ptr(out), n, threshold, _ptr(gamma),
-                                              _ptr(route), _ptr(ws), ws.numel(), _stream(stream)))
+    dev, n = _block_pair(inp, out)
+    if gamma is not None:
+        _tensor(gamma, "gamma", torch.float64, dev, 8)
+    if route is not None:
+        _tensor(route, "route", torch.int32, dev, 4)
+    if ws is not None:
+        _tensor(ws, "ws", torch.uint8, dev)
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        if gamma is None:
+            gamma = torch.empty(1, dtype=torch.float64, device=dev)
+        if route is None:
+            route = torch.empty(1, dtype=torch.int32, device=dev)
+        if ws is None:
+            ws = _bytes(lib.qlinear_route_ws_bytes(n), dev)
+        _check("qlinear_route", lib.qlinear_route(_ptr(inp), _ptr(out), n, threshold, _ptr(gamma),
+                                                  _ptr(route), _ptr(ws), ws.numel(), st))
     return gamma, route
 
 
@@ -205,15 +274,19 @@ def qlinear_gamma_sums(inp: torch.Tensor, out: torch.Tensor, sums: torch.Tensor 
                        ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Device float64 [2]: (sum |out - in|, sum |in|) over these elements,
     this rank's share of Gamma when a block's tokens are split across ranks."""
-    assert inp.dtype == torch.bfloat16 and out.dtype == torch.bfloat16
-    assert inp.shape == out.shape and inp.is_contiguous() and out.is_contiguous()
-    n = inp.numel()
-    if sums is None:
-        sums = torch.empty(2, dtype=torch.float64, device=inp.device)
-    if ws is None:
-        ws = _bytes(lib.qlinear_route_ws_bytes(n), inp.device)
-    _check("qlinear_gamma_sums", lib.qlinear_gamma_sums(_ptr(inp), _ptr(out), n, _ptr(sums), _ptr(ws),
-                                                        ws.numel(), _stream(stream)))
+    dev, n = _block_pair(inp, out)
+    if sums is not None:
+        _tensor(sums, "sums", torch.float64, dev, 16)
+    if ws is not None:
+        _tensor(ws, "ws", torch.uint8, dev)
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        if sums is None:
+            sums = torch.empty(2, dtype=torch.float64, device=dev)
+        if ws is None:
+            ws = _bytes(lib.qlinear_route_ws_bytes(n), dev)
+        _check("qlinear_gamma_sums", lib.qlinear_gamma_sums(_ptr(inp), _ptr(out), n, _ptr(sums), _ptr(ws),
+                                                            ws.numel(), st))
     return sums
 
 
@@ -221,83 +294,125 @@ def qlinear_route_from_sums(sums: torch.Tensor, threshold: float = 0.05, gamma: 
                             route: torch.Tensor | None = None, stream=None):
     """Device tensors (gamma float64 [1], route int32 [1]) from the summed
     (sum |out - in|, sum |in|) of all ranks."""
-    assert sums.dtype == torch.float64 and sums.is_cuda and sums.numel() == 2 and sums.is_contiguous()
-    if gamma is None:
-        gamma = torch.empty(1, dtype=torch.float64, device=sums.device)
-    if route is None:
-        route = torch.empty(1, dtype=torch.int32, device=sums.device)
-    _check("qlinear_route_from_sums", lib.qlinear_route_from_sums(_ptr(sums), threshold, _ptr(gamma), _ptr(route),
-                                                                  _stream(stream)))
+    _tensor(sums, "sums", torch.float64, min_bytes=16)
+    dev = sums.device
+    if gamma is not None:
+        _tensor(gamma, "gamma", torch.float64, dev, 8)
+    if route is not None:
+        _tensor(route, "route", torch.int32, dev, 4)
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        if gamma is None:
+            gamma = torch.empty(1, dtype=torch.float64, device=dev)
+        if route is None:
+            route = torch.empty(1, dtype=torch.int32, device=dev)
+        _check("qlinear_route_from_sums", lib.qlinear_route_from_sums(_ptr(sums), threshold, _ptr(gamma),
+                                                                      _ptr(route), st))
     return gamma, route
 
 
 def qlinear_tensor_amax(X: torch.Tensor, hadamard: bool = True, out: torch.Tensor | None = None,
                         ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Device fp32 [1]: max |H x| (or |x|) over the tensor."""
-    assert X.dtype == torch.bfloat16 and X.is_cuda and X.dim() == 2 and X.is_contiguous()
+    _tensor(X, "X", torch.bfloat16, dim=2)
+    dev = X.device
     M, K = X.shape
-    if out is None:
-        out = torch.empty(1, dtype=torch.float32, device=X.device)
-    if ws is None:
-        ws = _bytes(lib.qlinear_quantize_ws_bytes(M, K, QL_ROUTE_NVFP4), X.device)
-    _check("qlinear_tensor_amax", lib.qlinear_tensor_amax(_ptr(X), M, K, int(bool(hadamard)), _ptr(out),
-                                                          _ptr(ws), ws.numel(), _stream(stream)))
+    if out is not None:
+        _tensor(out, "out", torch.float32, dev, 4)
+    if ws is not None:
+        _tensor(ws, "ws", torch.uint8, dev)
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.empty(1, dtype=torch.float32, device=dev)
+        if ws is None:
+            ws = _bytes(lib.qlinear_quantize_ws_bytes(M, K, QL_ROUTE_NVFP4), dev)
+        _check("qlinear_tensor_amax", lib.qlinear_tensor_amax(_ptr(X), M, K, int(bool(hadamard)), _ptr(out),
+                                                              _ptr(ws), ws.numel(), st))
     return out
+
+
+_ACT_DTYPES = {QL_ROUTE_NVFP4: torch.uint8, QL_ACT_NVFP4_DECOMP: torch.uint8, QL_ROUTE_INT8: torch.int8,
+               QL_ROUTE_INT6: torch.int8, QL_ACT_INT8_F16: torch.float16, QL_ACT_INT6_F16: torch.float16,
+               QL_ACT_INT8_TENSOR: torch.int8, QL_ACT_INT6_TENSOR: torch.int8}
 
 
 def qlinear_quantize_act(X: torch.Tensor, act_fmt: int, hadamard: bool = True,
                          w: PackedWeights | None = None, rowmajor_scales: bool = True,
                          amax_in: torch.Tensor | None = None, out: dict | None = None, stream=None):
     """Quantized activations as a dict of device tensors (reuses `out`'s
-    buffers when given)."""
-    assert X.dtype == torch.bfloat16 and X.is_cuda and X.dim() == 2 and X.is_contiguous()
-    M, K = X.shape
+    buffers when given; they must be large enough for X)."""
+    _tensor(X, "X", torch.bfloat16, dim=2)
     dev = X.device
-    if out is not None:
-        _check("qlinear_quantize_act",
-               lib.qlinear_quantize_act(_ptr(X), M, K, act_fmt, int(bool(hadamard)),
-                                        C.byref(w.desc) if w is not None else None, _ptr(amax_in),
-                                        _ptr(out["codes"]), _ptr(out["sf_mma"]), _ptr(out["sf_rowmajor"]),
-                                        _ptr(out["scales"]), _ptr(out["_ws"]), out["_ws"].numel(),
-                                        _stream(stream)))
-        return out
-    out = {}
-    sf_mma = sf_rm = None
-    if act_fmt in (QL_ROUTE_NVFP4, QL_ACT_NVFP4_DECOMP):
-        kq = 2 * K if act_fmt == QL_ACT_NVFP4_DECOMP else K     # decomposed: [q1 | q2] per row
-        codes = torch.empty((M, kq // 2), dtype=torch.uint8, device=dev)
-        sf_mma = _bytes(lib.qlinear_sf_bytes(M, kq), dev)
-        if rowmajor_scales:
-            sf_rm = torch.empty((M, kq // 16), dtype=torch.uint8, device=dev)
-        scales = torch.empty(1, dtype=torch.float32, device=dev)
-    elif act_fmt in (QL_ROUTE_INT8, QL_ROUTE_INT6):
-        codes = torch.empty((M, K), dtype=torch.int8, device=dev)
-        scales = torch.empty(max(M, 1), dtype=torch.float32, device=dev)
-    elif act_fmt in (QL_ACT_INT8_F16, QL_ACT_INT6_F16):
-        codes = torch.empty((M, K), dtype=torch.float16, device=dev)
-        scales = torch.empty(max(M, 1), dtype=torch.float32, device=dev)
-    else:
-        assert w is not None
-        codes = torch.empty((M, w.desc.Kp), dtype=torch.int8, device=dev)
-        scales = torch.empty(1, dtype=torch.float32, device=dev)
-    ws = _bytes(lib.qlinear_quantize_ws_bytes(M, K, act_fmt), dev)
+    M, K = X.shape
+    if w is not None:
+        _weights(w)
+    if act_fmt not in _ACT_DTYPES:
+        raise ValueError(f"unknown activation format {act_fmt}")
+    need = _act_bytes(M, K, act_fmt, w)
+    if amax_in is not None:
+        _tensor(amax_in, "amax_in", torch.float32, dev, 4)
+    st = _stream(stream, dev)
     wd = C.byref(w.desc) if w is not None else None
-    _check("qlinear_quantize_act",
-           lib.qlinear_quantize_act(_ptr(X), M, K, act_fmt, int(bool(hadamard)), wd, _ptr(amax_in),
-                                    _ptr(codes), _ptr(sf_mma), _ptr(sf_rm), _ptr(scales), _ptr(ws),
-                                    ws.numel(), _stream(stream)))
-    out.update(codes=codes, sf_mma=sf_mma, sf_rowmajor=sf_rm, scales=scales, _ws=ws)
-    return out
+    if out is not None:
+        for key in ("codes", "sf_mma", "sf_rowmajor", "scales"):
+            if out.get(key) is not None:
+                _tensor(out[key], f"out[{key!r}]", None, dev, need[key] if need[key] is not None else 0)
+        if need["sf_mma"] is not None and out.get("sf_mma") is None:
+            raise ValueError("out['sf_mma'] is required for the NVFP4 formats")
+        _tensor(out["_ws"], "out['_ws']", torch.uint8, dev)
+        with torch.cuda.device(dev):
+            _check("qlinear_quantize_act",
+                   lib.qlinear_quantize_act(_ptr(X), M, K, act_fmt, int(bool(hadamard)), wd, _ptr(amax_in),
+                                            _ptr(out["codes"]), _ptr(out.get("sf_mma")),
+                                            _ptr(out.get("sf_rowmajor")), _ptr(out["scales"]), _ptr(out["_ws"]),
+                                            out["_ws"].numel(), st))
+        return out
+    with torch.cuda.device(dev):
+        if act_fmt in (QL_ROUTE_NVFP4, QL_ACT_NVFP4_DECOMP):
+            kq = 2 * K if act_fmt == QL_ACT_NVFP4_DECOMP else K     # decomposed: [q1 | q2] per row
+            codes = torch.empty((M, kq // 2), dtype=torch.uint8, device=dev)
+            sf_mma = _bytes(need["sf_mma"], dev)
+            sf_rm = torch.empty((M, kq // 16), dtype=torch.uint8, device=dev) if rowmajor_scales else None
+        else:
+            width = w.desc.Kp if act_fmt in (QL_ACT_INT8_TENSOR, QL_ACT_INT6_TENSOR) else K
+            codes = torch.empty((M, width), dtype=_ACT_DTYPES[act_fmt], device=dev)
+            sf_mma = sf_rm = None
+        scales = torch.empty(need["scales"] // 4, dtype=torch.float32, device=dev)
+        ws = _bytes(lib.qlinear_quantize_ws_bytes(M, K, act_fmt), dev)
+        _check("qlinear_quantize_act",
+               lib.qlinear_quantize_act(_ptr(X), M, K, act_fmt, int(bool(hadamard)), wd, _ptr(amax_in),
+                                        _ptr(codes), _ptr(sf_mma), _ptr(sf_rm), _ptr(scales), _ptr(ws),
+                                        ws.numel(), st))
+    return dict(codes=codes, sf_mma=sf_mma, sf_rowmajor=sf_rm, scales=scales, _ws=ws)
+
+
+def _output(Y, M: int, N: int, dev):
+    if Y is None:
+        return torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    return _tensor(Y, "Y", torch.bfloat16, dev, 2 * M * N)
 
 
 def qlinear_gemm(act_fmt: int, q: dict, M: int, w: PackedWeights, Y: torch.Tensor | None = None,
                  stream=None) -> torch.Tensor:
-    dev = q["codes"].device
-    if Y is None:
-        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=dev)
-    _check("qlinear_gemm", lib.qlinear_gemm(act_fmt, _ptr(q["codes"]), _ptr(q.get("sf_mma")),
-                                            _ptr(q["scales"]), M, C.byref(w.desc), _ptr(Y),
-                                            _stream(stream)))
+    """Y [M, N] bf16 from quantized activations `q` (qlinear_quantize_act's
+    dict; for QL_ROUTE_BF16, {"codes": the bf16 input, "scales": None})."""
+    _weights(w)
+    M = int(M)
+    if M < 0:
+        raise ValueError(f"M must be >= 0, got {M}")
+    need = _act_bytes(M, w.K, act_fmt, w if act_fmt in (QL_ACT_INT8_TENSOR, QL_ACT_INT6_TENSOR) else None)
+    codes = _tensor(q["codes"], "q['codes']", None, None, need["codes"])
+    dev = codes.device
+    if need["sf_mma"] is not None and q.get("sf_mma") is not None:
+        _tensor(q["sf_mma"], "q['sf_mma']", None, dev, need["sf_mma"])
+    if need["scales"] is not None and q.get("scales") is not None:
+        _tensor(q["scales"], "q['scales']", torch.float32, dev, need["scales"])
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        Y = _output(Y, M, w.N, dev)
+        _check("qlinear_gemm", lib.qlinear_gemm(act_fmt, _ptr(codes), _ptr(q.get("sf_mma")), _ptr(q.get("scales")),
+                                                M, C.byref(w.desc), _ptr(Y), st))
     return Y
 
 
@@ -305,23 +420,32 @@ class ForwardPlan:
     """Workspace for repeated qlinear_forward calls with fixed shapes."""
 
     def __init__(self, M: int, w: PackedWeights, route: int, device):
-        self.M, self.w, self.route = M, w, route
+        self.M, self.w, self.route = M, _weights(w), route
         self.ws = _bytes(lib.qlinear_forward_ws_bytes(M, C.byref(w.desc), route), device)
+
+
+def _layer_input(X, w):
+    _tensor(X, "X", torch.bfloat16, dim=2)
+    _weights(w)
+    if X.shape[1] != w.K:
+        raise ValueError(f"X has {X.shape[1]} columns, the weights take K = {w.K}")
+    return X.device, X.shape[0]
 
 
 def qlinear_forward(X: torch.Tensor, w: PackedWeights, route: int = QL_ROUTE_NVFP4,
                     Y: torch.Tensor | None = None, plan: ForwardPlan | None = None,
                     stream=None) -> torch.Tensor:
-    assert X.dtype == torch.bfloat16 and X.is_cuda and X.dim() == 2 and X.is_contiguous()
-    M, K = X.shape
-    assert K == w.K
-    if Y is None:
-        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
-    if plan is None:
-        plan = ForwardPlan(M, w, route, X.device)
-    _check("qlinear_forward",
-           lib.qlinear_forward(_ptr(X), M, C.byref(w.desc), route, _ptr(Y), _ptr(plan.ws),
-                               plan.ws.numel(), _stream(stream)))
+    dev, M = _layer_input(X, w)
+    if plan is not None:
+        _tensor(plan.ws, "plan.ws", torch.uint8, dev)
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        Y = _output(Y, M, w.N, dev)
+        if plan is None:
+            plan = ForwardPlan(M, w, route, dev)
+        _check("qlinear_forward",
+               lib.qlinear_forward(_ptr(X), M, C.byref(w.desc), route, _ptr(Y), _ptr(plan.ws),
+                                   plan.ws.numel(), st))
     return Y
 
 
@@ -329,17 +453,18 @@ def qlinear_forward_routed(X: torch.Tensor, w: PackedWeights, route: torch.Tenso
                            ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Forward with the route read on the device (int32 [1] tensor, e.g. the
     router's output or a TDC state's next_route): no host synchronization."""
-    assert X.dtype == torch.bfloat16 and X.is_cuda and X.dim() == 2 and X.is_contiguous()
-    assert route.dtype == torch.int32 and route.is_cuda
-    M, K = X.shape
-    assert K == w.K
-    if Y is None:
-        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
-    if ws is None:
-        ws = _bytes(lib.qlinear_forward_routed_ws_bytes(M, C.byref(w.desc)), X.device)
-    _check("qlinear_forward_routed",
-           lib.qlinear_forward_routed(_ptr(X), M, C.byref(w.desc), _ptr(route), _ptr(Y), _ptr(ws), ws.numel(),
-                                      _stream(stream)))
+    dev, M = _layer_input(X, w)
+    _tensor(route, "route", torch.int32, dev, 4)
+    if ws is not None:
+        _tensor(ws, "ws", torch.uint8, dev)
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        Y = _output(Y, M, w.N, dev)
+        if ws is None:
+            ws = _bytes(lib.qlinear_forward_routed_ws_bytes(M, C.byref(w.desc)), dev)
+        _check("qlinear_forward_routed",
+               lib.qlinear_forward_routed(_ptr(X), M, C.byref(w.desc), _ptr(route), _ptr(Y), _ptr(ws), ws.numel(),
+                                          st))
     return Y
 
 
@@ -372,33 +497,53 @@ class TdcCache:
 
 
 def qlinear_tdc_init(cache: TdcCache, stream=None):
-    _check("qlinear_tdc_init", lib.qlinear_tdc_init(_ptr(cache.state_buf), _stream(stream)))
+    dev = cache.state_buf.device
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check("qlinear_tdc_init", lib.qlinear_tdc_init(_ptr(cache.state_buf), st))
+
+
+def _block_input(t, name, cache):
+    _tensor(t, name, torch.bfloat16, cache.slots.device)
+    if t.numel() != cache.numel:
+        raise ValueError(f"{name} has {t.numel()} elements, the cache holds {cache.numel}")
+    return t
 
 
 def qlinear_tdc_refresh(inp: torch.Tensor, out: torch.Tensor, cache: TdcCache, stream=None):
     """After computing the block: new delta, Gamma, E and the next decision (on the device)."""
-    assert inp.dtype == torch.bfloat16 and out.dtype == torch.bfloat16 and inp.shape == out.shape
-    assert inp.is_contiguous() and out.is_contiguous() and inp.numel() == cache.numel
-    _check("qlinear_tdc_refresh",
-           lib.qlinear_tdc_refresh(_ptr(inp), _ptr(out), cache.numel, _ptr(cache.slots[0]), _ptr(cache.slots[1]),
-                                   _ptr(cache.state_buf), C.byref(cache.params), _ptr(cache.ws), cache.ws.numel(),
-                                   _stream(stream)))
+    _block_input(inp, "inp", cache)
+    _block_input(out, "out", cache)
+    dev = cache.slots.device
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check("qlinear_tdc_refresh",
+               lib.qlinear_tdc_refresh(_ptr(inp), _ptr(out), cache.numel, _ptr(cache.slots[0]), _ptr(cache.slots[1]),
+                                       _ptr(cache.state_buf), C.byref(cache.params), _ptr(cache.ws),
+                                       cache.ws.numel(), st))
 
 
 def qlinear_tdc_skip(inp: torch.Tensor, cache: TdcCache, out: torch.Tensor | None = None, stream=None):
     """Skip the block: out = bf16(in + latest delta)."""
-    assert inp.dtype == torch.bfloat16 and inp.is_contiguous() and inp.numel() == cache.numel
-    if out is None:
-        out = torch.empty_like(inp)
-    _check("qlinear_tdc_skip",
-           lib.qlinear_tdc_skip(_ptr(inp), cache.numel, _ptr(cache.slots[0]), _ptr(cache.slots[1]),
-                                _ptr(cache.state_buf), C.byref(cache.params), _ptr(out), _stream(stream)))
+    _block_input(inp, "inp", cache)
+    if out is not None:
+        _block_input(out, "out", cache)
+    dev = cache.slots.device
+    st = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        if out is None:
+            out = torch.empty_like(inp)
+        _check("qlinear_tdc_skip",
+               lib.qlinear_tdc_skip(_ptr(inp), cache.numel, _ptr(cache.slots[0]), _ptr(cache.slots[1]),
+                                    _ptr(cache.state_buf), C.byref(cache.params), _ptr(out), st))
     return out
 
 
 def qlinear_device_status(stream=None) -> int:
+    """The current device's status word (0: no kernel has reported an error)."""
     v = C.c_int32(0)
-    _check("qlinear_device_status", lib.qlinear_device_status(_stream(stream), C.byref(v)))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check("qlinear_device_status", lib.qlinear_device_status(_stream(stream, dev), C.byref(v)))
     return v.value
 
 
@@ -409,9 +554,10 @@ def qlinear_debug_set_wait_limit(cycles: int):
 def qlinear_debug_div_check(d: float, a_begin: int, count: int, stream=None) -> int:
     """Number of dividends (fp32 bit patterns a_begin .. a_begin+count-1)
     where the quantizer's block-scale division by d is not correctly rounded."""
-    out = torch.zeros(1, dtype=torch.int64, device="cuda")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    out = torch.zeros(1, dtype=torch.int64, device=dev)
     _check("qlinear_debug_div_check", lib.qlinear_debug_div_check(float(d), int(a_begin), int(count),
-                                                                  _ptr(out), _stream(stream)))
+                                                                  _ptr(out), _stream(stream, dev)))
     return int(out.item())
 
 
