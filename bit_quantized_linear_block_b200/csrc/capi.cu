@@ -1,6 +1,7 @@
 // C ABI of the qlinear library: argument checks, workspace layout, tensor
 // maps and kernel sequencing.  Every entry point validates on the host
 // before touching CUDA, so a bad call enqueues nothing.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -25,7 +26,7 @@ int* g_status[kMaxDevices] = {nullptr};
 bool g_checked[kMaxDevices] = {false};
 bool g_ok_arch[kMaxDevices] = {false};
 std::unordered_map<const void*, int> g_smem_set[kMaxDevices];
-long long g_wait_limit = kDefaultWaitLimit;
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
 
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
@@ -143,7 +144,7 @@ void fill_gemm_args(GemmArgs& p, int64_t M, int N, int K, int BN, int* status) {
   p.tiles_n = (N + BN - 1) / BN;
   p.num_tiles = p.tiles_m * p.tiles_n;
   p.group_m = 8;
-  p.wait_limit = g_wait_limit;
+  p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
   p.status = status;
 }
 
@@ -168,6 +169,11 @@ ql_status check_m(int64_t M) {
 // Streaming kernels index 128-element blocks with 32-bit integers.
 ql_status check_mk(int64_t M, int64_t K) {
   if ((M + 127) / 128 * 128 * (K / 128) >= (int64_t(1) << 32)) return QL_ERR_UNSUPPORTED_SHAPE;
+  return QL_OK;
+}
+// The GEMMs count output tiles of 128 x 128 (or wider) in 32 bits.
+ql_status check_mn(int64_t M, int64_t N) {
+  if ((M + 127) / 128 * ((N + 127) / 128) >= (int64_t(1) << 31)) return QL_ERR_UNSUPPORTED_SHAPE;
   return QL_OK;
 }
 ql_status check_w(const ql_weights* w) {
@@ -245,7 +251,7 @@ const char* qlinear_status_string(int s) {
 }
 
 void qlinear_debug_set_wait_limit(long long cycles) {
-  g_wait_limit = cycles < 0 ? kDefaultWaitLimit : cycles;
+  g_wait_limit.store(cycles < 0 ? kDefaultWaitLimit : cycles, std::memory_order_relaxed);
 }
 
 ql_status qlinear_debug_div_check(float d, uint32_t a_begin, uint64_t count, unsigned long long* mismatches_dev,
@@ -546,6 +552,7 @@ ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf, c
                        int64_t M, const ql_weights* w, void* Y, void* stream) {
   QL_TRY(check_m(M));
   QL_TRY(check_w(w));
+  QL_TRY(check_mn(M, w->N));
   if (M > 0 && (a_codes == nullptr || (a_scales == nullptr && act_fmt != QL_ROUTE_BF16) || Y == nullptr))
     return QL_ERR_INVALID_ARG;
   act_fmt = int_base_fmt(act_fmt);   // INT6 codes run through the INT8 GEMMs unchanged
@@ -601,6 +608,7 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
   QL_TRY(check_m(M));
   QL_TRY(check_w(w));
   QL_TRY(check_mk(M, w->K));
+  QL_TRY(check_mn(M, w->N));
   if (ws == nullptr || (M > 0 && (X == nullptr || Y == nullptr))) return QL_ERR_INVALID_ARG;
   if (w->fmt == QL_W_NVFP4_DECOMP && route != QL_ROUTE_NVFP4) return QL_ERR_INVALID_ARG;
   if (route == QL_ROUTE_BF16) {   // PDR's high-precision refresh: the input as it is
@@ -669,6 +677,7 @@ ql_status qlinear_forward_routed(const void* X, int64_t M, const ql_weights* w, 
   QL_TRY(check_m(M));
   QL_TRY(check_w(w));
   QL_TRY(check_mk(M, w->K));
+  QL_TRY(check_mn(M, w->N));
   if (w->fmt != QL_W_NVFP4 || route_dev == nullptr || ws == nullptr || (M > 0 && (X == nullptr || Y == nullptr)))
     return QL_ERR_INVALID_ARG;
   if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(ws, 256) || !aligned(route_dev, 4)) return QL_ERR_ALIGNMENT;

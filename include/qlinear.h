@@ -32,8 +32,12 @@
  *     enqueues nothing.
  *   - Matrices are row-major.  X is [M, K] (tokens x in-features), W is
  *     [N, K] (nn.Linear layout), Y = X W^T is [M, N], all bf16.
- *   - K must be a multiple of 128 (the Hadamard block) and N a multiple of
- *     16.  M may be any value >= 0.
+ *   - K must be a multiple of 128 (the Hadamard block), at most 2^20, and N
+ *     a multiple of 16, at most 2^24.  M may be any value from 0 to
+ *     2^31 - 128, with ceil(M/128) * K < 2^32 (the streaming kernels index
+ *     128-element blocks in 32 bits) and, for the GEMMs,
+ *     ceil(M/128) * ceil(N/128) < 2^31 (output tiles).  A call beyond these
+ *     limits returns QL_ERR_UNSUPPORTED_SHAPE.
  *   - Non-finite inputs give unspecified (but memory-safe) results.
  *
  * Data layouts:

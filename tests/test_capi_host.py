@@ -124,6 +124,22 @@ def test_other_entry_points_reject_bad_arguments(ql):
     assert L.qlinear_gemm(0, FAKE, FAKE, FAKE, 10, None, FAKE, None) == 1
 
 
+def test_gemm_tile_count_limit(ql):
+    """ceil(M/128) * ceil(N/128) must stay below 2^31: at the limit the GEMM
+    entry points refuse the shape before anything else."""
+    import torch
+    L = ql.lib
+    w = ql.Weights(fmt=ql.QL_W_NVFP4, N=1 << 22, K=128, hadamard=1, codes=FAKE, sf=FAKE, gscale=FAKE)
+    m_over = (1 << 16) * 128                      # 2^16 x 2^15 tiles = 2^31
+    assert L.qlinear_gemm(0, FAKE, FAKE, FAKE, m_over, C.byref(w), FAKE, None) == 2
+    assert L.qlinear_forward(FAKE, m_over, C.byref(w), 0, FAKE, FAKE, 1 << 62, None) == 2
+    assert L.qlinear_forward_routed(FAKE, m_over, C.byref(w), FAKE, FAKE, FAKE, 1 << 62, None) == 2
+    if not torch.cuda.is_available():             # one tile row less passes every check but the device
+        m_under = m_over - 128
+        assert L.qlinear_gemm(0, FAKE, FAKE, FAKE, m_under, C.byref(w), FAKE, None) == 7
+        assert L.qlinear_forward(FAKE, m_under, C.byref(w), 0, FAKE, FAKE, 1 << 62, None) == 7
+
+
 def test_valid_call_without_a_device_reports_no_device(ql):
     import torch
     if torch.cuda.is_available():
