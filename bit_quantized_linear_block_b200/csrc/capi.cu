@@ -166,9 +166,11 @@ ql_status check_m(int64_t M) {
   if (M > (int64_t(1) << 31) - 128) return QL_ERR_UNSUPPORTED_SHAPE;
   return QL_OK;
 }
-// Streaming kernels index 128-element blocks with 32-bit integers.
+// Streaming kernels index 128-element blocks with 32-bit integers and
+// address the input as 128-byte TMA rows with 32-bit row coordinates.
 ql_status check_mk(int64_t M, int64_t K) {
   if ((M + 127) / 128 * 128 * (K / 128) >= (int64_t(1) << 32)) return QL_ERR_UNSUPPORTED_SHAPE;
+  if (M * K >= (int64_t(1) << 37)) return QL_ERR_UNSUPPORTED_SHAPE;
   return QL_OK;
 }
 // The GEMMs count output tiles of 128 x 128 (or wider) in 32 bits.

@@ -34,8 +34,9 @@
  *     [N, K] (nn.Linear layout), Y = X W^T is [M, N], all bf16.
  *   - K must be a multiple of 128 (the Hadamard block), at most 2^20, and N
  *     a multiple of 16, at most 2^24.  M may be any value from 0 to
- *     2^31 - 128, with ceil(M/128) * K < 2^32 (the streaming kernels index
- *     128-element blocks in 32 bits) and, for the GEMMs,
+ *     2^31 - 128, with ceil(M/128) * K < 2^32 and M * K < 2^37 (the
+ *     streaming kernels index 128-element blocks in 32 bits and read the
+ *     input as 128-byte rows with 32-bit coordinates) and, for the GEMMs,
  *     ceil(M/128) * ceil(N/128) < 2^31 (output tiles).  A call beyond these
  *     limits returns QL_ERR_UNSUPPORTED_SHAPE.
  *   - Non-finite inputs give unspecified (but memory-safe) results.

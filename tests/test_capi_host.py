@@ -140,6 +140,15 @@ def test_gemm_tile_count_limit(ql):
         assert L.qlinear_forward(FAKE, m_under, C.byref(w), 0, FAKE, FAKE, 1 << 62, None) == 7
 
 
+def test_streaming_size_limit(ql):
+    """M * K < 2^37: the streaming kernels read the input as 128-byte TMA rows
+    with 32-bit row coordinates (2^20 x 2^17 passes the block-count rule)."""
+    L = ql.lib
+    assert L.qlinear_tensor_amax(FAKE, 1 << 20, 1 << 17, 1, FAKE, FAKE, 1 << 62, None) == 2
+    assert L.qlinear_quantize_act(FAKE, 1 << 20, 1 << 17, 0, 1, None, None, FAKE, FAKE, None, FAKE, FAKE,
+                                  1 << 62, None) == 2
+
+
 def test_valid_call_without_a_device_reports_no_device(ql):
     import torch
     if torch.cuda.is_available():
