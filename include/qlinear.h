@@ -200,7 +200,12 @@ QL_API size_t qlinear_sf_bytes(int64_t rows, int32_t K);
    Q-ARVD (Q-ARVD, Methodology / Formula and operation flow): channel norms,
    median/MAD z-score mask, class-ordered permutation, per-row dual INT4
    scales, INT4 codes.  The weight buffer (qlinear_weights_bytes) holds every
-   output; `ws` is scratch (qlinear_prepare_ws_bytes).  Asynchronous. */
+   output; `ws` is scratch (qlinear_prepare_ws_bytes).  Asynchronous.
+   Q-ARVD weights need hadamard = 0, tau > 0, alpha >= 0 and K <= 16384 (one
+   CTA sorts all channel norms in shared memory); otherwise the call returns
+   QL_ERR_INVALID_ARG.  The per-tensor Q-ARVD activation quantizer stages a
+   row in shared memory and returns QL_ERR_UNSUPPORTED_SHAPE when that does
+   not fit (about K > 29000). */
 QL_API size_t qlinear_weights_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg);
 QL_API size_t qlinear_prepare_ws_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg);
 QL_API ql_status qlinear_prepare_weights(const void* W_bf16, int32_t N, int32_t K,
