@@ -287,7 +287,10 @@ QL_API ql_status qlinear_tensor_amax(const void* X_bf16, int64_t M, int32_t K, i
    `hadamard` = 1 rotates each 128-block of K first (NVFP4 / INT8 routes).
    amax_in: optional device fp32 tensor amax (NVFP4 and per-tensor INT8),
    e.g. from qlinear_tensor_amax or a calibrated static value; NULL makes the
-   call compute the dynamic amax itself (one extra launch). */
+   call compute the dynamic amax itself (one extra launch).
+   The per-token formats keep two token rows per warp in shared memory:
+   K > 51200 returns QL_ERR_UNSUPPORTED_SHAPE there (and on the INT8 / INT6
+   routes of qlinear_forward). */
 QL_API size_t qlinear_quantize_ws_bytes(int64_t M, int32_t K, int32_t act_fmt);
 QL_API ql_status qlinear_quantize_act(const void* X_bf16, int64_t M, int32_t K,
                                       int32_t act_fmt, int32_t hadamard, const ql_weights* w,
