@@ -185,6 +185,11 @@ def _bytes(n: int, device) -> torch.Tensor:
     return torch.zeros(max(int(n), 256), dtype=torch.uint8, device=device)
 
 
+_WEIGHT_SIZES = ("fmt", "N", "K", "hadamard", "Kp")
+_WEIGHT_ARRAYS = ("codes", "sf", "gscale", "outlier_mask", "perm", "gather", "kinfo", "s_norm", "s_out", "norms",
+                  "w16", "w8", "wbf16")
+
+
 @dataclass
 class PackedWeights:
     """Packed weights: the C descriptor plus the device buffer it points into."""
@@ -200,6 +205,47 @@ class PackedWeights:
         off = addr - self.buf.data_ptr()
         itemsize = torch.empty(0, dtype=dtype).element_size()
         return self.buf[off:off + count * itemsize].view(dtype)
+
+    def state_dict(self) -> dict:
+        """Host copy for a checkpoint (torch.save): the descriptor's sizes,
+        each array as a byte offset into the weight buffer (None for an
+        absent one), and the buffer's bytes as a CPU uint8 tensor.  Copying
+        the buffer waits for the work that wrote it."""
+        base, end = self.buf.data_ptr(), self.buf.data_ptr() + self.buf.numel()
+        offsets = {}
+        for f in _WEIGHT_ARRAYS:
+            p = getattr(self.desc, f)
+            if p is None:
+                offsets[f] = None
+            elif base <= p < end:
+                offsets[f] = p - base
+            else:
+                raise ValueError(f"weights array {f} does not point into the weight buffer")
+        return {"abi": lib.qlinear_abi_version(),
+                "sizes": {f: int(getattr(self.desc, f)) for f in _WEIGHT_SIZES},
+                "offsets": offsets, "buf": self.buf.detach().to("cpu", copy=True)}
+
+    @classmethod
+    def from_state_dict(cls, sd: dict, device) -> "PackedWeights":
+        """Packed weights on `device` from state_dict()'s output (same ABI
+        version): the bytes are copied into a new buffer and every array
+        pointer is rebased onto it."""
+        if sd.get("abi") != lib.qlinear_abi_version():
+            raise ValueError(f"packed weights of ABI {sd.get('abi')}, this library is ABI {lib.qlinear_abi_version()}")
+        host = sd["buf"]
+        if not isinstance(host, torch.Tensor) or host.dtype != torch.uint8 or host.dim() != 1:
+            raise TypeError("state_dict['buf'] must be a 1-D uint8 tensor")
+        buf = torch.empty(host.numel(), dtype=torch.uint8, device=device)
+        buf.copy_(host)
+        desc = Weights()
+        for f in _WEIGHT_SIZES:
+            setattr(desc, f, int(sd["sizes"][f]))
+        for f in _WEIGHT_ARRAYS:
+            off = sd["offsets"][f]
+            if off is not None and not 0 <= off < buf.numel():
+                raise ValueError(f"offset of {f} lies outside the weight buffer")
+            setattr(desc, f, None if off is None else buf.data_ptr() + off)
+        return cls(desc, buf, desc.N, desc.K, desc.fmt)
 
 
 # ----------------------------------------------------------------------------

@@ -3,7 +3,9 @@ TDC skip output, is placed inside a larger buffer whose margins hold a
 canary pattern.  After the call the margins must be unchanged and Y must
 equal the output of the same call into a buffer of its own.  The shapes
 are ragged (M not a multiple of 128, N not a multiple of the tile width)
-so that the last tiles are partial."""
+so that the last tiles are partial.  The same prepared weights also go
+through a checkpoint (state_dict, torch.save, from_state_dict) and must
+give the identical forward."""
 import pytest
 import torch
 
@@ -83,3 +85,21 @@ def test_tdc_skip_writes_only_its_output(ql):
     assert ql.qlinear_device_status() == 0
     assert _margins_intact(big, numel)
     assert torch.equal(guarded.view(-1), plain)
+
+
+@pytest.mark.parametrize("kind,route,m,n,k", [CASES[0], CASES[3], CASES[5], CASES[7], CASES[8]])
+def test_checkpointed_weights_give_the_same_output(ql, kind, route, m, n, k):
+    """Packed weights saved with torch.save(pw.state_dict()) and reloaded onto
+    the device produce the identical forward."""
+    import io
+    x = S.activations_fixed_outliers(m, k, 8, 50.0, m + n, 1).cuda()
+    pw = _prepare(ql, kind, n, k, m + n + k)
+    y0 = ql.qlinear_forward(x, pw, route)
+    f = io.BytesIO()
+    torch.save(pw.state_dict(), f)
+    f.seek(0)
+    pw2 = ql.PackedWeights.from_state_dict(torch.load(f), "cuda")
+    y1 = ql.qlinear_forward(x, pw2, route)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    assert torch.equal(y0, y1)
