@@ -90,7 +90,8 @@ def test_tdc_skip_writes_only_its_output(ql):
 @pytest.mark.parametrize("kind,route,m,n,k", [CASES[0], CASES[3], CASES[5], CASES[7], CASES[8]])
 def test_checkpointed_weights_give_the_same_output(ql, kind, route, m, n, k):
     """Packed weights saved with torch.save(pw.state_dict()) and reloaded onto
-    the device produce the identical forward."""
+    the device produce the identical forward, with the original buffer
+    zeroed (the weight buffer holds no addresses)."""
     import io
     x = S.activations_fixed_outliers(m, k, 8, 50.0, m + n, 1).cuda()
     pw = _prepare(ql, kind, n, k, m + n + k)
@@ -99,6 +100,7 @@ def test_checkpointed_weights_give_the_same_output(ql, kind, route, m, n, k):
     torch.save(pw.state_dict(), f)
     f.seek(0)
     pw2 = ql.PackedWeights.from_state_dict(torch.load(f), "cuda")
+    pw.buf.zero_()        # the reloaded weights must not read the original buffer
     y1 = ql.qlinear_forward(x, pw2, route)
     torch.cuda.synchronize()
     assert ql.qlinear_device_status() == 0
