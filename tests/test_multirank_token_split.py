@@ -101,3 +101,25 @@ def test_two_gloo_ranks_reproduce_the_unsplit_block():
     packed, sb, _ = O.nvfp4_quantize(h)
     assert np.array_equal(np.concatenate([res[0][5], res[1][5]]), packed)
     assert np.array_equal(np.concatenate([res[0][6], res[1][6]]), sb)
+
+
+def test_activation_format_follows_the_forward():
+    """Which activation format the token-split forward quantizes to, whether
+    it rotates, and whether it needs the block-wide amax: the choices
+    qlinear_forward makes for each weight format and route."""
+    import torch
+    from bit_quantized_linear_block_b200 import qlinear as Q, sharded as SH
+
+    def packed(fmt, hadamard):
+        return Q.PackedWeights(Q.Weights(fmt=fmt, N=64, K=128, hadamard=hadamard), torch.zeros(1), 64, 128, fmt)
+
+    nv, qa, de = packed(Q.QL_W_NVFP4, 1), packed(Q.QL_W_QARVD_INT4, 0), packed(Q.QL_W_NVFP4_DECOMP, 1)
+    assert SH.activation_format(nv, Q.QL_ROUTE_NVFP4) == (Q.QL_ROUTE_NVFP4, True, True)
+    for route in (Q.QL_ROUTE_INT8, Q.QL_ROUTE_INT6, Q.QL_ACT_INT8_F16, Q.QL_ROUTE_BF16):
+        assert SH.activation_format(nv, route) == (route, True, False)      # per token or unquantized
+    assert SH.activation_format(qa, Q.QL_ACT_INT8_TENSOR) == (Q.QL_ACT_INT8_TENSOR, False, True)
+    assert SH.activation_format(qa, Q.QL_ROUTE_INT6) == (Q.QL_ACT_INT6_TENSOR, False, True)
+    assert SH.activation_format(qa, Q.QL_ACT_INT6_TENSOR) == (Q.QL_ACT_INT6_TENSOR, False, True)
+    assert SH.activation_format(de, Q.QL_ROUTE_NVFP4) == (Q.QL_ACT_NVFP4_DECOMP, True, True)
+    with pytest.raises(ValueError):
+        SH.activation_format(de, Q.QL_ROUTE_INT8)
