@@ -639,7 +639,7 @@ static ql_status launch_qarvd_pre(const void* a_codes, const float* s_x, int64_t
     (void)cudaGetLastError();
     return QL_ERR_CUDA;
   }
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  return QL_OK;
 }
 
 // Sign-extend the packed INT4 weight codes to int8 ([N, Kp/2] bytes ->

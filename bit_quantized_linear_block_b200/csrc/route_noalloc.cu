@@ -79,8 +79,16 @@ extern "C" ql_status qlinear_route_noalloc(const void* in, const void* out, int6
   if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + kTicketOffset, 0, sizeof(unsigned int), st) !=
       cudaSuccess)
     return QL_ERR_CUDA;
-  k_gamma_route_static<<<static_cast<unsigned int>(grid), ql::kThreadsHbm, 0, st>>>(
-      static_cast<const uint4*>(in), static_cast<const uint4*>(out), numel,
-      static_cast<unsigned char*>(scratch), threshold, gamma_dev, route_dev);
-  return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
+  // The launch's own return code decides success: an error left pending by
+  // an unrelated earlier call is not this call's failure.
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned int>(grid));
+  cfg.blockDim = dim3(ql::kThreadsHbm);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_gamma_route_static, static_cast<const uint4*>(in),
+                                           static_cast<const uint4*>(out), numel,
+                                           static_cast<unsigned char*>(scratch), threshold, gamma_dev,
+                                           route_dev);
+  return e == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }

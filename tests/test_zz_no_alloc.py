@@ -3,7 +3,8 @@ meant for callers that cannot allocate device memory or pass a workspace
 (an engine or plugin host that owns all device memory, a loop that must not
 call cudaMalloc).  It keeps its scratch in a static device array shared by
 every call, so this test calls it twice in a row, on different inputs, and
-checks each result against the workspace-based qlinear_route within the
+checks each result against the workspace-based qlinear_route and against
+the oracle's Gamma and route (6Bit-Diffusion, Methodology B.1) within the
 tolerance the other router tests use.  The file is named to be collected
 last."""
 import ctypes as C
@@ -11,6 +12,8 @@ import ctypes as C
 import numpy as np
 import pytest
 import torch
+
+from oracle import qlinear_oracle as O
 
 pytestmark = pytest.mark.gpu
 
@@ -43,4 +46,8 @@ def test_route_noalloc_matches_route_on_two_calls():
         torch.cuda.synchronize()
         assert float(g.item()) == pytest.approx(float(g_ref.item()), rel=1e-12)
         assert int(r.item()) == int(r_ref.item())
+        g_or = O.dmpq_gamma(S.bf16_bits(xd.cpu()), S.bf16_bits(yd.cpu()))
+        assert abs(g_or - 0.05) / 0.05 > 1e-9
+        assert float(g.item()) == pytest.approx(g_or, rel=1e-12)
+        assert int(r.item()) == O.dmpq_route(g_or, 0.05)
     assert int(r_ref.item()) == 0 and ql.qlinear_device_status() == 0
