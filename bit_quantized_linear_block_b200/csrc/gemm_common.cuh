@@ -138,7 +138,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t acc_tmem, uint64_t* tempt
   constexpr int CH = BN / kEpiChunkCols;
   if (row_scale != nullptr) {
     const int m = m0 + (threadIdx.x & 127);
-    alpha = (m < M) ? __fmul_rn(alpha, __ldg(row_scale + m)) : 0.f;
+    alpha = (m < M) ? __fmul_rn(alpha, ld_dep(row_scale + m)) : 0.f;
   }
 #pragma unroll 1
   for (int c = 0; c < CH; ++c) {
@@ -216,7 +216,7 @@ __device__ __forceinline__ void epilogue_warp_tile(uint32_t taddr, uint32_t rele
   if (lane == 0) mbar_arrive_cluster(release);
   if (row_scale != nullptr) {
     const int row = row0 + lane;
-    alpha = (row < M) ? __fmul_rn(alpha, __ldg(row_scale + row)) : 0.f;
+    alpha = (row < M) ? __fmul_rn(alpha, ld_dep(row_scale + row)) : 0.f;
   }
   if (row0 >= M) return;   // warp-uniform
   const uint32_t swz = (lane >> 1) & 3;

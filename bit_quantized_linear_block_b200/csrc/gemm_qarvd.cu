@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp >= 12) {
     // ------------------------------------------------------------ epilogue
-    const float sx = *p.g_a;
+    const float sx = ld_dep(p.g_a);
     const int ew = warp & 3;
     const int lane = lane_id();
     const int row = threadIdx.x & 127;
@@ -513,7 +513,7 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------ epilogue
     // y = bf16(s_x * (s_norm[n] * acc_normal + s_out[n] * acc_outlier)); a
     // class without channels contributes 0 (its accumulator is never written).
-    const float sx = *p.g_a;
+    const float sx = ld_dep(p.g_a);
     const int quarter = warp & 3;
     const int half = (warp - 4) >> 2;
     const int lane = lane_id();

@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp >= 12) {
     // ------------------------------------------------------------ epilogue
-    const float alpha = BF16 ? 1.f : __fmul_rn(*p.g_w, p.alpha_mul);   // the bf16 product is unscaled
+    const float alpha = BF16 ? 1.f : __fmul_rn(ld_dep(p.g_w), p.alpha_mul);   // the bf16 product is unscaled
     EpilogueState es{};
     int local = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {

@@ -313,6 +313,12 @@ __device__ __forceinline__ void tc_mma_i8_pair(uint32_t d_tmem, uint64_t adesc, 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// Load of a value that an earlier kernel of the stream wrote (a tensor amax,
+// per-token scales).  Never through the read-only path: a load the compiler
+// may treat as invariant could be hoisted above pdl_wait() and read the
+// value before its producer has written it.
+__device__ __forceinline__ float ld_dep(const float* p) { return *reinterpret_cast<const volatile float*>(p); }
+
 // Route gate of the device-routed forward: a launch of one route's kernel
 // returns at once when the route in device memory is another one.  Read
 // after pdl_wait() (an earlier kernel of the stream may have written it).
