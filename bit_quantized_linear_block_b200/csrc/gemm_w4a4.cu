@@ -21,23 +21,29 @@
 //   warp 2      tensor-memory allocation;
 //   warps 4-11  epilogue, two warps per TMEM lane quarter, each with half of
 //               the tile's columns: tcgen05.ld, * alpha, bf16, TMA store of
-//               32 x 32 boxes from per-warp staging buffers.  Two
-//               accumulators let the epilogue of one tile overlap the main
+//               32 x 32 boxes from per-warp staging buffers.  With two
+//               accumulators the epilogue of one tile overlaps the main
 //               loop of the next.
 //
-// The tensor pipe takes about the same time (~44 SM cycles) for every
-// tcgen05 instruction it is handed, scale copies included, so with three
-// scale copies per MMA (one atom of A scales, two of B scales for BN = 192)
-// the main loop is bound by instruction count, not by the MMA math.  Two
-// ways to feed the scales:
+// Measured on this GPU, the tensor pipe runs block-scaled MMAs at their
+// math rate (N / 2 cycles per 64-deep K step of a CTA pair) whatever the
+// number of scale copies issued beside them, and is not slowed by
+// concurrent shared-memory, tensor-memory or bulk-copy traffic.  The main
+// loop is bound by the latency of its operand loads instead: a stage of
+// TMA loads takes about 1500-2000 cycles to land, and shared memory holds
+// only four to six stages, so the deeper the ring (in MMA cycles per byte
+// of shared memory), the faster the loop.  Scale feeding:
 //   RES = true    (K <= 64 * kResKSteps) the activation scales of a
 //                 128-row block for the whole K range stay resident in
 //                 tensor memory while the unit walks the N tiles of that
 //                 row block (tiles are handed out in contiguous row-major
-//                 ranges); they are reloaded only when the row block
-//                 changes, so a K step costs its B-scale copies plus one
-//                 MMA.  The B scales of each K step go to one of SFB_SLOTS
-//                 small slots.
+//                 ranges); the B scales of each K step go to one of
+//                 SFB_SLOTS small slots.
+//     APANEL      additionally keeps the row block's A tiles for the whole K
+//                 range in shared memory, so only B and its scales stream
+//                 through the ring (half the bytes per stage); the panel is
+//                 reloaded chunk by chunk, each chunk as soon as the MMAs of
+//                 the row block's last tile have read it.
 //   RES = false   the A and B scales of each stage are copied per stage into
 //                 one of SF_SLOTS slots (rotating per stage).
 // The tensor pipe runs the copies and MMAs of one issuing thread in issue
@@ -52,7 +58,7 @@ namespace ql {
 
 constexpr int kResKSteps = 30;   // K steps (64 wide) of resident activation scales
 
-template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES, int BKB_ = 128>
+template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES, int BKB_ = 128, bool APANEL = false>
 struct W4A4Cfg {
   static constexpr int CTAS = PAIR ? 2 : 1;
   static constexpr int BM = 128;                     // rows per CTA
@@ -64,6 +70,11 @@ struct W4A4Cfg {
   static constexpr int B_CHUNK = BNL * 128;
   static constexpr int A_BYTES = KC * A_CHUNK;
   static constexpr int B_BYTES = KC * B_CHUNK;
+  // APANEL: the A tiles of the current row block for the whole K range stay
+  // in shared memory (one chunk of A_CHUNK bytes per K stage) while the unit
+  // walks that row block's N tiles, so only B streams through the ring.
+  static constexpr int APCH = APANEL ? (kResKSteps + KSTEPS - 1) / KSTEPS : 0;   // panel chunks
+  static constexpr int A_RING = APANEL ? APCH * A_CHUNK : STAGES * A_BYTES;
   // 128-row scale atoms per B tile.  Each CTA of a pair holds the weight
   // scales of all BN rows: each SM's MMA reads every B row's scales from its
   // own tensor memory.
@@ -76,13 +87,13 @@ struct W4A4Cfg {
   static constexpr int EPI_WARPS = 8;
   static constexpr int EPI_CH = BN / 2 / kWarpBoxCols;   // boxes per epilogue warp per tile
   static constexpr int OFF_A = 0;
-  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_B = OFF_A + A_RING;
   static constexpr int OFF_SFB = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_SFA = OFF_SFB + STAGES * SFB_BYTES;
   static constexpr int OFF_SFA_RES = OFF_SFA + STAGES * SFA_BYTES;
   static constexpr int OFF_C = OFF_SFA_RES + ((SFA_RES_BYTES + 1023) / 1024) * 1024;
   static constexpr int OFF_BAR = OFF_C + EPI_WARPS * EPI_BUF * kWarpBoxBytes;
-  static constexpr int NBAR = 2 * STAGES + 2 * ACC + 1 + 2;
+  static constexpr int NBAR = 2 * STAGES + 2 * ACC + 1 + 2 + 2 * APCH;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
   // Tensor memory: ACC accumulators of BN columns, then the scales.
@@ -103,6 +114,7 @@ struct W4A4Cfg {
   static_assert(A_CHUNK % 1024 == 0 && B_CHUNK % 1024 == 0, "1024-byte aligned chunks");
   static_assert(BKB % 128 == 0 && (RES || BKB == 128), "streamed scales take 128-byte stages");
   static_assert(EPI_BUF >= 1 && EPI_BUF <= EPI_CH, "staging buffers");
+  static_assert(!APANEL || (RES && KC == 1), "the A panel goes with resident scales and 128-byte stages");
   // Instruction descriptor (block-scaled): A/B = E2M1 (1), scale = UE4M3 (0),
   // both K-major, N >> 3 at bit 17, M >> 4 at bit 24, dense K = 64.
   static constexpr uint32_t IDESC =
@@ -136,12 +148,12 @@ struct TileWalk {
   }
 };
 
-template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES, int BKB_>
+template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES, int BKB_, bool APANEL>
 __global__ void __launch_bounds__(384, 1)
     k_gemm_w4a4(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
                 const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
-  using C = W4A4Cfg<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_>;
+  using C = W4A4Cfg<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_, APANEL>;
   if (p.gate != nullptr) {   // device-routed forward: both CTAs of a pair read the same route
     pdl_wait();
     if (gated_off(p.gate, p.gate_value)) {
@@ -158,6 +170,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* drain = tempty + C::ACC;
   uint64_t* sfa_full = drain + 1;                                   // RES: pair: the leader's is used
   uint64_t* sfa_empty = sfa_full + 1;
+  uint64_t* a_full = sfa_empty + 1;                                 // APANEL: per chunk; pair: the leader's
+  uint64_t* a_empty = a_full + C::APCH;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -185,6 +199,10 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(drain, 1);
     mbar_init(sfa_full, 1);
     mbar_init(sfa_empty, 1);
+    for (int i = 0; i < C::APCH; ++i) {
+      mbar_init(&a_full[i], 1);
+      mbar_init(&a_empty[i], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -204,11 +222,12 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (elect_one()) {
-      int it = 0, nsfa = 0, cur_mb = -1;
+      int it = 0, nsfa = 0, cur_mb = -1, a_issued = 0;
       bool ok = true;
       for (int t = walk.begin; t < walk.end && ok; t += walk.step) {
         int mb, nb;
         walk.coords(t, p, mb, nb);
+        const bool newrb = mb != cur_mb;   // first tile of a row block (RES walks)
         const int n0 = nb * BN;
         const int ra0 = n0 >> 7;
         const int a_row = mb * C::BM * C::CTAS + static_cast<int>(rank) * C::BM;
@@ -237,10 +256,31 @@ __global__ void __launch_bounds__(384, 1)
         int nsfb = 0;
 #pragma unroll
         for (int r = 0; r < C::NSFB; ++r) nsfb += (ra0 + r < p.sfb_atoms);
-        const uint32_t tx = C::A_BYTES + C::B_BYTES + C::SFA_BYTES + nsfb * C::SFB_GROUP;
+        const uint32_t tx = (APANEL ? 0u : C::A_BYTES) + C::B_BYTES + C::SFA_BYTES + nsfb * C::SFB_GROUP;
+        if (APANEL && newrb) a_issued = 0;
         for (int ks = 0; ks < p.num_kst; ++ks, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
+          if constexpr (APANEL) {
+            if (newrb) {
+              // Chunk ks of the new row block's A panel, once the MMAs of the
+              // previous row block's last tile have read the old chunk.
+              const int gen = nsfa - 1;
+              if (gen > 0 && (*abort_flag || !mbar_wait(&a_empty[ks], (gen - 1) & 1, p.wait_limit))) {
+                ok = false;
+                break;
+              }
+              uint8_t* pa = smem + C::OFF_A + ks * C::A_CHUNK;
+              if constexpr (PAIR) {
+                if (leader) mbar_arrive_expect_tx(&a_full[ks], 2 * C::A_CHUNK);
+                tma_load_2d_pair(pa, &tm_a, map_to_rank(smem_u32(&a_full[ks]), 0), ks * C::BKB, a_row);
+              } else {
+                mbar_arrive_expect_tx(&a_full[ks], C::A_CHUNK);
+                tma_load_2d(pa, &tm_a, &a_full[ks], ks * C::BKB, a_row);
+              }
+              a_issued = ks + 1;
+            }
+          }
           if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1, p.wait_limit)) {
             ok = false;
             break;
@@ -255,7 +295,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t bar = map_to_rank(smem_u32(&full[s]), 0);
 #pragma unroll
             for (int c = 0; c < C::KC; ++c) {
-              tma_load_2d_pair(sa + c * C::A_CHUNK, &tm_a, bar, ks * C::BKB + 128 * c, a_row);
+              if constexpr (!APANEL) tma_load_2d_pair(sa + c * C::A_CHUNK, &tm_a, bar, ks * C::BKB + 128 * c, a_row);
               tma_load_2d_pair(sb + c * C::B_CHUNK, &tm_b, bar, ks * C::BKB + 128 * c, b_row);
             }
             if constexpr (!RES) tma_load_3d_pair(ssfa, &tm_sfa, bar, 0, C::KSTEPS * ks, sfa_group);
@@ -267,7 +307,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_arrive_expect_tx(&full[s], tx);
 #pragma unroll
             for (int c = 0; c < C::KC; ++c) {
-              tma_load_2d(sa + c * C::A_CHUNK, &tm_a, &full[s], ks * C::BKB + 128 * c, a_row);
+              if constexpr (!APANEL) tma_load_2d(sa + c * C::A_CHUNK, &tm_a, &full[s], ks * C::BKB + 128 * c, a_row);
               tma_load_2d(sb + c * C::B_CHUNK, &tm_b, &full[s], ks * C::BKB + 128 * c, b_row);
             }
             if constexpr (!RES) tma_load_3d(ssfa, &tm_sfa, &full[s], 0, C::KSTEPS * ks, sfa_group);
@@ -282,12 +322,18 @@ __global__ void __launch_bounds__(384, 1)
       if (leader) {
         drain_loads(full, it, STAGES, p.status);   // pair: covers both CTAs' bytes
         if (RES && nsfa > 0 && !mbar_wait(sfa_full, (nsfa - 1) & 1, kDrainLimit)) record_error(p.status, QL_ERR_TIMEOUT);
+        if (APANEL)   // the last panel's chunks have landed
+          for (int c = 0; c < a_issued; ++c)
+            if (!mbar_wait(&a_full[c], (nsfa - 1) & 1, kDrainLimit)) record_error(p.status, QL_ERR_TIMEOUT);
       } else {
         // The peer's loads complete on the leader's barriers; the leader frees
         // each stage (empty) only after the MMAs consumed both halves.
         for (int j = max(0, it - STAGES); j < it; ++j)
           if (!mbar_wait(&empty[j % STAGES], (j / STAGES) & 1, kDrainLimit)) record_error(p.status, QL_ERR_TIMEOUT);
         if (RES && nsfa > 0 && !mbar_wait(sfa_empty, (nsfa - 1) & 1, kDrainLimit)) record_error(p.status, QL_ERR_TIMEOUT);
+        if (APANEL)   // ... and each panel chunk after the last tile's MMAs read it
+          for (int c = 0; c < a_issued; ++c)
+            if (!mbar_wait(&a_empty[c], (nsfa - 1) & 1, kDrainLimit)) record_error(p.status, QL_ERR_TIMEOUT);
       }
     }
   } else if (warp == 1) {
@@ -311,6 +357,13 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = walk.begin; t < walk.end && ok; t += walk.step, ++local) {
         int mb, nb;
         walk.coords(t, p, mb, nb);
+        const bool newrb = mb != cur_mb;
+        bool lastrb = true;   // the unit's last tile of this row block: it releases the A panel
+        if (t + walk.step < walk.end) {
+          int mb2, nb2;
+          walk.coords(t + walk.step, p, mb2, nb2);
+          lastrb = mb2 != mb;
+        }
         if constexpr (RES) {
           if (mb != cur_mb) {
             if (*abort_flag || !mbar_wait(sfa_full, nsfa & 1, p.wait_limit)) {
@@ -341,9 +394,16 @@ __global__ void __launch_bounds__(384, 1)
             ok = false;
             break;
           }
+          if constexpr (APANEL) {
+            if (newrb && (*abort_flag || !mbar_wait(&a_full[ks], (nsfa - 1) & 1, p.wait_limit))) {
+              ok = false;
+              break;
+            }
+          }
           tc_fence_after();
           const int nk = min(C::KSTEPS, p.k_atoms - C::KSTEPS * ks);
-          const uint32_t a_base = smem_u32(smem + C::OFF_A + s * C::A_BYTES);
+          const uint32_t a_base = APANEL ? smem_u32(smem + C::OFF_A + ks * C::A_CHUNK)
+                                         : smem_u32(smem + C::OFF_A + s * C::A_BYTES);
           const uint32_t b_base = smem_u32(smem + C::OFF_B + s * C::B_BYTES);
           const uint32_t sfa_base = smem_u32(smem + C::OFF_SFA + s * C::SFA_BYTES);
           const uint32_t sfb_base = smem_u32(smem + C::OFF_SFB + s * C::SFB_BYTES);
@@ -373,6 +433,7 @@ __global__ void __launch_bounds__(384, 1)
               tc_mma_nvf4(d_tmem, adesc, bdesc, C::IDESC, t_sfa, t_sfb + sfb_shift, accum);
           }
           commit_to(&empty[s]);
+          if (APANEL && lastrb) commit_to(&a_empty[ks]);
         }
         if (!ok) break;
         commit_to(&tfull[acc]);
@@ -387,7 +448,7 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
-    const float alpha = __fmul_rn(__fmul_rn(*p.g_a, *p.g_w), p.alpha_mul);
+    const float alpha = __fmul_rn(__fmul_rn(ld_dep(p.g_a), ld_dep(p.g_w)), p.alpha_mul);
     const int quarter = warp & 3;
     const int half = (warp - 4) >> 2;
     uint8_t* stage = smem + C::OFF_C + (warp - 4) * EPI_BUF * kWarpBoxBytes;
@@ -425,11 +486,11 @@ __global__ void __launch_bounds__(384, 1)
 // --------------------------------------------------------------------------
 // Host side
 // --------------------------------------------------------------------------
-template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES, int BKB_ = 128>
+template <int BN, int STAGES, bool PAIR, int ACC_, int EPI_BUF, bool RES, int BKB_ = 128, bool APANEL = false>
 static ql_status launch_w4a4_cfg(const void* a_codes, const uint8_t* a_sf, const float* g_a,
                                  int64_t M, const ql_weights* w, void* Y, cudaStream_t st,
                                  int* status, Gate gate) {
-  using C = W4A4Cfg<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_>;
+  using C = W4A4Cfg<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_, APANEL>;
   const int N = w->N, K = w->K;
   if (RES && K / 64 > kResKSteps) return QL_ERR_UNSUPPORTED_SHAPE;
   CUtensorMap ta, tb, tsa, tsb, ty;
@@ -453,7 +514,7 @@ static ql_status launch_w4a4_cfg(const void* a_codes, const uint8_t* a_sf, const
   p.alpha_mul = w->hadamard ? (1.0f / 128.0f) : 1.0f;
   p.gate = gate.route;
   p.gate_value = gate.value;
-  auto kern = k_gemm_w4a4<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_>;
+  auto kern = k_gemm_w4a4<BN, STAGES, PAIR, ACC_, EPI_BUF, RES, BKB_, APANEL>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int units = std::min(p.num_tiles, num_sms() / C::CTAS);
   if (launch_pdl(kern, dim3(static_cast<unsigned>(units * C::CTAS)), dim3(384), C::SMEM, st, C::CTAS, ta, tb,
@@ -468,20 +529,38 @@ ql_status launch_gemm_w4a4(const void* a_codes, const uint8_t* a_sf, const float
                            const ql_weights* w, void* Y, cudaStream_t st, int* status, Gate gate) {
   if (M == 0) return QL_OK;
   const bool res = w->K / 64 <= kResKSteps;
+  const int64_t N = w->N;
   // 192-wide tiles spend fewer tensor-pipe instructions per output column
   // than 128-wide ones (measured 1.4x on the 5120-column Wan-14B FFN-down);
   // a ragged last tile reads zero weight rows past N (TMA fill, zero scales
   // in the padded scale rows) and stores no column past N.  128-wide tiles
   // remain for N <= 128 and where the last 192-wide tile would waste more
   // than 30% of the columns.
-  const int64_t n192 = (static_cast<int64_t>(w->N) + 191) / 192 * 192;
-  const bool wide = w->N > 128 && 10 * n192 <= 13 * static_cast<int64_t>(w->N);
+  const int64_t n192 = (N + 191) / 192 * 192, n256 = (N + 255) / 256 * 256;
+  const bool wide = N > 128 && 10 * n192 <= 13 * N;
   if (M > 128) {   // CTA pairs on 256-row tiles
-    if (wide) {
-      if (res) return launch_w4a4_cfg<192, 5, true, 2, 3, true>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
-      return launch_w4a4_cfg<192, 5, true, 2, 3, false>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
+    if (res) {
+      // K <= 1920: the activation scales of a row block stay in tensor
+      // memory while the unit walks the row block's N tiles.  With many N
+      // tiles per row block the A tiles stay in shared memory too and only
+      // the weights stream (half the L2 reads; measured 4-5% faster on the
+      // 5760- and 7680-column linears).  With few, each unit reloads the
+      // panel about once per ten tiles and the streamed form is faster.
+      const int64_t tiles_n = wide ? n192 / 192 : (N + 127) / 128;
+      if (tiles_n >= 16) {
+        if (wide)
+          return launch_w4a4_cfg<192, 4, true, 2, 1, true, 128, true>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
+        return launch_w4a4_cfg<128, 5, true, 2, 1, true, 128, true>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
+      }
+      if (wide) return launch_w4a4_cfg<192, 5, true, 2, 3, true>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
+      return launch_w4a4_cfg<128, 6, true, 2, 2, true>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
     }
-    if (res) return launch_w4a4_cfg<128, 6, true, 2, 2, true>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
+    // Longer K: A and its scales stream with B.  256-wide tiles load the
+    // fewest operand bytes per MMA cycle; their single accumulator costs an
+    // epilogue bubble per tile that long K amortizes.
+    if (N > 192 && 10 * n256 <= 13 * N)
+      return launch_w4a4_cfg<256, 5, true, 1, 2, false>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
+    if (wide) return launch_w4a4_cfg<192, 5, true, 2, 3, false>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
     return launch_w4a4_cfg<128, 6, true, 2, 2, false>(a_codes, a_sf, g_a, M, w, Y, st, status, gate);
   }
   if (wide) {
