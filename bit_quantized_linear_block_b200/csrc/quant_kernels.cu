@@ -128,8 +128,11 @@ __device__ __forceinline__ void fwht128_half(float2 (&P)[32]) {
 // lane owns (half_index = 2 * block + (lane & 1)).  `bars` holds kRing
 // mbarriers per warp.  A wait that runs out of its cycle budget records
 // QL_ERR_TIMEOUT, waits (bounded) for the warp's loads still in flight and
-// ends the warp's walk.
-template <int WARPS, class Body>
+// ends the warp's walk.  REVERSE walks each warp's chunks from the last to
+// the first (the grid sweeps the tensor from its end): a pass that follows a
+// front-to-back pass over the same tensor meets the most recently read part,
+// the part most likely still in L2, first.
+template <int WARPS, bool REVERSE = false, class Body>
 __device__ __forceinline__ void stream_blocks(const CUtensorMap* tm, int64_t total_bytes, int hadamard,
                                               uint8_t* ring_all, uint64_t* bars, int* status, Body body) {
   const int wid = threadIdx.x >> 5;
@@ -146,11 +149,12 @@ __device__ __forceinline__ void stream_blocks(const CUtensorMap* tm, int64_t tot
     fence_mbar_init();
   }
   __syncwarp();
-  auto issue = [&](int64_t k) {   // chunk k of this warp into slot k % kRing
+  auto chunk = [&](int64_t k) { return gw + (REVERSE ? (mine - 1 - k) : k) * nw; };   // k-th chunk walked
+  auto issue = [&](int64_t k) {   // chunk k of this warp's walk into slot k % kRing
     if (leader) {
       const int slot = static_cast<int>(k % kRing);
       mbar_arrive_expect_tx(&bar[slot], kChunkBytes);
-      tma_load_2d(ring_g + slot * kChunkBytes, tm, &bar[slot], 0, static_cast<int32_t>((gw + k * nw) * 32));
+      tma_load_2d(ring_g + slot * kChunkBytes, tm, &bar[slot], 0, static_cast<int32_t>(chunk(k) * 32));
     }
   };
   for (int64_t i = 0; i < kRing - 1 && i < mine; ++i) issue(i);
@@ -167,7 +171,7 @@ __device__ __forceinline__ void stream_blocks(const CUtensorMap* tm, int64_t tot
     read_half(ring_g + slot * kChunkBytes, P);
     __syncwarp();
     if (hadamard) fwht128_half(P);
-    body(P, (gw + k * nw) * 32 + lane_id());
+    body(P, chunk(k) * 32 + lane_id());
   }
   if (k < mine && leader) {   // timed out: let the loads in flight land before the CTA may exit
     record_error(status, QL_ERR_TIMEOUT);
@@ -353,7 +357,7 @@ __device__ __forceinline__ void nvfp4_half(const float2 (&P)[32], const Nvfp4Sca
 template <bool DECOMP>
 __global__ void __launch_bounds__(kQuantThreads, 1)
     k_quant_nvfp4(const __grid_constant__ CUtensorMap tm_x, int64_t M, int32_t K, int hadamard,
-                  const float* __restrict__ amax_in, uint8_t* __restrict__ codes,
+                  const float* amax_in, uint8_t* __restrict__ codes,
                   uint8_t* __restrict__ sf_mma, uint8_t* __restrict__ sf_rm,
                   float* __restrict__ g_out, int* status, const int32_t* gate, int32_t gate_value) {
   extern __shared__ uint8_t ring_raw[];
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
     pdl_release();
     return;
   }
-  const float amax_t = __ldg(amax_in);
+  const float amax_t = ld_dep(amax_in);
   const float g = (amax_t == 0.f) ? 1.f : __fdiv_rn(amax_t, 2688.f);
   if (blockIdx.x == 0 && threadIdx.x == 0 && g_out != nullptr) *g_out = g;
   const Nvfp4ScaleDiv sd(__fmul_rn(6.f, g));
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
   const int64_t row_bytes = kq >> 1;
   const int64_t units = M * upr;
   const int64_t halves = 2 * units;
-  stream_blocks<kQuantWarps>(&tm_x, M * K * 2, hadamard, ring_all, bars, status, [&](float2 (&P)[32], int64_t hu) {
+  stream_blocks<kQuantWarps, true>(&tm_x, M * K * 2, hadamard, ring_all, bars, status, [&](float2 (&P)[32], int64_t hu) {
     if (hu >= halves) return;
     // half index -> (row, first scale index, first code byte); 32-bit division (units < 2^32)
     const uint32_t u = static_cast<uint32_t>(hu >> 1);
@@ -443,18 +447,31 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
 // ---------------------------------------------------------------------------
 // F16 = true writes each code as the equal f16 value (an integer in
 // [-127, 127], exact), the operand layout of the f16 MMA.
+//
+// No clamp is needed: with inv = RN(qmax / amax) and |h| <= amax,
+// |RN(h * inv)| <= qmax (1 + 2^-24)^2 < qmax + 1/2, so the rounded code
+// never leaves [-qmax, qmax].  The int8 path keeps each code's low byte
+// (two's complement) and packs four with byte permutes; the f16 path
+// rounds in fp32 (rint), turns -0 into +0 (the code 0 is stored as +0) and
+// converts two codes per instruction.
+__device__ __forceinline__ uint32_t pack4_s8(int a0, int a1, int a2, int a3) {
+  const uint32_t t01 = __byte_perm(static_cast<uint32_t>(a0), static_cast<uint32_t>(a1), 0x0040);
+  const uint32_t t23 = __byte_perm(static_cast<uint32_t>(a2), static_cast<uint32_t>(a3), 0x0040);
+  return __byte_perm(t01, t23, 0x5410);
+}
+
 template <bool F16>
-__device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv, int qmax, uint8_t* dst) {
+__device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv, uint8_t* dst) {
   if constexpr (F16) {
-    uint32_t w[32];   // element pairs (4i+b) and (32+4i+b) -> f16 words
+    uint32_t w[32];   // element pairs (2i, 2i+1) and (32+2i, 32+2i+1) -> f16 words
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
-      const int ql0 = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[2 * i].x, inv))));
-      const int ql1 = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[2 * i + 1].x, inv))));
-      const int qh0 = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[2 * i].y, inv))));
-      const int qh1 = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[2 * i + 1].y, inv))));
-      const __half2 lo = __halves2half2(__int2half_rn(ql0), __int2half_rn(ql1));
-      const __half2 hi = __halves2half2(__int2half_rn(qh0), __int2half_rn(qh1));
+      const float2 a = __fmul2_rn(P[2 * i], make_float2(inv, inv));       // (x_2i, x_32+2i)
+      const float2 c = __fmul2_rn(P[2 * i + 1], make_float2(inv, inv));   // (x_2i+1, x_32+2i+1)
+      const float l0 = __fadd_rn(rintf(a.x), 0.f), l1 = __fadd_rn(rintf(c.x), 0.f);
+      const float h0 = __fadd_rn(rintf(a.y), 0.f), h1 = __fadd_rn(rintf(c.y), 0.f);
+      const __half2 lo = __floats2half2_rn(l0, l1);
+      const __half2 hi = __floats2half2_rn(h0, h1);
       w[i] = *reinterpret_cast<const uint32_t*>(&lo);          // elements 2i, 2i+1
       w[16 + i] = *reinterpret_cast<const uint32_t*>(&hi);     // elements 32+2i, 32+2i+1
     }
@@ -463,18 +480,13 @@ __device__ __forceinline__ void quant_int8_half(const float2 (&P)[32], float inv
     for (int i = 0; i < 8; ++i) d[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
   } else {
     uint32_t w[16];
+    const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {   // elements 4i..4i+3 (.x halves) and 32+4i.. (.y halves)
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int ql = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[4 * i + b].x, inv))));
-        const int qh = max(-qmax, min(qmax, __float2int_rn(__fmul_rn(P[4 * i + b].y, inv))));
-        lo |= (static_cast<uint32_t>(ql) & 0xFFu) << (8 * b);
-        hi |= (static_cast<uint32_t>(qh) & 0xFFu) << (8 * b);
-      }
-      w[i] = lo;
-      w[8 + i] = hi;
+      const float2 y0 = __fmul2_rn(P[4 * i], inv2), y1 = __fmul2_rn(P[4 * i + 1], inv2);
+      const float2 y2 = __fmul2_rn(P[4 * i + 2], inv2), y3 = __fmul2_rn(P[4 * i + 3], inv2);
+      w[i] = pack4_s8(__float2int_rn(y0.x), __float2int_rn(y1.x), __float2int_rn(y2.x), __float2int_rn(y3.x));
+      w[8 + i] = pack4_s8(__float2int_rn(y0.y), __float2int_rn(y1.y), __float2int_rn(y2.y), __float2int_rn(y3.y));
     }
     uint4* d = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -499,7 +511,8 @@ __global__ void __launch_bounds__(kThreadsHbm)
   const int wid = threadIdx.x >> 5;
   const int32_t halves = K >> 6;                 // 64-element half blocks (128-byte rows) per token row
   const int32_t passes = (halves + 31) >> 5;
-  uint8_t* rows[2] = {s_rows + (2 * wid) * buf_bytes, s_rows + (2 * wid + 1) * buf_bytes};
+  uint8_t* const rows0 = s_rows + (2 * wid) * buf_bytes;   // the warp's two row buffers
+  auto rows = [&](int b) { return rows0 + b * buf_bytes; };
   uint64_t* bar = bars + 2 * wid;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + wid;
   const int64_t nw = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
@@ -513,7 +526,7 @@ __global__ void __launch_bounds__(kThreadsHbm)
     if (lane == 0) {
       mbar_arrive_expect_tx(&bar[b], static_cast<uint32_t>(halves) * kLaneBytes);
       for (int32_t y = 0; y < halves; y += box_rows)
-        tma_load_2d(rows[b] + y * kLaneBytes, &tm_x, &bar[b], 0, static_cast<int32_t>(r * halves + y));
+        tma_load_2d(rows(b) + y * kLaneBytes, &tm_x, &bar[b], 0, static_cast<int32_t>(r * halves + y));
     }
   };
   auto load_half = [&](const uint8_t* row, int p, float2 (&P)[32]) {
@@ -533,7 +546,7 @@ __global__ void __launch_bounds__(kThreadsHbm)
     if (r + nw < M) issue_row(r + nw, (k + 1) & 1);
     ok = __all_sync(0xffffffffu, mbar_wait(&bar[k & 1], static_cast<uint32_t>((k >> 1) & 1), kDrainLimit));
     if (!ok) break;
-    const uint8_t* row = rows[k & 1];
+    const uint8_t* row = rows(k & 1);
     float2 P[32];
     float m = 0.f;
     for (int p = 0; p < passes; ++p) {
@@ -551,7 +564,7 @@ __global__ void __launch_bounds__(kThreadsHbm)
     for (int p = 0; p < passes; ++p) {
       if (passes > 1) load_half(row, p, P);    // one pass: P still holds the rotated half
       const int32_t hb = 32 * p + static_cast<int32_t>(lane);
-      if (hb < halves) quant_int8_half<F16>(P, inv, qmax, crow + 64 * kElemBytes * hb);
+      if (hb < halves) quant_int8_half<F16>(P, inv, crow + 64 * kElemBytes * hb);
     }
     __syncwarp();
   }
@@ -569,71 +582,94 @@ __global__ void __launch_bounds__(kThreadsHbm)
 // Per-tensor INT8 in Q-ARVD channel order.  Output row = Kp bytes; slot j
 // takes input channel gather[j] (or 0 for a padding slot).  The scale comes
 // from the device amax of the un-rotated tensor.
-// One CTA per row at a time: the bf16 row is copied into shared memory with
-// coalesced 16-byte cp.async (the next row's copy is in flight while this
-// one is quantized); each thread takes 4 consecutive slots per step, reads
-// their channels through the gather table (int16 in shared memory) and
-// writes 4 codes as one word of a shared output row, which leaves with
-// 16-byte stores.
+// One CTA per row at a time, kPermRing rows in flight: each bf16 row comes
+// into one of kPermRing shared-memory buffers by one bulk copy (tracked by
+// the buffer's mbarrier), issued kPermRing rows ahead.  Each row buffer ends
+// with 16 zero bytes, and the gather table (int16 in shared memory) sends
+// padding slots to that zero element, so every slot is one table read, one
+// row read and no branch.  Each thread takes 4 consecutive slots per step
+// and writes 4 codes as one word of a shared output row, which leaves with
+// 16-byte stores.  As in the per-token quantizer the codes need no clamp
+// (|RN(x * RN(qmax / amax))| < qmax + 1/2).
 // ---------------------------------------------------------------------------
-struct PermLayout {
-  int32_t gather_bytes, row_bytes, out_bytes, total;
+constexpr int kPermRing = 4;
+struct PermLayout {   // row buffers: the bf16 row (K * 2 bytes) and 16 zero bytes
+  int32_t gather_bytes, row_bytes, buf_bytes, out_bytes, total;
   __host__ __device__ PermLayout(int32_t K, int32_t Kp)
-      : gather_bytes((Kp * 2 + 15) / 16 * 16), row_bytes(K * 2), out_bytes((Kp + 15) / 16 * 16),
-        total((Kp * 2 + 15) / 16 * 16 + 2 * K * 2 + (Kp + 15) / 16 * 16) {}
+      : gather_bytes((Kp * 2 + 15) / 16 * 16), row_bytes(K * 2), buf_bytes(K * 2 + 16),
+        out_bytes((Kp + 15) / 16 * 16),
+        total((Kp * 2 + 15) / 16 * 16 + kPermRing * (K * 2 + 16) + (Kp + 15) / 16 * 16) {}
 };
-constexpr int kPermThreads = 256;
+constexpr int kPermThreads = 512;
 
 __global__ void __launch_bounds__(kPermThreads)
     k_quant_int8_tensor_perm(const uint8_t* __restrict__ x, int64_t M, int32_t K, int32_t Kp,
-                             const int32_t* __restrict__ gather, const float* __restrict__ amax_in, int qmax,
-                             int8_t* __restrict__ codes, float* __restrict__ scale_out) {
+                             const int32_t* __restrict__ gather, const float* amax_in, int qmax,
+                             int8_t* __restrict__ codes, float* __restrict__ scale_out, int* status) {
   extern __shared__ __align__(16) uint8_t s_perm[];
-  pdl_wait();
+  __shared__ uint64_t full[kPermRing];
+  __shared__ int s_ok;
   const PermLayout L(K, Kp);
   int16_t* s_gather = reinterpret_cast<int16_t*>(s_perm);
-  uint8_t* rows[2] = {s_perm + L.gather_bytes, s_perm + L.gather_bytes + L.row_bytes};
-  uint32_t* orow = reinterpret_cast<uint32_t*>(s_perm + L.gather_bytes + 2 * L.row_bytes);
-  for (int i = threadIdx.x; i < Kp; i += blockDim.x) s_gather[i] = static_cast<int16_t>(gather[i]);
-  const float amax = __ldg(amax_in);
+  uint8_t* rows = s_perm + L.gather_bytes;
+  uint32_t* orow = reinterpret_cast<uint32_t*>(s_perm + L.gather_bytes + kPermRing * L.buf_bytes);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kPermRing; ++i) mbar_init(&full[i], 1);
+    fence_mbar_init();
+    s_ok = 1;
+  }
+  __syncthreads();
+  if (threadIdx.x < kPermRing)   // the zero element after each row buffer
+    *reinterpret_cast<uint4*>(rows + threadIdx.x * L.buf_bytes + L.row_bytes) = make_uint4(0, 0, 0, 0);
+  pdl_wait();
+  for (int i = threadIdx.x; i < Kp; i += blockDim.x) {   // padding slots (-1) read the zero element
+    const int32_t g = gather[i];
+    s_gather[i] = static_cast<int16_t>(g < 0 ? K : g);
+  }
+  const float amax = ld_dep(amax_in);
   const float fq = static_cast<float>(qmax);
   const float inv = (amax == 0.f) ? 0.f : __fdiv_rn(fq, amax);
   if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = (amax == 0.f) ? 0.f : __fdiv_rn(amax, fq);
-  auto issue_row = [&](int64_t r, uint8_t* dst) {
-    const uint8_t* src = x + r * L.row_bytes;
-    const uint32_t d = smem_u32(dst);
-    for (int32_t o = 16 * static_cast<int32_t>(threadIdx.x); o < L.row_bytes; o += 16 * kPermThreads) {
-      const bool ok = r < M;
-      cp_async16(d + o, ok ? static_cast<const void*>(src + o) : static_cast<const void*>(x), ok ? 16u : 0u);
-    }
+  auto issue_row = [&](int64_t r, int slot) {   // thread 0 only
+    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(L.row_bytes));
+    bulk_load(rows + slot * L.buf_bytes, x + r * L.row_bytes, static_cast<uint32_t>(L.row_bytes), &full[slot]);
   };
-  auto q8 = [&](const unsigned short* xr, int32_t src) -> uint32_t {
-    if (src < 0) return 0u;
-    const float v = __uint_as_float(static_cast<uint32_t>(xr[src]) << 16);
-    return static_cast<uint32_t>(max(-qmax, min(qmax, __float2int_rn(__fmul_rn(v, inv))))) & 0xFFu;
-  };
-  issue_row(blockIdx.x, rows[0]);
-  cp_async_commit();
+  const float2 inv2 = make_float2(inv, inv);
+  const int64_t first = blockIdx.x, step = gridDim.x;
+  if (threadIdx.x == 0)
+    for (int i = 0; i < kPermRing && first + i * step < M; ++i) issue_row(first + i * step, i);
   int k = 0;
-  for (int64_t r = blockIdx.x; r < M; r += gridDim.x, ++k) {
-    issue_row(r + gridDim.x, rows[(k + 1) & 1]);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();   // this row landed (all threads' copies); gather table ready
-    const unsigned short* xr = reinterpret_cast<const unsigned short*>(rows[k & 1]);
+  for (int64_t r = first; r < M; r += step, ++k) {
+    const int slot = k % kPermRing;
+    if (threadIdx.x == 0) s_ok = (mbar_wait(&full[slot], static_cast<uint32_t>((k / kPermRing) & 1), kDrainLimit)) ? 1 : 0;
+    __syncthreads();   // this row landed; gather table ready; the previous output row was stored
+    if (!s_ok) break;
+    const unsigned short* xr = reinterpret_cast<const unsigned short*>(rows + slot * L.buf_bytes);
     for (int32_t w = threadIdx.x; 4 * w < Kp; w += kPermThreads) {
-      const uint2 gi = *reinterpret_cast<const uint2*>(s_gather + 4 * w);   // 4 int16 indices
-      const int32_t g0 = static_cast<int16_t>(gi.x & 0xFFFFu), g1 = static_cast<int16_t>(gi.x >> 16);
-      const int32_t g2 = static_cast<int16_t>(gi.y & 0xFFFFu), g3 = static_cast<int16_t>(gi.y >> 16);
-      orow[w] = q8(xr, g0) | (q8(xr, g1) << 8) | (q8(xr, g2) << 16) | (q8(xr, g3) << 24);
+      const uint2 gi = *reinterpret_cast<const uint2*>(s_gather + 4 * w);   // 4 channel indices
+      const float2 v01 = make_float2(__uint_as_float(static_cast<uint32_t>(xr[gi.x & 0xFFFFu]) << 16),
+                                     __uint_as_float(static_cast<uint32_t>(xr[gi.x >> 16]) << 16));
+      const float2 v23 = make_float2(__uint_as_float(static_cast<uint32_t>(xr[gi.y & 0xFFFFu]) << 16),
+                                     __uint_as_float(static_cast<uint32_t>(xr[gi.y >> 16]) << 16));
+      const float2 y01 = __fmul2_rn(v01, inv2), y23 = __fmul2_rn(v23, inv2);
+      orow[w] = pack4_s8(__float2int_rn(y01.x), __float2int_rn(y01.y), __float2int_rn(y23.x), __float2int_rn(y23.y));
     }
     __syncthreads();   // output row complete; the row buffer may be refilled
+    if (threadIdx.x == 0 && r + kPermRing * step < M) issue_row(r + kPermRing * step, slot);
     int8_t* dst = codes + r * Kp;
     for (int32_t o = 16 * static_cast<int32_t>(threadIdx.x); o < Kp; o += 16 * kPermThreads)
       *reinterpret_cast<uint4*>(dst + o) = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(orow) + o);
   }
   pdl_release();
-  cp_async_wait<0>();
+  if (threadIdx.x == 0) {
+    // every copy issued has landed before the CTA may exit (only a timed-out
+    // wait leaves copies in flight: wait for them with a bounded budget)
+    int64_t r = first + static_cast<int64_t>(k) * step;
+    if (!s_ok) record_error(status, QL_ERR_TIMEOUT);
+    for (int i = 0; i < kPermRing && r < M; ++i, r += step)
+      if (!s_ok || i > 0) (void)mbar_wait(&full[(k + i) % kPermRing], static_cast<uint32_t>(((k + i) / kPermRing) & 1), kDrainLimit);
+  }
+  __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -785,12 +821,19 @@ ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int
                                         float* scale_out, cudaStream_t st, int qmax) {
   const PermLayout L(K, Kp);
   if (L.total > 200 * 1024) return QL_ERR_UNSUPPORTED_SHAPE;
-  const int per_sm = std::max(1, std::min(4, (220 * 1024) / L.total));
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(M, static_cast<int64_t>(per_sm) * num_sms())));
   if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_int8_tensor_perm), L.total)) return QL_ERR_CUDA;
+  // as many CTAs as can be resident at once: each walks rows blockIdx.x,
+  // blockIdx.x + gridDim.x, ..., so a CTA that waited for a free SM would
+  // start its rows late
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_int8_tensor_perm, kPermThreads, L.total) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return QL_ERR_CUDA;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(M, static_cast<int64_t>(per_sm) * num_sms())));
   if (launch_pdl(k_quant_int8_tensor_perm, dim3(grid), dim3(kPermThreads), L.total, st, 1,
                  static_cast<const uint8_t*>(x), M, K, Kp, gather, amax_in, qmax, static_cast<int8_t*>(codes),
-                 scale_out) != cudaSuccess) {
+                 scale_out, status_word()) != cudaSuccess) {
     (void)cudaGetLastError();
     return QL_ERR_CUDA;
   }
