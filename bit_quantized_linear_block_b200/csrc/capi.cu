@@ -566,7 +566,6 @@ ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* a_sf, c
   }
   if (act_fmt == QL_ROUTE_NVFP4 || act_fmt == QL_ROUTE_INT8 || act_fmt == QL_ACT_INT8_F16) {
     if (w->fmt != QL_W_NVFP4) return QL_ERR_INVALID_ARG;
-    if (act_fmt == QL_ACT_INT8_F16 && w->w16 == nullptr) return QL_ERR_INVALID_ARG;
     if (act_fmt == QL_ROUTE_NVFP4 && M > 0 && a_sf == nullptr) return QL_ERR_INVALID_ARG;
   } else if (act_fmt == QL_ACT_INT8_TENSOR) {
     if (w->fmt != QL_W_QARVD_INT4) return QL_ERR_INVALID_ARG;
@@ -602,7 +601,7 @@ size_t qlinear_forward_ws_bytes(int64_t M, const ql_weights* w, int32_t route) {
   if (route == QL_ROUTE_BF16) return w->wbf16 != nullptr ? 256 : 0;
   route = int_base_fmt(route);
   if (route != QL_ROUTE_NVFP4 && route != QL_ROUTE_INT8) return 0;
-  return forward_act_bytes(M, w->K, 0, route, w->w16 != nullptr);
+  return forward_act_bytes(M, w->K, 0, route, true);
 }
 
 ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t route, void* Y,
@@ -650,13 +649,12 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
     return launch_gemm_w4a4(codes, sf, g, M, &w2, Y, st, status);
   }
   if (fmt == QL_ROUTE_INT8) {
-    // with an f16 weight copy the codes are written as f16 values and both
-    // GEMM operands go straight from TMA to the MMA
-    const int f16 = w->w16 != nullptr ? 1 : 0;
-    uint8_t* codes = c.take<uint8_t>(static_cast<size_t>(M) * K * (f16 ? 2 : 1));
+    // codes as f16 values: the f16 MMA's operand type (weights from their f16
+    // copy, or widened into tensor memory without one)
+    uint8_t* codes = c.take<uint8_t>(static_cast<size_t>(M) * K * 2);
     float* s = c.take<float>(4 * static_cast<size_t>(M));
-    QL_TRY(launch_quant_int8_token(X, M, K, w->hadamard, codes, s, st, f16, qmax));
-    return launch_gemm_w4a8(codes, s, M, w, Y, st, status, f16);
+    QL_TRY(launch_quant_int8_token(X, M, K, w->hadamard, codes, s, st, 1, qmax));
+    return launch_gemm_w4a8(codes, s, M, w, Y, st, status, 1);
   }
   void* aws = c.take<uint8_t>(kAmaxWsBytes);
   float* amax = c.take<float>(256);
@@ -671,7 +669,7 @@ ql_status qlinear_forward(const void* X, int64_t M, const ql_weights* w, int32_t
 size_t qlinear_forward_routed_ws_bytes(int64_t M, const ql_weights* w) {
   if (M < 0 || check_w(w) != QL_OK || w->fmt != QL_W_NVFP4) return 0;
   return forward_act_bytes(M, w->K, 0, QL_ROUTE_NVFP4) +
-         forward_act_bytes(M, w->K, 0, QL_ROUTE_INT8, w->w16 != nullptr);
+         forward_act_bytes(M, w->K, 0, QL_ROUTE_INT8, true);
 }
 
 ql_status qlinear_forward_routed(const void* X, int64_t M, const ql_weights* w, const int32_t* route_dev, void* Y,
@@ -701,11 +699,10 @@ ql_status qlinear_forward_routed(const void* X, int64_t M, const ql_weights* w, 
   QL_TRY(launch_quant_nvfp4(X, M, K, w->hadamard, amax, codes4, sf, nullptr, g, st, 0, g_fp4));
   QL_TRY(launch_gemm_w4a4(codes4, sf, g, M, w, Y, st, status, g_fp4));
   // INT8 route
-  const int f16 = w->w16 != nullptr ? 1 : 0;
-  uint8_t* codes8 = c.take<uint8_t>(static_cast<size_t>(M) * K * (f16 ? 2 : 1));
+  uint8_t* codes8 = c.take<uint8_t>(static_cast<size_t>(M) * K * 2);
   float* s8 = c.take<float>(4 * static_cast<size_t>(M));
-  QL_TRY(launch_quant_int8_token(X, M, K, w->hadamard, codes8, s8, st, f16, 127, g_int8));
-  QL_TRY(launch_gemm_w4a8(codes8, s8, M, w, Y, st, status, f16, g_int8));
+  QL_TRY(launch_quant_int8_token(X, M, K, w->hadamard, codes8, s8, st, 1, 127, g_int8));
+  QL_TRY(launch_gemm_w4a8(codes8, s8, M, w, Y, st, status, 1, g_int8));
   // BF16 (PDR's refresh) when the weights were kept
   if (w->wbf16 != nullptr) QL_TRY(launch_gemm_bf16(X, M, w, Y, st, status, g_bf16));
   return QL_OK;

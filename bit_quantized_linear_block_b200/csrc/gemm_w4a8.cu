@@ -346,12 +346,329 @@ static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int
   return QL_OK;
 }
 
+// ---------------------------------------------------------------------------
+// INT8 route without the f16 weight copy: the weights are the MMA's A operand
+// in tensor memory, so the on-chip widening never passes through shared
+// memory.  The kernel computes the transposed tile D[n, m] = sum_k
+// W[n, k] q[m, k] (128 weight rows on the TMEM lanes, BMT tokens as the MMA's
+// N) and writes Y[m, n] = bf16(RN(RN(g_w * alpha_mul) * s_m) * D[n, m]), the
+// rounding of the other forms.
+//
+// Persistent, one CTA (512 or 640 threads) per SM, tiles of 128 weight rows x BMT
+// tokens, weight tiles fastest (the CTAs running at once share a few token
+// tiles and sweep the whole weight matrix, which stays in L2):
+//   warp 0      TMA producer: the f16-coded activation tile (BMT x 64,
+//               128-byte swizzle), the FP4 weight tile (128 rows x 32 bytes)
+//               and its 512-byte scale column, into an RS-deep ring;
+//   warp 1      TMEM allocator and MMA issuer (kind::f16, 128 x BMT x 16,
+//               A from tensor memory);
+//   XW transform warps (4 or 8, from warp 4): lane l of warp w owns weight
+//               row 32 (w % 4) + l and 64 / (XW / 4) of the stage's 64 K
+//               elements; it widens the row's FP4 codes times their E4M3
+//               scales to f16 (hardware e2m1x2 -> f16x2 convert, f16
+//               multiply: exact) and writes the words into one of AS
+//               32-column A slots of its TMEM lane with tcgen05.st;
+//   8 epilogue warps (after the transform warps): warp w reads TMEM lane
+//               quarter w % 4 and half of the BMT columns, scales column m
+//               by s_m, and stores 32 x 32 boxes of Y (tokens x weight rows)
+//               through its own staging buffers with TMA.
+// Tensor memory: two BMT-column accumulators (one for BMT = 256) and
+// AS = (512 - NACC BMT) / 32 A slots.  All waits are bounded (the W4A4 kernel's timeout protocol).
+// ---------------------------------------------------------------------------
+template <int BMT, int RS, int XW>
+struct W4A8TsCfg {
+  static constexpr int BK = 64;                    // K elements per stage
+  // two accumulators where they leave room for four A slots, else one
+  static constexpr int NACC = (2 * BMT + 4 * 32 <= 512) ? 2 : 1;
+  static constexpr int AS = (512 - NACC * BMT) / 32;  // A slots (64 f16 of K per TMEM lane)
+  static constexpr int B_BYTES = BMT * BK * 2;     // f16 activation codes, 128-byte rows
+  static constexpr int W_BYTES = 128 * BK / 2;     // FP4 codes, 32 bytes per weight row
+  static constexpr int SF_BYTES = 512;             // the stage's column of the 128-row scale atom
+  static constexpr int OFF_B = 0;
+  static constexpr int OFF_W = OFF_B + RS * B_BYTES;
+  static constexpr int OFF_SF = OFF_W + RS * W_BYTES;
+  static constexpr int OFF_C = OFF_SF + RS * SF_BYTES;     // 8 epilogue warps x 2 staging boxes
+  static constexpr int OFF_BAR = OFF_C + 8 * 2 * kWarpBoxBytes;
+  static constexpr int NBAR = 2 * RS + 2 * AS + 2 * 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static constexpr int EPI0 = 4 + XW;              // first epilogue warp
+  static constexpr int THREADS = (EPI0 + 8) * 32;
+  static constexpr int KPT = 64 / (XW / 4);         // K elements per transform thread and stage
+  static constexpr int EPI_CH = BMT / 2 / 32;      // 32-column boxes per epilogue warp and tile
+  static_assert(XW == 4 || XW == 8, "transform warps");
+  static_assert(AS >= 2, "tensor memory budget");
+  static_assert(B_BYTES % 1024 == 0 && BMT % 64 == 0, "swizzled tiles, whole epilogue boxes");
+  static_assert(SMEM <= 232448, "shared memory budget");
+  // kind::f16: D = F32 (bit 4), A = B = F16, both K-major, N = BMT, M = 128
+  static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BMT >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+};
+
+template <int BMT, int RS, int XW>
+__global__ void __launch_bounds__(W4A8TsCfg<BMT, RS, XW>::THREADS, 1)
+    k_gemm_w4a8_ts(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                   const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
+  using C = W4A8TsCfg<BMT, RS, XW>;
+  if (p.gate != nullptr) {   // device-routed forward
+    pdl_wait();
+    if (gated_off(p.gate, p.gate_value)) {
+      pdl_release();
+      return;
+    }
+  }
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* raw_empty = raw_full + RS;
+  uint64_t* xf_full = raw_empty + RS;
+  uint64_t* xf_empty = xf_full + C::AS;
+  uint64_t* tfull = xf_empty + C::AS;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = lane_id();
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_y);
+    for (int i = 0; i < RS; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], 1);   // the stage's MMA commit (issued after the transform read it)
+    }
+    for (int i = 0; i < C::AS; ++i) {
+      mbar_init(&xf_full[i], XW);    // the transform warps
+      mbar_init(&xf_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);      // the eight epilogue warps
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t a_slots = tmem + C::NACC * BMT;
+  pdl_wait();   // everything above touched only shared and tensor memory
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (elect_one()) {
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        const int mb = t / p.tiles_n, nb = t - (t / p.tiles_n) * p.tiles_n;
+        for (int ks = 0; ks < p.num_kst; ++ks, ++it) {
+          const int s = it % RS;
+          if (*abort_flag || !mbar_wait(&raw_empty[s], ((it / RS) & 1) ^ 1, p.wait_limit)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&raw_full[s], C::B_BYTES + C::W_BYTES + C::SF_BYTES);
+          tma_load_2d(smem + C::OFF_B + s * C::B_BYTES, &tm_x, &raw_full[s], ks * C::BK, mb * BMT);
+          tma_load_2d(smem + C::OFF_W + s * C::W_BYTES, &tm_w, &raw_full[s], ks * (C::BK / 2), nb * 128);
+          bulk_load(smem + C::OFF_SF + s * C::SF_BYTES, p.sfb + (static_cast<size_t>(nb) * p.k_atoms + ks) * 512,
+                    C::SF_BYTES, &raw_full[s]);
+        }
+      }
+      if (!ok) fail_timeout(p.status, abort_flag);
+      drain_loads(raw_full, it, RS, p.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
+        const int acc = local % C::NACC;
+        if (*abort_flag || !mbar_wait(&tempty[acc], ((local / C::NACC) & 1) ^ 1, p.wait_limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + acc * BMT;
+        for (int ks = 0; ks < p.num_kst; ++ks, ++it) {
+          const int rs = it % RS, sl = it % C::AS;
+          if (*abort_flag || !mbar_wait(&raw_full[rs], (it / RS) & 1, p.wait_limit) ||
+              !mbar_wait(&xf_full[sl], (it / C::AS) & 1, p.wait_limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b_base = smem_u32(smem + C::OFF_B + rs * C::B_BYTES);
+#pragma unroll
+          for (int i = 0; i < C::BK / 16; ++i)
+            tc_mma_f16_ts(d_tmem, a_slots + 32 * sl + 8 * i, smem_desc(b_base + 32 * i, 0, 1024, kSwizzle128B),
+                          C::IDESC, (ks > 0 || i > 0) ? 1u : 0u);
+          tc_commit(&raw_empty[rs]);
+          tc_commit(&xf_empty[sl]);
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+      }
+      if (!ok) fail_timeout(p.status, abort_flag);
+      drain_mma(drain, p.status);
+    }
+  } else if (warp >= 4 && warp < C::EPI0) {
+    // ------------------------------------------------------------ transform
+    const uint32_t q = static_cast<uint32_t>(warp & 3);
+    const uint32_t row = 32 * q + lane;   // weight row within the tile = TMEM lane
+    const uint32_t kh = static_cast<uint32_t>(warp - 4) >> 2;   // this warp's share of the stage's K
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      for (int ks = 0; ks < p.num_kst; ++ks, ++it) {
+        const int rs = it % RS, sl = it % C::AS;
+        if (!warp_wait2(&raw_full[rs], (it / RS) & 1, &xf_empty[sl], ((it / C::AS) & 1) ^ 1, p.wait_limit,
+                        abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // scale atom: byte (row % 32) * 16 + (row / 32) * 4 + k16 holds the block scale of K block k16
+        const uint32_t sb4 = *reinterpret_cast<const uint32_t*>(smem + C::OFF_SF + rs * C::SF_BYTES + lane * 16 + q * 4);
+        const uint4* wr = reinterpret_cast<const uint4*>(smem + C::OFF_W + rs * C::W_BYTES + row * 32 + kh * (C::KPT / 2));
+        const uint32_t col = a_slots + ((32 * q) << 16) + 32 * sl + kh * (C::KPT / 2);
+        if constexpr (XW == 4) {
+          const uint4 c0 = wr[0], c1 = wr[1];
+          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          uint32_t v[32];
+#pragma unroll
+          for (int w8 = 0; w8 < 8; ++w8) {   // codes 8 w8 .. 8 w8 + 7: half of block w8 / 2
+            const uint4 o = fp4x8_scaled_to_f16(cw[w8], (sb4 >> (8 * (w8 >> 1))) & 0xFFu);
+            v[4 * w8] = o.x;
+            v[4 * w8 + 1] = o.y;
+            v[4 * w8 + 2] = o.z;
+            v[4 * w8 + 3] = o.w;
+          }
+          tmem_st32(col, v);
+        } else {   // K elements 32 kh .. 32 kh + 31: blocks 2 kh, 2 kh + 1
+          const uint4 c0 = wr[0];
+          const uint32_t cw[4] = {c0.x, c0.y, c0.z, c0.w};
+          uint32_t v[16];
+#pragma unroll
+          for (int w8 = 0; w8 < 4; ++w8) {
+            const uint4 o = fp4x8_scaled_to_f16(cw[w8], (sb4 >> (8 * (2 * kh + (w8 >> 1)))) & 0xFFu);
+            v[4 * w8] = o.x;
+            v[4 * w8 + 1] = o.y;
+            v[4 * w8 + 2] = o.z;
+            v[4 * w8 + 3] = o.w;
+          }
+          tmem_st16(col, v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xf_full[sl]);
+      }
+    }
+    if (!ok && lane == 0) fail_timeout(p.status, abort_flag);
+  } else if (warp >= C::EPI0) {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t q = static_cast<uint32_t>(warp & 3);
+    const int half = (warp - C::EPI0) >> 2;
+    const float alpha = __fmul_rn(ld_dep(p.g_w), p.alpha_mul);
+    uint8_t* stage = smem + C::OFF_C + (warp - C::EPI0) * 2 * kWarpBoxBytes;
+    int next = 0, local = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+      const int mb = t / p.tiles_n, nb = t - (t / p.tiles_n) * p.tiles_n;
+      const int acc = local % C::NACC;
+      if (!warp_wait_uniform(&tfull[acc], (local / C::NACC) & 1, p.wait_limit, abort_flag, p.status)) break;
+      tc_fence_after();
+      const int n0 = nb * 128 + 32 * static_cast<int>(q);   // this warp's weight rows = output columns
+#pragma unroll 1
+      for (int c = 0; c < C::EPI_CH; ++c) {
+        const int col = half * (BMT / 2) + 32 * c;          // accumulator column = token offset
+        const int m0 = mb * BMT + col;
+        uint32_t r[32];
+        tmem_ld32(tmem + ((32 * q) << 16) + acc * BMT + col, r);
+        tmem_ld_wait();
+        if (c == C::EPI_CH - 1) {   // the whole accumulator share is read: free it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
+        }
+        if (m0 >= p.M || n0 >= p.N) continue;   // warp-uniform: the box is outside Y
+        const int m = m0 + static_cast<int>(lane);
+        const float a_l = (m < p.M) ? __fmul_rn(alpha, ld_dep(p.row_scale + m)) : 0.f;
+        uint8_t* buf = stage + next * kWarpBoxBytes;
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        // box row j = token m0 + j, column = this lane's weight row
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(buf) + lane;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          dst[32 * j] = __float2bfloat16_rn(__fmul_rn(__shfl_sync(0xffffffffu, a_l, j), __uint_as_float(r[j])));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, buf, n0, m0);
+          bulk_commit();
+        }
+        next ^= 1;
+      }
+    }
+    epilogue_warp_finish();
+  }
+
+  pdl_release();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int BMT, int RS, int XW>
+static ql_status launch_w4a8_ts_cfg(const void* a_codes, const float* a_scales, int64_t M, const ql_weights* w,
+                                    void* Y, cudaStream_t st, int* status, Gate gate) {
+  using C = W4A8TsCfg<BMT, RS, XW>;
+  const int N = w->N, K = w->K;
+  CUtensorMap tx, tw, ty;
+  if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a_codes, K, M, static_cast<int64_t>(K) * 2, C::BK, BMT,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, K / 2, N, K / 2, C::BK / 2, 128,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<int64_t>(N) * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+    return QL_ERR_CUDA;
+  GemmArgs p{};
+  fill_gemm_args(p, M, N, K, 128, status);
+  p.tiles_m = static_cast<int32_t>((M + BMT - 1) / BMT);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.num_kst = K / C::BK;
+  p.k_atoms = K / 64;
+  p.sfb_atoms = (N + 127) / 128;
+  p.sfb = static_cast<const uint8_t*>(w->sf);
+  p.g_w = w->gscale;
+  p.row_scale = a_scales;
+  p.alpha_mul = w->hadamard ? (1.0f / 128.0f) : 1.0f;
+  p.gate = gate.route;
+  p.gate_value = gate.value;
+  auto kern = k_gemm_w4a8_ts<BMT, RS, XW>;
+  if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
+  const int grid = std::min(p.num_tiles, num_sms());
+  if (launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, tx, tw, ty, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
+}
+
 ql_status launch_gemm_w4a8(const void* a_codes, const float* a_scales, int64_t M, const ql_weights* w,
                            void* Y, cudaStream_t st, int* status, int a_f16, Gate gate) {
   if (M == 0) return QL_OK;
   const bool n192 = w->N % 192 == 0;
-  if (a_f16) {   // f16 activations and pre-expanded weights: both operands by TMA
-    if (w->w16 == nullptr) return QL_ERR_UNSUPPORTED_SHAPE;
+  if (a_f16) {
+    // without the weight copy: the weights widened into tensor memory
+    if (w->w16 == nullptr) return launch_w4a8_ts_cfg<192, 6, 8>(a_codes, a_scales, M, w, Y, st, status, gate);
+    // f16 activations and pre-expanded weights: both operands by TMA
     if (n192) return launch_w4a8_cfg<192, 1, 4, true, true>(a_codes, a_scales, M, w, Y, st, status, gate);
     return launch_w4a8_cfg<128, 1, 5, true, true>(a_codes, a_scales, M, w, Y, st, status, gate);
   }

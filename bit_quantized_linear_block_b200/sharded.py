@@ -95,7 +95,9 @@ def activation_format(w: Q.PackedWeights, route: int) -> tuple[int, bool, bool]:
         return Q.QL_ACT_NVFP4_DECOMP, bool(w.desc.hadamard), True
     if route == Q.QL_ROUTE_NVFP4:
         return Q.QL_ROUTE_NVFP4, bool(w.desc.hadamard), True
-    return route, bool(w.desc.hadamard), False
+    # per-token integer codes are kept as f16 values, the f16 MMA's operand type
+    per_token_f16 = {Q.QL_ROUTE_INT8: Q.QL_ACT_INT8_F16, Q.QL_ROUTE_INT6: Q.QL_ACT_INT6_F16}
+    return per_token_f16.get(route, route), bool(w.desc.hadamard), False
 
 
 def forward_with_amax(x_local: torch.Tensor, w: Q.PackedWeights, route: int, amax: torch.Tensor,

@@ -99,8 +99,8 @@ typedef enum {
   QL_ROUTE_INT8 = 1,        /* W4A8: per-token INT8 activations              */
   QL_ACT_INT8_TENSOR = 2,   /* Q-ARVD: per-tensor INT8, permuted K           */
   QL_ACT_INT8_F16 = 3,      /* W4A8: per-token INT8 codes stored as the equal
-                               f16 values, f16 [M, K]; the GEMM needs weights
-                               prepared with expand_f16                      */
+                               f16 values, f16 [M, K] (the operand type of
+                               the f16 MMA)                                  */
   QL_ACT_NVFP4_DECOMP = 4,  /* activation decomposition (SemanticDialect,
                                Methodology 2.2): NVFP4 of h, then NVFP4 of the
                                residual r = RN(h - RN(e2m1(q1) RN(sb1 g))) with
@@ -112,8 +112,7 @@ typedef enum {
      integer GEMMs multiply exactly. */
   QL_ROUTE_INT6 = 5,        /* per-token INT6 (int8 [M, K] + fp32 [M]); also
                                a qlinear_forward route                        */
-  QL_ACT_INT6_F16 = 6,      /* per-token INT6 codes as f16 values (weights with
-                               expand_f16)                                    */
+  QL_ACT_INT6_F16 = 6,      /* per-token INT6 codes as f16 values           */
   QL_ACT_INT6_TENSOR = 7,   /* Q-ARVD per-tensor INT6 in the permuted K order  */
   QL_ROUTE_BF16 = 8         /* unquantized bf16 product X W^T (PDR's
                                high-precision refresh); the activations are
@@ -205,7 +204,7 @@ QL_API size_t qlinear_sf_bytes(int64_t rows, int32_t K);
    CTA sorts all channel norms in shared memory); otherwise the call returns
    QL_ERR_INVALID_ARG.  The per-tensor Q-ARVD activation quantizer stages a
    row in shared memory and returns QL_ERR_UNSUPPORTED_SHAPE when that does
-   not fit (about K > 29000). */
+   not fit (about K > 22000). */
 QL_API size_t qlinear_weights_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg);
 QL_API size_t qlinear_prepare_ws_bytes(int32_t N, int32_t K, const ql_weight_cfg* cfg);
 QL_API ql_status qlinear_prepare_weights(const void* W_bf16, int32_t N, int32_t K,
@@ -305,8 +304,10 @@ QL_API ql_status qlinear_quantize_act(const void* X_bf16, int64_t M, int32_t K,
    QL_ROUTE_INT8:      INT8 x NVFP4 weights (their f16 copy when prepared with
                        expand_f16, else expanded on chip to f16);
                        alpha_m = s_m g_w (/128 if rotated).
-   QL_ACT_INT8_F16:    as QL_ROUTE_INT8 with f16 codes; needs the f16 copy;
-                       both operands go straight to the f16 MMA.
+   QL_ACT_INT8_F16:    as QL_ROUTE_INT8 with f16 codes: with the f16 copy both
+                       operands go straight to the f16 MMA; without it the
+                       FP4 weights are widened into tensor memory and fed to
+                       the MMA from there (same results).
    QL_ACT_INT8_TENSOR: INT8 x INT4 integer MMA, two class accumulators;
                        y = s_x (s_norm[n] acc_normal + s_out[n] acc_outlier).
    QL_ACT_NVFP4_DECOMP: the W4A4 GEMM over K' = 2K ([q1 | q2] x [W | W]).
@@ -323,10 +324,8 @@ QL_API ql_status qlinear_gemm(int32_t act_fmt, const void* a_codes, const void* 
    QL_ROUTE_INT6 or QL_ACT_INT6_TENSOR selects per-tensor INT6 activations,
    any other value per-tensor INT8; QL_ROUTE_NVFP4 only for
    QL_W_NVFP4_DECOMP weights.  Scratch for the quantized activations lives
-   in `ws`.  On the INT8
-   route with weights prepared with expand_f16, the INT8 codes are kept as
-   the equal f16 values (2 bytes each) so that the GEMM reads both operands
-   straight into the f16 MMA. */
+   in `ws`.  On the INT8 route the codes are kept as the equal f16 values
+   (2 bytes each, QL_ACT_INT8_F16), the f16 MMA's operand type. */
 QL_API size_t qlinear_forward_ws_bytes(int64_t M, const ql_weights* w, int32_t route);
 QL_API ql_status qlinear_forward(const void* X_bf16, int64_t M, const ql_weights* w,
                           int32_t route, void* Y_bf16,
@@ -335,8 +334,8 @@ QL_API ql_status qlinear_forward(const void* X_bf16, int64_t M, const ql_weights
 /* ---- forward with the route in device memory ----------------------------
    DMPQ routes a block from the previous step's Gamma, which the router (or
    a TDC state's next_route) leaves in device memory.  This forward enqueues
-   the kernels of every route the weights support -- NVFP4, INT8 (f16-coded
-   with an f16 weight copy) and, with keep_bf16, BF16 -- and each kernel
+   the kernels of every route the weights support -- NVFP4, INT8 (f16-coded)
+   and, with keep_bf16, BF16 -- and each kernel
    waits for its predecessor, reads *route_dev and returns at once unless
    the route is its own.  So the call never synchronizes with the host and
    a whole step can be captured in one CUDA graph.  Weights: QL_W_NVFP4.

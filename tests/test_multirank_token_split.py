@@ -115,8 +115,11 @@ def test_activation_format_follows_the_forward():
 
     nv, qa, de = packed(Q.QL_W_NVFP4, 1), packed(Q.QL_W_QARVD_INT4, 0), packed(Q.QL_W_NVFP4_DECOMP, 1)
     assert SH.activation_format(nv, Q.QL_ROUTE_NVFP4) == (Q.QL_ROUTE_NVFP4, True, True)
-    for route in (Q.QL_ROUTE_INT8, Q.QL_ROUTE_INT6, Q.QL_ACT_INT8_F16, Q.QL_ROUTE_BF16):
+    for route in (Q.QL_ACT_INT8_F16, Q.QL_ACT_INT6_F16, Q.QL_ROUTE_BF16):
         assert SH.activation_format(nv, route) == (route, True, False)      # per token or unquantized
+    # the per-token integer routes quantize to f16-coded integers, as qlinear_forward does
+    assert SH.activation_format(nv, Q.QL_ROUTE_INT8) == (Q.QL_ACT_INT8_F16, True, False)
+    assert SH.activation_format(nv, Q.QL_ROUTE_INT6) == (Q.QL_ACT_INT6_F16, True, False)
     assert SH.activation_format(qa, Q.QL_ACT_INT8_TENSOR) == (Q.QL_ACT_INT8_TENSOR, False, True)
     assert SH.activation_format(qa, Q.QL_ROUTE_INT6) == (Q.QL_ACT_INT6_TENSOR, False, True)
     assert SH.activation_format(qa, Q.QL_ACT_INT6_TENSOR) == (Q.QL_ACT_INT6_TENSOR, False, True)
