@@ -453,7 +453,9 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
 // never leaves [-qmax, qmax].  The int8 path keeps each code's low byte
 // (two's complement) and packs four with byte permutes; the f16 path
 // rounds in fp32 (rint), turns -0 into +0 (the code 0 is stored as +0) and
-// converts two codes per instruction.
+// converts two codes per instruction.  The rounding is a conversion of the
+// rounded product, never an addition after it: the compiler may fuse a
+// product and a following addition into one FMA, which rounds once.
 __device__ __forceinline__ uint32_t pack4_s8(int a0, int a1, int a2, int a3) {
   const uint32_t t01 = __byte_perm(static_cast<uint32_t>(a0), static_cast<uint32_t>(a1), 0x0040);
   const uint32_t t23 = __byte_perm(static_cast<uint32_t>(a2), static_cast<uint32_t>(a3), 0x0040);
@@ -582,92 +584,150 @@ __global__ void __launch_bounds__(kThreadsHbm)
 // Per-tensor INT8 in Q-ARVD channel order.  Output row = Kp bytes; slot j
 // takes input channel gather[j] (or 0 for a padding slot).  The scale comes
 // from the device amax of the un-rotated tensor.
-// One CTA per row at a time, kPermRing rows in flight: each bf16 row comes
-// into one of kPermRing shared-memory buffers by one bulk copy (tracked by
-// the buffer's mbarrier), issued kPermRing rows ahead.  Each row buffer ends
-// with 16 zero bytes, and the gather table (int16 in shared memory) sends
-// padding slots to that zero element, so every slot is one table read, one
-// row read and no branch.  Each thread takes 4 consecutive slots per step
-// and writes 4 codes as one word of a shared output row, which leaves with
-// 16-byte stores.  As in the per-token quantizer the codes need no clamp
-// (|RN(x * RN(qmax / amax))| < qmax + 1/2).
+//
+// A CTA walks groups of G consecutive rows (G from the host: about 12 KB of
+// bf16 per group) through a ring of R group buffers (R from the host, 2 to
+// 4: the depth that keeps the most groups in flight per SM at the occupancy
+// it allows), R - 1 groups in flight while one is read.  Thread 0 brings each row of
+// a group into its own shared-memory buffer by one bulk copy; each buffer
+// ends with 16 zero bytes, and the gather table (uint16 in shared memory)
+// sends padding slots to that zero element, so every slot is one table
+// read, one row read and no branch.  The warps work independently: each
+// waits on the group's mbarrier, takes whole 512-slot units (lane l: slots
+// 4l + 128s + c, s, c < 4; consecutive lanes read neighbouring channels),
+// writes four codes per lane and step as one coalesced word, and arrives on
+// the group's release barrier; thread 0 refills a buffer once every warp has
+// released it.  Units are numbered across groups and dealt to the warps
+// round-robin, so a group's ragged unit count does not load one warp more
+// than the others.
+//
+// Codes: rint(RN(x * RN(qmax / amax))), low bytes packed by byte permutes;
+// no clamp is needed, as in the per-token quantizer (|y| < qmax + 1/2).
 // ---------------------------------------------------------------------------
-constexpr int kPermRing = 4;
-struct PermLayout {   // row buffers: the bf16 row (K * 2 bytes) and 16 zero bytes
-  int32_t gather_bytes, row_bytes, buf_bytes, out_bytes, total;
-  __host__ __device__ PermLayout(int32_t K, int32_t Kp)
-      : gather_bytes((Kp * 2 + 15) / 16 * 16), row_bytes(K * 2), buf_bytes(K * 2 + 16),
-        out_bytes((Kp + 15) / 16 * 16),
-        total((Kp * 2 + 15) / 16 * 16 + kPermRing * (K * 2 + 16) + (Kp + 15) / 16 * 16) {}
+constexpr int kPermMaxRing = 4;
+constexpr int kPermThreads = 256;
+constexpr int kPermWarps = kPermThreads / 32;
+constexpr int kPermUnit = 512;   // slots per warp unit
+struct PermLayout {
+  int32_t G, row_stride, group_bytes, table_bytes, ring;
+  PermLayout(int32_t K, int32_t Kp, int32_t R)
+      : G(std::max(1, 12288 / (2 * K))), row_stride(2 * K + 16), group_bytes(G * (2 * K + 16)),
+        table_bytes((2 * Kp + 15) / 16 * 16), ring(R) {}
+  int32_t total() const { return table_bytes + ring * group_bytes; }
 };
-constexpr int kPermThreads = 512;
 
 __global__ void __launch_bounds__(kPermThreads)
     k_quant_int8_tensor_perm(const uint8_t* __restrict__ x, int64_t M, int32_t K, int32_t Kp,
                              const int32_t* __restrict__ gather, const float* amax_in, int qmax,
-                             int8_t* __restrict__ codes, float* __restrict__ scale_out, int* status) {
+                             int8_t* __restrict__ codes, float* __restrict__ scale_out, int* status,
+                             int32_t G, int32_t row_stride, int32_t group_bytes, int32_t table_bytes, int32_t R) {
   extern __shared__ __align__(16) uint8_t s_perm[];
-  __shared__ uint64_t full[kPermRing];
-  __shared__ int s_ok;
-  const PermLayout L(K, Kp);
-  int16_t* s_gather = reinterpret_cast<int16_t*>(s_perm);
-  uint8_t* rows = s_perm + L.gather_bytes;
-  uint32_t* orow = reinterpret_cast<uint32_t*>(s_perm + L.gather_bytes + kPermRing * L.buf_bytes);
+  __shared__ uint64_t full[kPermMaxRing], release[kPermMaxRing];
+  __shared__ int s_fail;
+  uint16_t* s_gather = reinterpret_cast<uint16_t*>(s_perm);
+  uint8_t* ring = s_perm + table_bytes;
+  const int64_t ngroups = (M + G - 1) / G;
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = lane_id();
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kPermRing; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < R; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&release[i], kPermWarps);
+    }
     fence_mbar_init();
-    s_ok = 1;
+    s_fail = 0;
   }
+  for (int i = threadIdx.x; i < R * G; i += kPermThreads)   // the zero element after each row buffer
+    *reinterpret_cast<uint4*>(ring + (i / G) * group_bytes + (i % G) * row_stride + 2 * K) = make_uint4(0, 0, 0, 0);
   __syncthreads();
-  if (threadIdx.x < kPermRing)   // the zero element after each row buffer
-    *reinterpret_cast<uint4*>(rows + threadIdx.x * L.buf_bytes + L.row_bytes) = make_uint4(0, 0, 0, 0);
   pdl_wait();
-  for (int i = threadIdx.x; i < Kp; i += blockDim.x) {   // padding slots (-1) read the zero element
+  const int64_t first = blockIdx.x, step = gridDim.x;
+  auto issue = [&](int64_t grp, int slot) {   // thread 0 only
+    const int32_t rows = static_cast<int32_t>(M - grp * G < G ? M - grp * G : G);
+    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(rows) * 2u * static_cast<uint32_t>(K));
+    for (int32_t r = 0; r < rows; ++r)
+      bulk_load(ring + slot * group_bytes + r * row_stride, x + (grp * G + r) * 2 * K, 2u * static_cast<uint32_t>(K),
+                &full[slot]);
+  };
+  int issued = 0;   // groups issued by thread 0 (iterations 0 .. issued - 1)
+  if (threadIdx.x == 0)
+    for (; issued < R && first + issued * step < ngroups; ++issued) issue(first + issued * step, issued);
+  for (int i = threadIdx.x; i < Kp; i += kPermThreads) {   // padding slots (-1) read the zero element
     const int32_t g = gather[i];
-    s_gather[i] = static_cast<int16_t>(g < 0 ? K : g);
+    s_gather[i] = static_cast<uint16_t>(g < 0 ? K : g);
   }
   const float amax = ld_dep(amax_in);
   const float fq = static_cast<float>(qmax);
   const float inv = (amax == 0.f) ? 0.f : __fdiv_rn(fq, amax);
   if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = (amax == 0.f) ? 0.f : __fdiv_rn(amax, fq);
-  auto issue_row = [&](int64_t r, int slot) {   // thread 0 only
-    mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(L.row_bytes));
-    bulk_load(rows + slot * L.buf_bytes, x + r * L.row_bytes, static_cast<uint32_t>(L.row_bytes), &full[slot]);
-  };
   const float2 inv2 = make_float2(inv, inv);
-  const int64_t first = blockIdx.x, step = gridDim.x;
-  if (threadIdx.x == 0)
-    for (int i = 0; i < kPermRing && first + i * step < M; ++i) issue_row(first + i * step, i);
+  __syncthreads();   // gather table complete
+  const int32_t upr = (Kp + kPermUnit - 1) / kPermUnit;   // units per row
+  int32_t deal = 0;                                       // units dealt before this group, mod kPermWarps
   int k = 0;
-  for (int64_t r = first; r < M; r += step, ++k) {
-    const int slot = k % kPermRing;
-    if (threadIdx.x == 0) s_ok = (mbar_wait(&full[slot], static_cast<uint32_t>((k / kPermRing) & 1), kDrainLimit)) ? 1 : 0;
-    __syncthreads();   // this row landed; gather table ready; the previous output row was stored
-    if (!s_ok) break;
-    const unsigned short* xr = reinterpret_cast<const unsigned short*>(rows + slot * L.buf_bytes);
-    for (int32_t w = threadIdx.x; 4 * w < Kp; w += kPermThreads) {
-      const uint2 gi = *reinterpret_cast<const uint2*>(s_gather + 4 * w);   // 4 channel indices
-      const float2 v01 = make_float2(__uint_as_float(static_cast<uint32_t>(xr[gi.x & 0xFFFFu]) << 16),
-                                     __uint_as_float(static_cast<uint32_t>(xr[gi.x >> 16]) << 16));
-      const float2 v23 = make_float2(__uint_as_float(static_cast<uint32_t>(xr[gi.y & 0xFFFFu]) << 16),
-                                     __uint_as_float(static_cast<uint32_t>(xr[gi.y >> 16]) << 16));
-      const float2 y01 = __fmul2_rn(v01, inv2), y23 = __fmul2_rn(v23, inv2);
-      orow[w] = pack4_s8(__float2int_rn(y01.x), __float2int_rn(y01.y), __float2int_rn(y23.x), __float2int_rn(y23.y));
+  bool ok = true;
+  for (int64_t grp = first; grp < ngroups; grp += step, ++k) {
+    const int slot = k % R;
+    if (threadIdx.x == 0 && k > 0 && first + static_cast<int64_t>(k - 1 + R) * step < ngroups) {
+      // refill the buffer of iteration k - 1 with iteration k - 1 + R's rows
+      // once every warp has released it
+      const int prev = (k - 1) % R;
+      if (!mbar_wait(&release[prev], static_cast<uint32_t>(((k - 1) / R) & 1), kDrainLimit)) {
+        s_fail = 1;
+        record_error(status, QL_ERR_TIMEOUT);
+      } else {
+        issue(first + static_cast<int64_t>(k - 1 + R) * step, prev);
+        ++issued;
+      }
     }
-    __syncthreads();   // output row complete; the row buffer may be refilled
-    if (threadIdx.x == 0 && r + kPermRing * step < M) issue_row(r + kPermRing * step, slot);
-    int8_t* dst = codes + r * Kp;
-    for (int32_t o = 16 * static_cast<int32_t>(threadIdx.x); o < Kp; o += 16 * kPermThreads)
-      *reinterpret_cast<uint4*>(dst + o) = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(orow) + o);
+    int w_ok = 1;
+    if (lane == 0)
+      w_ok = *reinterpret_cast<volatile int*>(&s_fail) == 0 &&
+             mbar_wait(&full[slot], static_cast<uint32_t>((k / R) & 1), kDrainLimit);
+    if (!__shfl_sync(0xffffffffu, w_ok, 0)) {
+      if (lane == 0 && !s_fail) {
+        s_fail = 1;
+        record_error(status, QL_ERR_TIMEOUT);
+      }
+      ok = false;
+      break;
+    }
+    const int32_t rows = static_cast<int32_t>(M - grp * G < G ? M - grp * G : G);
+    const int32_t units = rows * upr;
+    const uint8_t* buf = ring + slot * group_bytes;
+    for (int32_t u = (warp - deal + kPermWarps) % kPermWarps; u < units; u += kPermWarps) {
+      const int32_t r = u / upr;
+      const int32_t j0 = (u - r * upr) * kPermUnit + 4 * static_cast<int32_t>(lane);
+      const unsigned short* xr = reinterpret_cast<const unsigned short*>(buf + r * row_stride);
+      int8_t* dst = codes + (grp * G + r) * Kp;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const int32_t j = j0 + 128 * s;
+        if (j < Kp) {   // Kp is a multiple of 32: four slots are all in or all out
+          const uint2 gi = *reinterpret_cast<const uint2*>(s_gather + j);
+          const float2 v01 = make_float2(__uint_as_float(static_cast<uint32_t>(xr[gi.x & 0xFFFFu]) << 16),
+                                         __uint_as_float(static_cast<uint32_t>(xr[gi.x >> 16]) << 16));
+          const float2 v23 = make_float2(__uint_as_float(static_cast<uint32_t>(xr[gi.y & 0xFFFFu]) << 16),
+                                         __uint_as_float(static_cast<uint32_t>(xr[gi.y >> 16]) << 16));
+          const float2 y01 = __fmul2_rn(v01, inv2), y23 = __fmul2_rn(v23, inv2);
+          *reinterpret_cast<uint32_t*>(dst + j) =
+              pack4_s8(__float2int_rn(y01.x), __float2int_rn(y01.y), __float2int_rn(y23.x), __float2int_rn(y23.y));
+        }
+      }
+    }
+    deal = (deal + units) % kPermWarps;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&release[slot]);
   }
   pdl_release();
   if (threadIdx.x == 0) {
-    // every copy issued has landed before the CTA may exit (only a timed-out
-    // wait leaves copies in flight: wait for them with a bounded budget)
-    int64_t r = first + static_cast<int64_t>(k) * step;
-    if (!s_ok) record_error(status, QL_ERR_TIMEOUT);
-    for (int i = 0; i < kPermRing && r < M; ++i, r += step)
-      if (!s_ok || i > 0) (void)mbar_wait(&full[(k + i) % kPermRing], static_cast<uint32_t>(((k + i) / kPermRing) & 1), kDrainLimit);
+    // every copy issued must land before the CTA exits; after a normal walk
+    // each was consumed, after a failure wait for the rest with a bounded budget
+    // (only the last R issued can be in flight: a buffer is refilled
+    // after every warp consumed its previous copy)
+    if (!ok || *reinterpret_cast<volatile int*>(&s_fail))
+      for (int j = issued > R ? issued - R : 0; j < issued; ++j)
+        (void)mbar_wait(&full[j % R], static_cast<uint32_t>((j / R) & 1), kDrainLimit);
   }
   __syncthreads();
 }
@@ -819,21 +879,40 @@ ql_status launch_quant_int8_token(const void* x, int64_t M, int32_t K, int hadam
 ql_status launch_quant_int8_tensor_perm(const void* x, int64_t M, int32_t K, int32_t Kp,
                                         const int32_t* gather, const float* amax_in, void* codes,
                                         float* scale_out, cudaStream_t st, int qmax) {
-  const PermLayout L(K, Kp);
-  if (L.total > 200 * 1024) return QL_ERR_UNSUPPORTED_SHAPE;
-  if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_int8_tensor_perm), L.total)) return QL_ERR_CUDA;
-  // as many CTAs as can be resident at once: each walks rows blockIdx.x,
-  // blockIdx.x + gridDim.x, ..., so a CTA that waited for a free SM would
-  // start its rows late
+  if (K > 65535) return QL_ERR_UNSUPPORTED_SHAPE;   // uint16 gather table
+  // ring depth: the most groups in flight per SM ((depth - 1) per resident
+  // CTA, the one being read aside), fewer slots where that fits more CTAs
+  PermLayout L(K, Kp, 0);
+  int best = 0, best_flight = 0;
+  for (int R = kPermMaxRing; R >= 2; --R) {
+    L.ring = R;
+    if (L.total() > 220 * 1024) continue;
+    if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_int8_tensor_perm), L.total())) return QL_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_int8_tensor_perm, kPermThreads,
+                                                      L.total()) != cudaSuccess)
+      return QL_ERR_CUDA;
+    if (per_sm * (R - 1) > best_flight) {
+      best_flight = per_sm * (R - 1);
+      best = R;
+    }
+  }
+  if (best == 0) return QL_ERR_UNSUPPORTED_SHAPE;   // not even two row groups fit in shared memory
+  L.ring = best;
+  if (!set_smem_attr(reinterpret_cast<const void*>(k_quant_int8_tensor_perm), L.total())) return QL_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_int8_tensor_perm, kPermThreads, L.total) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_int8_tensor_perm, kPermThreads, L.total()) !=
           cudaSuccess ||
       per_sm < 1)
     return QL_ERR_CUDA;
-  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(M, static_cast<int64_t>(per_sm) * num_sms())));
-  if (launch_pdl(k_quant_int8_tensor_perm, dim3(grid), dim3(kPermThreads), L.total, st, 1,
+  // as many CTAs as can be resident at once: each walks row groups
+  // blockIdx.x, blockIdx.x + gridDim.x, ..., so a CTA that waited for a free
+  // SM would start its rows late
+  const int64_t ngroups = (M + L.G - 1) / L.G;
+  const int grid = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(ngroups, static_cast<int64_t>(per_sm) * num_sms())));
+  if (launch_pdl(k_quant_int8_tensor_perm, dim3(grid), dim3(kPermThreads), L.total(), st, 1,
                  static_cast<const uint8_t*>(x), M, K, Kp, gather, amax_in, qmax, static_cast<int8_t*>(codes),
-                 scale_out, status_word()) != cudaSuccess) {
+                 scale_out, status_word(), L.G, L.row_stride, L.group_bytes, L.table_bytes, L.ring) != cudaSuccess) {
     (void)cudaGetLastError();
     return QL_ERR_CUDA;
   }
