@@ -44,6 +44,8 @@ THRESHOLD = 0.05
 M_TOKENS = S.M_COGVIDEOX
 BLOCK_SIGMA = 0.01          # stable block: Gamma ~ 0.01 < 0.05 -> NVFP4 route
 FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
+FP4_DATASHEET_TFLOPS = 9000.0   # B200 dense FP4, datasheet (context only)
+L2_BYTES = 126e6
 NVFP4_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # bf16 in, E2M1 out, E4M3 per 16
 # DRAM bytes per launch of the W4A4 GEMM from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of the GEMM sources).
@@ -65,7 +67,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--configs", action="store_true",
                     help="time every kernel of the five workload configurations (one JSON line, not the contract line)")
-    ap.add_argument("--profile-case", choices=["quant", "gemm", "qarvd", "tdc", "decomp"], default=None,
+    ap.add_argument("--profile-case", choices=["quant", "gemm", "qarvd", "tdc", "decomp", "int8", "w4a8", "route",
+                                               "qarvd_quant", "bf16"], default=None,
                     help="run one small standalone case for an ncu capture (prints no JSON)")
     return ap.parse_args()
 
@@ -112,6 +115,52 @@ def profile_case(which: str):
         for _ in range(2):
             ql.qlinear_quantize_act(x, ql.QL_ACT_NVFP4_DECOMP, True, amax_in=amax, out=q)
             ql.qlinear_gemm(ql.QL_ACT_NVFP4_DECOMP, q, x.shape[0], pw, Y=y)
+    elif which == "int8":    # per-token INT8 / f16-coded quantizer on [65536, 1920] (252 MB of bf16)
+        m, k = 65536, 1920
+        x = S.activations_with_outlier_channels(m, k, 0.01, 30.0, 1, 1).to(dev)
+        q = ql.qlinear_quantize_act(x, ql.QL_ROUTE_INT8, True)
+        q16 = ql.qlinear_quantize_act(x, ql.QL_ACT_INT8_F16, True)
+        for _ in range(2):
+            ql.qlinear_quantize_act(x, ql.QL_ROUTE_INT8, True, out=q)
+            ql.qlinear_quantize_act(x, ql.QL_ACT_INT8_F16, True, out=q16)
+    elif which in ("w4a8", "bf16"):   # INT8-route / BF16 GEMM, M=8192, N=7680, K=1920 (FFN-up shape)
+        m, n, k = 8192, 7680, 1920
+        x = S.activations_with_outlier_channels(m, k, 0.01, 30.0, 1, 1).to(dev)
+        w = S.weights(n, k, 0.02, 1, 2).to(dev)
+        if which == "w4a8":   # per round: f16 codes with the weights widened into tensor memory, int8 codes
+            # with both operands widened in shared memory, f16 codes with the f16 weight copy (both by TMA)
+            pw = ql.qlinear_prepare_weights(w, ql.QL_W_NVFP4, True)
+            pwx = ql.qlinear_prepare_weights(w, ql.QL_W_NVFP4, True, expand_f16=True)
+            q = ql.qlinear_quantize_act(x, ql.QL_ROUTE_INT8, True)
+            q16 = ql.qlinear_quantize_act(x, ql.QL_ACT_INT8_F16, True)
+            y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+            for _ in range(2):
+                ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q16, m, pw, Y=y)
+                ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, m, pw, Y=y)
+                ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q16, m, pwx, Y=y)
+        else:
+            pwb = ql.qlinear_prepare_weights(w, ql.QL_W_NVFP4, True, keep_bf16=True)
+            y = ql.qlinear_gemm(ql.QL_ROUTE_BF16, {"codes": x, "scales": None}, m, pwb)
+            for _ in range(2):
+                ql.qlinear_gemm(ql.QL_ROUTE_BF16, {"codes": x, "scales": None}, m, pwb, Y=y)
+    elif which == "route":   # router on a block pair [65536, 1920] (2 x 252 MB of bf16)
+        rng = np.random.default_rng(5)
+        xi = rng.standard_normal((65536, 1920), dtype=np.float32)
+        bi = S.to_bf16(xi).to(dev)
+        bo = S.to_bf16(xi + np.float32(0.01) * rng.standard_normal((65536, 1920), dtype=np.float32)).to(dev)
+        rws = torch.zeros(ql.lib.qlinear_route_ws_bytes(bi.numel()), dtype=torch.uint8, device=dev)
+        g, r = ql.qlinear_route(bi, bo, THRESHOLD, ws=rws)
+        for _ in range(2):
+            ql.qlinear_route(bi, bo, THRESHOLD, gamma=g, route=r, ws=rws)
+    elif which == "qarvd_quant":   # Q-ARVD per-tensor INT8 with the channel permutation, [32768, 3072] / [8192, 12288]
+        for m, k, nout in ((32768, 3072, 1024), (8192, 12288, 1024)):
+            x = S.activations_with_outlier_channels(m, k, 0.01, 30.0, 1, 1).to(dev)
+            w = S.weights(nout, k, 0.02, 3, 9, outlier_frac=0.02, outlier_scale=20.0).to(dev)
+            pw = ql.qlinear_prepare_weights(w, ql.QL_W_QARVD_INT4, False)
+            amax = ql.qlinear_tensor_amax(x, False)
+            q = ql.qlinear_quantize_act(x, ql.QL_ACT_INT8_TENSOR, False, w=pw, amax_in=amax)
+            for _ in range(2):
+                ql.qlinear_quantize_act(x, ql.QL_ACT_INT8_TENSOR, False, w=pw, amax_in=amax, out=q)
     else:                    # W4A4 GEMM M=8192, N=7680, K=1920 (FFN-up shape, fewer tokens)
         m, n, k = 8192, 7680, 1920
         x = S.activations_with_outlier_channels(m, k, 0.01, 30.0, 1, 1).to(dev)
@@ -183,46 +232,53 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50", "-i", str(self.dev)],
+                 "-lms", "10", "-i", str(self.dev)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
 
-    def stop(self, t_begin: float | None = None, t_end: float | None = None):
-        """Median SM clock and throttle reasons of the samples whose host
-        timestamp lies in [t_begin, t_end] (all samples when not given)."""
+    def stop(self):
+        """Stop sampling; keep the samples as (host time, SM MHz, max MHz,
+        active throttle reasons)."""
+        self.samples = []
         if self.proc is None:
-            return None
+            return
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        sm, mx, reasons = [], [], set()
         for line in out.strip().splitlines():
             f = [c.strip() for c in line.split(",")]
             if len(f) < 10:
                 continue
             try:
                 ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-            except ValueError:
-                ts = None
-            if t_begin is not None and ts is not None and not (t_begin <= ts <= t_end):
-                continue
-            f = f[1:]
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
+                sm, mx = float(f[2]), float(f[3])
             except ValueError:
                 continue
-            for name, v in zip(self.NAMES, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(name)
-        if not sm:
+            reasons = {name for name, v in zip(self.NAMES, f[6:10]) if v.lower() == "active"}
+            self.samples.append((ts, sm, mx, reasons))
+
+    def window(self, t_begin: float | None = None, t_end: float | None = None):
+        """Median SM clock and throttle reasons of the samples whose host
+        timestamp lies in [t_begin, t_end] (all samples when not given).  A
+        window shorter than the sampling interval may hold no sample: it is
+        then widened by 100 ms on each side, and the record says so."""
+        samples = getattr(self, "samples", [])
+        sel = [s for s in samples if t_begin is None or t_begin <= s[0] <= t_end]
+        widened = 0
+        if not sel and t_begin is not None:
+            widened = 100
+            sel = [s for s in samples if t_begin - 0.1 <= s[0] <= t_end + 0.1]
+        if not sel:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
-                "reasons": sorted(reasons)}
+        rec = {"sm_mhz": statistics.median(s[1] for s in sel), "sm_max_mhz": max(s[2] for s in sel),
+               "samples": len(sel), "reasons": sorted(set().union(*(s[3] for s in sel)))}
+        if widened:
+            rec["window_widened_ms"] = widened
+        return rec
 
 
 def measured_peaks():
@@ -331,56 +387,111 @@ def run_ours(args, rank, world, local):
     t1.record(stream)
     torch.cuda.synchronize()
     th1 = time.time()
-    clocks = sampler.stop(th0, th1)
+    sampler.stop()
+    clocks = sampler.window(th0, th1)
     dist_barrier(world)
     assert ql.qlinear_device_status() == 0
     ms = t0.elapsed_time(t1)
     ms_max = dist_max(ms, world)
     del graph
 
-    # Per-kernel breakdown: each kernel alone, 10 launches per CUDA graph,
-    # CUDA events around `reps` replays (device time per launch, us).
-    def launch_us(fn, reps=20, per_graph=10):
+    # Per-kernel breakdown: each kernel alone in a CUDA graph whose launches
+    # rotate over enough copies of the kernel's operands that one replay
+    # touches more than twice the 126 MB L2 (no launch finds its inputs
+    # left in L2 by the launch before); CUDA events around replays that
+    # fill at least 0.2 s, with the SM clock sampled over each window.
+    rot_bytes = 2 * L2_BYTES
+
+    def nrot(nbytes):
+        return int(min(8, max(1, -(-rot_bytes // nbytes))))
+
+    windows = {}
+    ksampler = ClockSampler(local)
+    ksampler.start()
+    time.sleep(0.3)
+
+    def launch_us(name, fn, per_graph=12, windows_n=8, window_s=0.025, pause_s=0.04):
+        # `windows_n` replay windows of about `window_s` each, `pause_s`
+        # apart: bursts like the step the kernel belongs to, together at
+        # least 0.2 s of timing with several clock samples.  Median window.
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            for _ in range(per_graph):
-                fn()
+            for j in range(per_graph):
+                fn(j)
         g.replay()
         torch.cuda.synchronize()
         a, b = pair()
         a.record(stream)
-        for _ in range(reps):
-            g.replay()
+        g.replay()
         b.record(stream)
         torch.cuda.synchronize()
+        reps = max(3, int(window_s / max(1e-6, a.elapsed_time(b) * 1e-3)) + 1)
+        per, wins = [], []
+        for _ in range(windows_n):
+            time.sleep(pause_s)
+            th0 = time.time()
+            a.record(stream)
+            for _ in range(reps):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            wins.append((th0, time.time()))
+            per.append(1e3 * a.elapsed_time(b) / (reps * per_graph))
+        windows[name] = wins
         del g
-        return 1e3 * a.elapsed_time(b) / (reps * per_graph)
+        return statistics.median(per)
 
-    route_us = launch_us(lambda: ql.qlinear_route(bin_d, bout_d, THRESHOLD, gamma=gamma_d, route=route_d,
-                                                  ws=route_ws))
+    rin = [bin_d] + [bin_d.clone() for _ in range(nrot(4 * bin_d.numel()) - 1)]
+    rout = [bout_d] + [bout_d.clone() for _ in range(len(rin) - 1)]
+    route_us = launch_us("route", lambda j: ql.qlinear_route(rin[j % len(rin)], rout[j % len(rin)], THRESHOLD,
+                                                             gamma=gamma_d, route=route_d, ws=route_ws))
+    del rin, rout
     kt = []
-    for i in range(len(lins)):
+    for i, (lin, _, _) in enumerate(lins):
+        rx = [xs[i]] + [xs[i].clone() for _ in range(nrot(2 * xs[i].numel()) - 1)]
+        rq = [qbufs[i]] + [ql.qlinear_quantize_act(x, host_route, True, amax_in=amax[i], rowmajor_scales=False)
+                           for x in rx[1:]]
+        ry = [ys[i]] + [torch.empty_like(ys[i]) for _ in range(nrot(2 * ys[i].numel() + M_TOKENS * lin.k // 2) - 1)]
+        nx, ny = len(rx), len(ry)
         kt.append({
-            "amax": launch_us(lambda i=i: ql.qlinear_tensor_amax(xs[i], True, out=amax[i], ws=amax_ws[i])),
-            "quant": launch_us(lambda i=i: ql.qlinear_quantize_act(xs[i], host_route, True, amax_in=amax[i],
-                                                                   out=qbufs[i])),
-            "gemm": launch_us(lambda i=i: ql.qlinear_gemm(host_route, qbufs[i], M_TOKENS, pws[i], Y=ys[i]))})
+            "amax": launch_us(f"amax{i}", lambda j: ql.qlinear_tensor_amax(rx[j % nx], True, out=amax[i],
+                                                                         ws=amax_ws[i])),
+            "quant": launch_us(f"quant{i}", lambda j: ql.qlinear_quantize_act(rx[j % nx], host_route, True,
+                                                                            amax_in=amax[i], out=rq[j % nx])),
+            "gemm": launch_us(f"gemm{i}", lambda j: ql.qlinear_gemm(host_route, rq[j % nx], M_TOKENS, pws[i],
+                                                                  Y=ry[j % ny])),
+            "rotation": {"x": nx, "y": ny}})
+        del rx, rq, ry
+    torch.cuda.synchronize()
+    ksampler.stop()
     assert ql.qlinear_device_status() == 0
+
+    def mhz(name):
+        sel = [smp for smp in getattr(ksampler, "samples", [])
+               if any(t0 <= smp[0] <= t1 for t0, t1 in windows[name])]
+        return statistics.median(smp[1] for smp in sel) if sel else None
 
     def tot(key, i):
         return kt[i][key] * 1e-3     # ms
 
     per = {}
     for i, (lin, _, _) in enumerate(lins):
-        per[lin.name] = {"amax_us": 1e3 * tot("amax", i), "quant_us": 1e3 * tot("quant", i),
-                         "gemm_us": 1e3 * tot("gemm", i),
-                         "gemm_tflops": 2.0 * M_TOKENS * lin.n * lin.k / (tot("gemm", i) * 1e-3) / 1e12}
+        per[lin.name] = {"amax_us": 1e3 * tot("amax", i), "amax_sm_mhz": mhz(f"amax{i}"),
+                         "quant_us": 1e3 * tot("quant", i), "quant_sm_mhz": mhz(f"quant{i}"),
+                         "gemm_us": 1e3 * tot("gemm", i), "gemm_sm_mhz": mhz(f"gemm{i}"),
+                         "gemm_tflops": 2.0 * M_TOKENS * lin.n * lin.k / (tot("gemm", i) * 1e-3) / 1e12,
+                         "rotation": kt[i]["rotation"]}
     gemm_ms = sum(tot("gemm", i) for i in range(len(lins)))
     quant_ms = sum(tot("quant", i) for i in range(len(lins)))
     amax_ms = sum(tot("amax", i) for i in range(len(lins)))
     elems = sum(M_TOKENS * lin.k for lin, _, _ in lins)
     peaks, peak_kind = measured_peaks()
-    peak_fp4 = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
+    # The per-kernel GEMM figures are short isolated replays: a burst
+    # measurement, so the denominator is the burst bf16 rate times the
+    # nominal FP4/BF16 ratio.  The sustained rate and the datasheet figure
+    # are carried beside it for context.
+    peak_fp4 = peaks["bf16_tflops"] * FP4_PER_BF16
+    peak_fp4_sustained = peaks["bf16_tflops_sustained"] * FP4_PER_BF16
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
     sha = gemm_source_sha()
     traffic = GEMM_TRAFFIC.get(sha)
@@ -396,16 +507,24 @@ def run_ours(args, rank, world, local):
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": peak_fp4, "unit": "TFLOP/s",
                      "frac": gemm_tflops / peak_fp4, "traffic": traffic,
                      "kernel": "k_gemm_w4a4 (all four linears)",
-                     "peak_note": f"{peak_kind} bf16 sustained x {FP4_PER_BF16:g} (nominal FP4/BF16)"},
+                     "peak_note": f"{peak_kind} bf16 burst x {FP4_PER_BF16:g} (nominal FP4/BF16): the GEMM times "
+                                  "are isolated CUDA-graph replays, a burst measurement",
+                     "frac_of_sustained_x4": gemm_tflops / peak_fp4_sustained,
+                     "frac_of_datasheet_fp4": gemm_tflops / FP4_DATASHEET_TFLOPS,
+                     "sm_mhz": [mhz(f"gemm{i}") for i in range(len(lins))]},
         "quant": {"kernel": "k_quant_nvfp4", "gbs": elems * NVFP4_BYTES_PER_ELEM / (quant_ms * 1e-3) / 1e9,
                   "hbm_frac": elems * NVFP4_BYTES_PER_ELEM / (quant_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                   "bytes_per_elem": NVFP4_BYTES_PER_ELEM},
-        "amax": {"kernel": "k_amax", "gbs": elems * 2.0 / (amax_ms * 1e-3) / 1e9},
-        "route_kernel": {"kernel": "k_gamma_route", "us": route_us,
+        "amax": {"kernel": "k_amax", "gbs": elems * 2.0 / (amax_ms * 1e-3) / 1e9,
+                 "hbm_frac": elems * 2.0 / (amax_ms * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "route_kernel": {"kernel": "k_gamma_route", "us": route_us, "sm_mhz": mhz("route"),
                          "gbs": 4.0 * M_TOKENS * 1920 / (route_us * 1e-6) / 1e9},
+        "amax_quant_share_of_step": (amax_ms + quant_ms) / (ms_max / args.steps),
         "per_linear": per,
         "gpu_launches": args.steps * (1 + 3 * len(lins)),
-        "timing": "step replayed as one CUDA graph; per-kernel figures from CUDA-graph replays of each kernel alone",
+        "timing": "step replayed as one CUDA graph; per-kernel figures: median of 8 bursts of about 25 ms of "
+                  "CUDA-graph replays of each kernel alone over rotating operand copies (> 2x L2 per replay), "
+                  "0.2 s of timing per kernel; SM clock = median nvidia-smi sample inside the bursts",
         "clocks": clocks,
         "gemm_source_sha": sha,
     }
@@ -584,60 +703,95 @@ def run_reference(args, rank, world):
 # --configs: every kernel of the five workload configurations
 # ---------------------------------------------------------------------------
 def run_configs(reps: int = 20):
-    """Device time (CUDA events around CUDA-graph replays of 10 launches,
-    median of `reps` replays) of each kernel of the five configurations,
-    with its roofline fraction: HBM
-    kernels against the measured copy bandwidth, GEMMs against the measured
-    sustained bf16 rate times the nominal ratio of their MMA kind (FP4 4x,
-    INT8 2x, f16 1x)."""
+    """Device time of each kernel of the five configurations with its
+    roofline fraction: HBM kernels against the measured copy bandwidth,
+    GEMMs against the measured burst bf16 rate times the nominal ratio of
+    their MMA kind (FP4 4x, INT8 2x, f16 1x; the kernels are timed alone in
+    short replays, a burst measurement).  Each kernel runs in a CUDA graph
+    of 12 launches that rotate over enough copies of its operands that one
+    replay touches more than twice the 126 MB L2; the figure is the median
+    over `reps` replays of the mean time per launch."""
     from bit_quantized_linear_block_b200 import qlinear as ql
     dev = torch.device("cuda", 0)
     peaks, kind = measured_peaks()
-    hbm, bf16 = peaks["hbm_gbs"], peaks["bf16_tflops_sustained"]
+    hbm, bf16 = peaks["hbm_gbs"], peaks["bf16_tflops"]
 
-    def med(fn, per_graph=10):
-        # Launches replayed from a CUDA graph (no host launch gaps): median
-        # over `reps` replays of the mean time per launch.
-        for _ in range(3):
-            fn()
+    def copies(t, nbytes):
+        """t and enough clones of it that the launches of one replay,
+        each moving nbytes, touch more than twice the L2."""
+        n = int(min(8, max(1, -(-2 * L2_BYTES // nbytes))))
+        return [t] + [t.clone() for _ in range(n - 1)]
+
+    sampler = ClockSampler(0)
+    sampler.start()
+    time.sleep(0.3)
+    pending = []   # (record, replay windows): the SM clock is filled in once sampling stops
+
+    def med(fn, per_graph=12, windows_n=8, window_s=0.025, pause_s=0.04):
+        # fn(j) enqueues launch j of the graph; `windows_n` replay windows of
+        # about `window_s` each, `pause_s` apart (0.2 s of timing with
+        # several clock samples); the median window's time per launch
+        for j in range(3):
+            fn(j)
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            for _ in range(per_graph):
-                fn()
+            for j in range(per_graph):
+                fn(j)
         graph.replay()
         torch.cuda.synchronize()
-        ts = []
-        for _ in range(reps):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        rp = max(3, int(window_s / max(1e-6, a.elapsed_time(b) * 1e-3)) + 1)
+        per, wins = [], []
+        for _ in range(windows_n):
+            time.sleep(pause_s)
+            th0 = time.time()
             a.record()
-            graph.replay()
+            for _ in range(rp):
+                graph.replay()
             b.record()
             torch.cuda.synchronize()
-            ts.append(a.elapsed_time(b) * 1e3 / per_graph)
+            wins.append((th0, time.time()))
+            per.append(a.elapsed_time(b) * 1e3 / (rp * per_graph))
         del graph
-        return statistics.median(ts)
+        return statistics.median(per), wins
 
-    def hbm_rec(us, nbytes):
-        return {"us": round(us, 2), "gbs": round(nbytes / us / 1e3, 1), "hbm_frac": round(nbytes / us / 1e3 / hbm, 3)}
+    def hbm_rec(t, nbytes):
+        us, wins = t
+        rec = {"us": round(us, 2), "gbs": round(nbytes / us / 1e3, 1), "hbm_frac": round(nbytes / us / 1e3 / hbm, 3)}
+        pending.append((rec, wins))
+        return rec
 
-    def mma_rec(us, m, n, k, ratio):
-        t = 2.0 * m * n * k / us / 1e6
-        return {"us": round(us, 2), "tflops": round(t, 1), "frac": round(t / (bf16 * ratio), 3)}
+    def mma_rec(t, m, n, k, ratio):
+        us, wins = t
+        tf = 2.0 * m * n * k / us / 1e6
+        rec = {"us": round(us, 2), "tflops": round(tf, 1), "frac": round(tf / (bf16 * ratio), 3)}
+        pending.append((rec, wins))
+        return rec
 
-    out = {"peaks": {"hbm_gbs": hbm, "bf16_tflops_sustained": bf16, "kind": kind}}
+    out = {"peaks": {"hbm_gbs": hbm, "bf16_tflops_burst": bf16, "kind": kind,
+                     "gemm_denominator": "burst bf16 x nominal ratio (FP4 4, INT8 2, f16/bf16 1)"}}
 
     def w4a4_linear(x, w, m, n, k):
         xd, wd = x.to(dev), w.to(dev)
         pw = ql.qlinear_prepare_weights(wd, ql.QL_W_NVFP4, hadamard=True)
         aws = torch.zeros(ql.lib.qlinear_quantize_ws_bytes(m, k, ql.QL_ROUTE_NVFP4), dtype=torch.uint8, device=dev)
         amax = ql.qlinear_tensor_amax(xd, True, ws=aws)
-        q = ql.qlinear_quantize_act(xd, ql.QL_ROUTE_NVFP4, True, rowmajor_scales=False, amax_in=amax)
-        y = ql.qlinear_gemm(ql.QL_ROUTE_NVFP4, q, m, pw)
-        rec = {"amax": hbm_rec(med(lambda: ql.qlinear_tensor_amax(xd, True, out=amax, ws=aws)), 2.0 * m * k),
-               "quant_nvfp4": hbm_rec(med(lambda: ql.qlinear_quantize_act(xd, ql.QL_ROUTE_NVFP4, True, amax_in=amax,
-                                                                          out=q)), NVFP4_BYTES_PER_ELEM * m * k),
-               "gemm_w4a4": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ROUTE_NVFP4, q, m, pw, Y=y)), m, n, k, 4.0)}
+        rx = copies(xd, 2.0 * m * k)
+        rq = [ql.qlinear_quantize_act(x_, ql.QL_ROUTE_NVFP4, True, rowmajor_scales=False, amax_in=amax) for x_ in rx]
+        y = ql.qlinear_gemm(ql.QL_ROUTE_NVFP4, rq[0], m, pw)
+        ry = copies(y, 2.0 * m * n + m * k / 2)
+        nx, ny = len(rx), len(ry)
+        rec = {"amax": hbm_rec(med(lambda j: ql.qlinear_tensor_amax(rx[j % nx], True, out=amax, ws=aws)), 2.0 * m * k),
+               "quant_nvfp4": hbm_rec(med(lambda j: ql.qlinear_quantize_act(rx[j % nx], ql.QL_ROUTE_NVFP4, True,
+                                                                            amax_in=amax, out=rq[j % nx])),
+                                      NVFP4_BYTES_PER_ELEM * m * k),
+               "gemm_w4a4": mma_rec(med(lambda j: ql.qlinear_gemm(ql.QL_ROUTE_NVFP4, rq[j % nx], m, pw,
+                                                                   Y=ry[j % ny])), m, n, k, 4.0)}
         return rec
 
     # 1: single linear [256,1920] x [1920,1920]
@@ -647,6 +801,7 @@ def run_configs(reps: int = 20):
     for lin in S.COGVIDEOX_2B:
         x, w = S.cogvideox2b_linear(lin)
         out[f"cfg2_{lin.name}"] = w4a4_linear(x, w, M_TOKENS, lin.n, lin.k)
+        torch.cuda.empty_cache()
     # 3: routing sweep (4 of the 30 blocks for timing) and the INT8-routed FFN-up
     wd = S.dmpq_ffn_up_weights().to(dev)
     pw = ql.qlinear_prepare_weights(wd, ql.QL_W_NVFP4, hadamard=True)
@@ -658,31 +813,45 @@ def run_configs(reps: int = 20):
         rws = torch.zeros(ql.lib.qlinear_route_ws_bytes(bi.numel()), dtype=torch.uint8, device=dev)
         g, r = ql.qlinear_route(bi, bo, THRESHOLD, ws=rws)
         gg, rr = g.clone(), r.clone()
-        us = med(lambda: ql.qlinear_route(bi, bo, THRESHOLD, gamma=gg, route=rr, ws=rws))
+        ri, ro = copies(bi, 4.0 * bi.numel()), copies(bo, 4.0 * bi.numel())
+        us = med(lambda j: ql.qlinear_route(ri[j % len(ri)], ro[j % len(ri)], THRESHOLD, gamma=gg, route=rr, ws=rws))
         routes[f"block{blk}"] = dict(hbm_rec(us, 4.0 * M_TOKENS * 1920), sigma=round(sigma, 5),
                                      gamma=float(g.item()), route=int(r.item()))
+        del ri, ro
     out["cfg3_route"] = routes
-    q = ql.qlinear_quantize_act(bi, ql.QL_ROUTE_INT8, True)
-    q16 = ql.qlinear_quantize_act(bi, ql.QL_ACT_INT8_F16, True)
-    y = ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, M_TOKENS, pw)
+    rx = copies(bi, 2.0 * bi.numel())
+    nx = len(rx)
+    q = [ql.qlinear_quantize_act(x_, ql.QL_ROUTE_INT8, True) for x_ in rx]
+    q16 = [ql.qlinear_quantize_act(x_, ql.QL_ACT_INT8_F16, True) for x_ in rx]
+    y = ql.qlinear_gemm(ql.QL_ROUTE_INT8, q[0], M_TOKENS, pw)
+    ry = copies(y, 2.0 * y.numel())
+    ny = len(ry)
     out["cfg3_int8_ffn_up"] = {
-        # the path qlinear_forward takes with an f16 weight copy: f16-coded INT8 activations
-        "quant_int8_token_f16": hbm_rec(med(lambda: ql.qlinear_quantize_act(bi, ql.QL_ACT_INT8_F16, True, out=q16)),
+        # the path qlinear_forward takes: f16-coded INT8 activations ...
+        "quant_int8_token_f16": hbm_rec(med(lambda j: ql.qlinear_quantize_act(rx[j % nx], ql.QL_ACT_INT8_F16, True,
+                                                                             out=q16[j % nx])),
                                         M_TOKENS * 1920 * (4.0 + 4.0 / 1920)),
-        "gemm_w4a8": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q16, M_TOKENS, pwx, Y=y)),
-                             M_TOKENS, 7680, 1920, 1.0),
-        # int8 codes, FP4 weights expanded on chip (no f16 weight copy)
-        "quant_int8_token": hbm_rec(med(lambda: ql.qlinear_quantize_act(bi, ql.QL_ROUTE_INT8, True, out=q)),
+        # ... into the GEMM with the NVFP4 weights widened on chip into tensor memory (no weight copy)
+        "gemm_w4a8_onchip": mma_rec(med(lambda j: ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q16[j % nx], M_TOKENS, pw,
+                                                                   Y=ry[j % ny])), M_TOKENS, 7680, 1920, 1.0),
+        # ... or into the GEMM with the f16 weight copy (expand_f16)
+        "gemm_w4a8_f16copy": mma_rec(med(lambda j: ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q16[j % nx], M_TOKENS, pwx,
+                                                                    Y=ry[j % ny])), M_TOKENS, 7680, 1920, 1.0),
+        # int8 codes, both operands widened on chip in shared memory (qlinear_gemm only)
+        "quant_int8_token": hbm_rec(med(lambda j: ql.qlinear_quantize_act(rx[j % nx], ql.QL_ROUTE_INT8, True,
+                                                                         out=q[j % nx])),
                                     M_TOKENS * 1920 * (3.0 + 4.0 / 1920)),
-        "gemm_w4a8_onchip": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, M_TOKENS, pw, Y=y)),
-                                    M_TOKENS, 7680, 1920, 1.0)}
+        "gemm_w4a8_onchip_smem": mma_rec(med(lambda j: ql.qlinear_gemm(ql.QL_ROUTE_INT8, q[j % nx], M_TOKENS, pw,
+                                                                        Y=ry[j % ny])), M_TOKENS, 7680, 1920, 1.0)}
     # PDR's BF16 refresh: the unquantized product of the same FFN-up (bf16
     # input and kept bf16 weights, kind::f16 with bf16 operands)
     pwb = ql.qlinear_prepare_weights(wd, ql.QL_W_NVFP4, hadamard=True, keep_bf16=True)
     out["cfg3_int8_ffn_up"]["gemm_bf16"] = mma_rec(
-        med(lambda: ql.qlinear_gemm(ql.QL_ROUTE_BF16, {"codes": bi, "scales": None}, M_TOKENS, pwb, Y=y)),
+        med(lambda j: ql.qlinear_gemm(ql.QL_ROUTE_BF16, {"codes": rx[j % nx], "scales": None}, M_TOKENS, pwb,
+                                      Y=ry[j % ny])),
         M_TOKENS, 7680, 1920, 1.0)
-    del bi, bo, q, q16, y, pw, pwx, pwb, wd
+    del bi, bo, q, q16, y, pw, pwx, pwb, wd, rx, ry
+    torch.cuda.empty_cache()
     # Temporal delta cache on a sweep block pair [17776, 1920] (6Bit-Diffusion,
     # B.2): the fused refresh reads in, out and the latest delta and writes
     # the new delta (8 B/elem); the skip reads in and the delta and writes
@@ -690,12 +859,18 @@ def run_configs(reps: int = 20):
     bi, bo, _ = S.dmpq_block_pair(0)
     bi, bo = bi.to(dev), bo.to(dev)
     nel = bi.numel()
-    cache = ql.TdcCache(nel, dev)
-    ql.qlinear_tdc_refresh(bi, bo, cache)        # a delta is cached: the timed refreshes read it
-    ys = torch.empty_like(bi)
-    out["tdc"] = {"refresh": hbm_rec(med(lambda: ql.qlinear_tdc_refresh(bi, bo, cache)), 8.0 * nel),
-                  "skip": hbm_rec(med(lambda: ql.qlinear_tdc_skip(bi, cache, out=ys)), 6.0 * nel)}
-    del bi, bo, ys, cache
+    ri, ro = copies(bi, 8.0 * nel), copies(bo, 8.0 * nel)
+    caches = [ql.TdcCache(nel, dev) for _ in ri]
+    for c_, i_, o_ in zip(caches, ri, ro):
+        ql.qlinear_tdc_refresh(i_, o_, c_)        # a delta is cached: the timed refreshes read it
+    ys = [torch.empty_like(bi) for _ in ri]
+    nr = len(ri)
+    out["tdc"] = {"refresh": hbm_rec(med(lambda j: ql.qlinear_tdc_refresh(ri[j % nr], ro[j % nr], caches[j % nr])),
+                                     8.0 * nel),
+                  "skip": hbm_rec(med(lambda j: ql.qlinear_tdc_skip(ri[j % nr], caches[j % nr], out=ys[j % nr])),
+                                  6.0 * nel)}
+    del bi, bo, ys, caches, ri, ro
+    torch.cuda.empty_cache()
     # Activation decomposition (SemanticDialect 2.2) on the CogVideoX-2B FFN
     # linears: the quantizer reads 2 B/elem and writes both levels' codes and
     # scales (1 + 1/8 B/elem); the GEMM contracts over K' = 2K
@@ -706,14 +881,21 @@ def run_configs(reps: int = 20):
         aws = torch.zeros(ql.lib.qlinear_quantize_ws_bytes(M_TOKENS, lin.k, ql.QL_ROUTE_NVFP4), dtype=torch.uint8,
                           device=dev)
         amax = ql.qlinear_tensor_amax(xd, True, ws=aws)
-        q = ql.qlinear_quantize_act(xd, ql.QL_ACT_NVFP4_DECOMP, True, rowmajor_scales=False, amax_in=amax)
-        y = ql.qlinear_gemm(ql.QL_ACT_NVFP4_DECOMP, q, M_TOKENS, pwd)
+        rx = copies(xd, 2.0 * xd.numel())
+        nx = len(rx)
+        q = [ql.qlinear_quantize_act(x_, ql.QL_ACT_NVFP4_DECOMP, True, rowmajor_scales=False, amax_in=amax)
+             for x_ in rx]
+        y = ql.qlinear_gemm(ql.QL_ACT_NVFP4_DECOMP, q[0], M_TOKENS, pwd)
+        ry = copies(y, 2.0 * y.numel() + xd.numel())
+        ny = len(ry)
         out[f"decomp_{lin.name}"] = {
-            "quant_nvfp4_decomp": hbm_rec(med(lambda: ql.qlinear_quantize_act(
-                xd, ql.QL_ACT_NVFP4_DECOMP, True, amax_in=amax, out=q)), 3.125 * M_TOKENS * lin.k),
-            "gemm_w4a4_2k": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ACT_NVFP4_DECOMP, q, M_TOKENS, pwd, Y=y)),
+            "quant_nvfp4_decomp": hbm_rec(med(lambda j: ql.qlinear_quantize_act(
+                rx[j % nx], ql.QL_ACT_NVFP4_DECOMP, True, amax_in=amax, out=q[j % nx])), 3.125 * M_TOKENS * lin.k),
+            "gemm_w4a4_2k": mma_rec(med(lambda j: ql.qlinear_gemm(ql.QL_ACT_NVFP4_DECOMP, q[j % nx], M_TOKENS, pwd,
+                                                                   Y=ry[j % ny])),
                                     M_TOKENS, lin.n, 2 * lin.k, 4.0)}
-        del xd, wd, pwd, q, y
+        del xd, wd, pwd, q, y, rx, ry
+        torch.cuda.empty_cache()
     # 4: CogVideoX-5B linears, Q-ARVD dual-scale weights, per-tensor INT8
     for lin in S.COGVIDEOX_5B:
         x, w = S.cogvideox5b_qarvd_linear(lin)
@@ -724,28 +906,41 @@ def run_configs(reps: int = 20):
         aws = torch.zeros(ql.lib.qlinear_quantize_ws_bytes(M_TOKENS, lin.k, ql.QL_ROUTE_NVFP4), dtype=torch.uint8,
                           device=dev)
         amax = ql.qlinear_tensor_amax(xd, False, ws=aws)
-        q = ql.qlinear_quantize_act(xd, ql.QL_ACT_INT8_TENSOR, False, w=pw, amax_in=amax)
-        y = ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q, M_TOKENS, pw)
+        rx = copies(xd, 2.0 * xd.numel())
+        nx = len(rx)
+        q = [ql.qlinear_quantize_act(x_, ql.QL_ACT_INT8_TENSOR, False, w=pw, amax_in=amax) for x_ in rx]
+        y = ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q[0], M_TOKENS, pw)
+        ry = copies(y, 2.0 * y.numel() + M_TOKENS * kp)
+        ny = len(ry)
         out[f"cfg4_{lin.name}"] = {
-            "amax": hbm_rec(med(lambda: ql.qlinear_tensor_amax(xd, False, out=amax, ws=aws)), 2.0 * M_TOKENS * lin.k),
-            "quant_int8_tensor": hbm_rec(med(lambda: ql.qlinear_quantize_act(xd, ql.QL_ACT_INT8_TENSOR, False, w=pw,
-                                                                              amax_in=amax, out=q)),
+            "amax": hbm_rec(med(lambda j: ql.qlinear_tensor_amax(rx[j % nx], False, out=amax, ws=aws)),
+                            2.0 * M_TOKENS * lin.k),
+            "quant_int8_tensor": hbm_rec(med(lambda j: ql.qlinear_quantize_act(rx[j % nx], ql.QL_ACT_INT8_TENSOR,
+                                                                              False, w=pw, amax_in=amax,
+                                                                              out=q[j % nx])),
                                          M_TOKENS * (2.0 * lin.k + kp)),
             # int8 weight copy: both operands by TMA
-            "gemm_qarvd": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q, M_TOKENS, pw8, Y=y)),
-                                  M_TOKENS, lin.n, lin.k, 2.0),
-            # INT4 codes widened on chip
-            "gemm_qarvd_onchip": mma_rec(med(lambda: ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q, M_TOKENS, pw, Y=y)),
+            "gemm_qarvd": mma_rec(med(lambda j: ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q[j % nx], M_TOKENS, pw8,
+                                                                 Y=ry[j % ny])), M_TOKENS, lin.n, lin.k, 2.0),
+            # INT4 codes widened on chip into tensor memory (no int8 copy; the form qlinear_forward takes)
+            "gemm_qarvd_onchip": mma_rec(med(lambda j: ql.qlinear_gemm(ql.QL_ACT_INT8_TENSOR, q[j % nx], M_TOKENS,
+                                                                        pw, Y=ry[j % ny])),
                                          M_TOKENS, lin.n, lin.k, 2.0)}
-        del xd, wd, pw, pw8, q, y
+        del xd, wd, pw, pw8, q, y, rx, ry
+        torch.cuda.empty_cache()
     # 5: Wan-14B linears
     for lin in S.WAN_14B:
         x, w = S.wan14b_linear(lin)
         out[f"cfg5_{lin.name}"] = w4a4_linear(x, w, S.M_WAN, lin.n, lin.k)
         torch.cuda.empty_cache()
     out["device_status"] = ql.qlinear_device_status()
+    sampler.stop()
+    for rec, wins in pending:   # median SM clock over the record's replay windows
+        sel = [smp[1] for smp in getattr(sampler, "samples", []) if any(t0 <= smp[0] <= t1 for t0, t1 in wins)]
+        rec["sm_mhz"] = statistics.median(sel) if sel else None
+    out["peaks"]["timing"] = ("median of 8 windows of about 25 ms of CUDA-graph replays of the kernel alone, 40 ms "
+                              "apart; sm_mhz = median nvidia-smi sample inside the windows")
     return out
-
 
 
 def main():

@@ -184,6 +184,9 @@ W4A4_CASES = [
     (300, 1040, 640),    # ragged last 192-wide tile, N not a multiple of 128 (padded scale rows)
     (520, 5120, 2048),   # ragged 192-wide tiles with streamed scales (the Wan-14B FFN-down form)
     (100, 1040, 2048),   # one SM per tile (M <= 128), ragged, streamed scales
+    (2048, 384, 1920),   # two N tiles per row block: the resident A panel reloaded many times per unit
+    (4000, 192, 256),    # one N tile per row block, ragged M, one K chunk
+    (600, 1920, 7680),   # streamed 256-wide tiles, ragged last tile (N = 7.5 tiles), long K
 ]
 
 
@@ -232,7 +235,9 @@ def test_gemm_timeout_path_reports_and_recovers(ql):
 
 # ---------------------------------------------------------------- W4A8 (INT8 route)
 
-W4A8_CASES = [(256, 1920, 1920), (300, 384, 640), (129, 640, 384), (1000, 5760, 1920), (1, 192, 128)]
+W4A8_CASES = [(256, 1920, 1920), (300, 384, 640), (129, 640, 384), (1000, 5760, 1920), (1, 192, 128),
+              (2048, 576, 1024),   # several tiles per CTA (persistent loop over both accumulators)
+              (700, 320, 256)]     # 128-wide tiles, the last one half past N
 
 
 @pytest.mark.parametrize("expand", [False, True])
@@ -256,18 +261,56 @@ def test_forward_w4a8_int8_route_parity(ql, m, n, k, expand):
     yn = _np(y.float())[rows].astype(np.float64)
     assert np.isfinite(yn).all()
     assert excess_err(yn, ref) <= 1e-5
-    if expand:   # int8 codes through qlinear_gemm: on-chip A expansion, f16 weight copy
-        q = ql.qlinear_quantize_act(x.cuda(), ql.QL_ROUTE_INT8, hadamard=True)
-        y2 = ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, m, pw)
-        # the same codes stored as f16 values, both GEMM operands by TMA
-        q3 = ql.qlinear_quantize_act(x.cuda(), ql.QL_ACT_INT8_F16, hadamard=True)
-        y3 = ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q3, m, pw)
-        torch.cuda.synchronize()
-        assert ql.qlinear_device_status() == 0
-        assert np.array_equal(_np(q3["codes"].float()), _np(q["codes"].float()))
-        assert np.array_equal(_np(q3["scales"]), _np(q["scales"]))
-        assert excess_err(_np(y2.float())[rows].astype(np.float64), ref) <= 1e-5
-        assert excess_err(_np(y3.float())[rows].astype(np.float64), ref) <= 1e-5
+    # int8 codes through qlinear_gemm: both operands widened on chip (no copy)
+    # or the activations widened next to the f16 weight copy
+    q = ql.qlinear_quantize_act(x.cuda(), ql.QL_ROUTE_INT8, hadamard=True)
+    y2 = ql.qlinear_gemm(ql.QL_ROUTE_INT8, q, m, pw)
+    # the same codes stored as f16 values: with the copy both operands by TMA,
+    # without it the weights widened into tensor memory (the MMA's A operand)
+    q3 = ql.qlinear_quantize_act(x.cuda(), ql.QL_ACT_INT8_F16, hadamard=True)
+    y3 = ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q3, m, pw)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    assert np.array_equal(_np(q3["codes"].float()), _np(q["codes"].float()))
+    assert np.array_equal(_np(q3["scales"]), _np(q["scales"]))
+    assert excess_err(_np(y2.float())[rows].astype(np.float64), ref) <= 1e-5
+    assert excess_err(_np(y3.float())[rows].astype(np.float64), ref) <= 1e-5
+    assert torch.equal(y3, y)   # the forward takes the f16-coded form
+
+
+@pytest.mark.parametrize("m,n,k", [(300, 384, 640), (1, 320, 256), (700, 1040, 1024), (2000, 1920, 1920),
+                                   (193, 128, 7680)])
+def test_w4a8_forms_agree(ql, m, n, k):
+    """The four INT8-route GEMM forms multiply the same exact f16 values with
+    fp32 accumulation: weights widened into tensor memory (f16 codes, no
+    copy), both operands widened on chip (int8 codes, no copy), and the f16
+    weight copy with f16 or int8 codes.  Each is held to the oracle's product
+    and all four must give the same bits.  Shapes: ragged token tiles (193,
+    300, 700, 2000 rows against 192-row tiles), weight tiles past N (320,
+    1040), one K stage per scale atom up to K = 7680."""
+    x = _x(m, k, seed=m + 5 * n + k)
+    w = S.weights(n, k, 0.02, 8, m + 2 * n + k)
+    xb, wb = S.bf16_bits(x), S.bf16_bits(w)
+    wq = O.prepare_weights_nvfp4(wb)
+    rows = np.arange(m) if m <= 512 else np.unique(np.r_[np.random.default_rng(2).choice(m, 256, replace=False), m - 1])
+    ref = O.forward(xb, wq, O.ROUTE_INT8, rows=rows)
+    pw = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True)
+    pwx = ql.qlinear_prepare_weights(w.cuda(), ql.QL_W_NVFP4, hadamard=True, expand_f16=True)
+    xc = x.cuda()
+    q8 = ql.qlinear_quantize_act(xc, ql.QL_ROUTE_INT8, hadamard=True)
+    q16 = ql.qlinear_quantize_act(xc, ql.QL_ACT_INT8_F16, hadamard=True)
+    ys = {"tmem": ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q16, m, pw),
+          "onchip": ql.qlinear_gemm(ql.QL_ROUTE_INT8, q8, m, pw),
+          "copy_f16": ql.qlinear_gemm(ql.QL_ACT_INT8_F16, q16, m, pwx),
+          "copy_int8": ql.qlinear_gemm(ql.QL_ROUTE_INT8, q8, m, pwx)}
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    for name, y in ys.items():
+        yn = _np(y.float())[rows].astype(np.float64)
+        assert np.isfinite(yn).all(), name
+        assert excess_err(yn, ref) <= 1e-5, name
+    for name, y in ys.items():
+        assert torch.equal(y, ys["copy_f16"]), name
 
 
 # ---------------------------------------------------------------- Q-ARVD
@@ -338,6 +381,40 @@ def test_qarvd_activation_quant_and_forward_parity(ql, m, n, k, frac, expand):
     assert excess_err(_np(y.float()).astype(np.float64), ref) <= 1e-5
 
 
+@pytest.mark.parametrize("m,n,k,frac,seed", [(300, 384, 384, 0.05, 3), (77, 128, 128, 0.05, 4),
+                                             (700, 640, 3072, 0.02, 5), (256, 256, 640, 0.0, 5),
+                                             (1000, 200, 1024, 0.05, 6)])
+def test_qarvd_forms_agree(ql, m, n, k, frac, seed):
+    """The INT4 weights widened on chip into tensor memory and the int8
+    weight copy multiply the same integers with exact int32 accumulation and
+    the same epilogue rounding: identical outputs, each held to the oracle.
+    Shapes: ragged 128-token tiles (77, 300, 700, 1000), weight tiles past N
+    (200, 640), a weight set without outlier channels (frac 0: the outlier
+    class is empty), and an outlier class that follows a partial K stage."""
+    w = S.weights(n, k, 0.02, seed, 77, outlier_frac=frac, outlier_scale=20.0)
+    pk = O.qarvd_pack(S.bf16_bits(w), 3.5, 2.0)
+    _assert_guard_band(pk)
+    if frac == 0.0:
+        assert pk["n_out"] == 0
+    x = _x(m, k, seed=m + 3 * k)
+    qx, sx = O.int8_per_tensor(O.bf16_bits_to_f32(S.bf16_bits(x)))
+    qxp = O.qarvd_permute_activations(qx, pk["perm"], pk["k_norm"], pk["k_norm_pad"], pk["n_out"], pk["k_out_pad"])
+    ref = O.gemm_qarvd(qxp, sx, pk["codes"], pk["s_norm"], pk["s_out"], pk["k_norm_pad"])
+    wc = w.cuda()
+    pw = ql.qlinear_prepare_weights(wc, ql.QL_W_QARVD_INT4, hadamard=False)
+    pw8 = ql.qlinear_prepare_weights(wc, ql.QL_W_QARVD_INT4, hadamard=False, expand_i8=True)
+    xc = x.cuda()
+    y_tmem = ql.qlinear_forward(xc, pw)
+    y_copy = ql.qlinear_forward(xc, pw8)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    for y in (y_tmem, y_copy):
+        yn = _np(y.float()).astype(np.float64)
+        assert np.isfinite(yn).all()
+        assert excess_err(yn, ref) <= 1e-5
+    assert torch.equal(y_tmem, y_copy)
+
+
 # ---------------------------------------------------------------- W4A6 (INT6 activations)
 
 @pytest.mark.parametrize("expand", [False, True])
@@ -363,12 +440,13 @@ def test_w4a6_token_route_parity(ql, m, n, k, expand):
     assert np.abs(q6.astype(int)).max() <= 31
     assert excess_err(_np(y.float()).astype(np.float64), ref) <= 1e-5
     assert excess_err(_np(y2.float()).astype(np.float64), ref) <= 1e-5
-    if expand:
-        qf = ql.qlinear_quantize_act(xc, ql.QL_ACT_INT6_F16, hadamard=True)
-        y3 = ql.qlinear_gemm(ql.QL_ACT_INT6_F16, qf, m, pw)
-        torch.cuda.synchronize()
-        assert np.array_equal(_np(qf["codes"].float()), q6.astype(np.float32))
-        assert excess_err(_np(y3.float()).astype(np.float64), ref) <= 1e-5
+    qf = ql.qlinear_quantize_act(xc, ql.QL_ACT_INT6_F16, hadamard=True)
+    y3 = ql.qlinear_gemm(ql.QL_ACT_INT6_F16, qf, m, pw)
+    torch.cuda.synchronize()
+    assert ql.qlinear_device_status() == 0
+    assert np.array_equal(_np(qf["codes"].float()), q6.astype(np.float32))
+    assert excess_err(_np(y3.float()).astype(np.float64), ref) <= 1e-5
+    assert torch.equal(y3, y)   # the forward quantizes to f16-coded INT6
 
 
 @pytest.mark.parametrize("expand", [False, True])
