@@ -8,51 +8,19 @@
 // is a contiguous, MMA-aligned K range and gets its own int32 accumulator:
 //   Y[m, n] = bf16(s_x * (s_norm[n] * acc_normal[m, n] + s_out[n] * acc_outlier[m, n])).
 // The MMA is tcgen05 kind::i8 (int32 accumulation, exact).  Two kernels:
+//   k_gemm_qarvd_ts   INT4 weights widened on chip into tensor memory as the
+//                     MMA's A operand (described further down);
 //   k_gemm_qarvd_pre  weights kept as int8 (expand_i8): CTA pairs, both
-//                     operands by TMA (described further down);
-//   k_gemm_qarvd      INT4 weights widened on chip, below.
+//                     operands by TMA (described further down).
 // Activations may carry INT8 or INT6 codes (W4A6); the product is the same.
-//
-// k_gemm_qarvd: persistent, warp-specialized, one CTA (512 threads) per SM:
-//   warps 0-7   transform: INT4 nibbles -> sign-extended int8 in the
-//               128-byte-swizzled K-major layout;
-//   warp 8      TMA producer: int8 activations straight into the MMA layout
-//               (128-byte swizzle), raw INT4 weight tiles;
-//   warp 9      MMA issuer (each 32-wide K step goes to its class's accumulator);
-//   warp 10     TMEM allocator (2 tiles x 2 classes x 128 columns = 512);
-//   warps 12-15 epilogue (column scales staged in shared memory per tile).
 #include "ql_common.cuh"
 #include "gemm_common.cuh"
 #include "launchers.h"
 
 namespace ql {
 
-template <int S>
-struct QarvdCfg {
-  static constexpr int BM = 128, BN = 128;
-  static constexpr int BK = 128;                 // K bytes (= int8 elements) per stage
-  static constexpr int CONV_A = BM * BK;         // int8, swizzled, written by TMA
-  static constexpr int CONV_B = BN * BK;         // int8, swizzled, written by the transform
-  static constexpr int RAW_B = BN * BK / 2;      // INT4
-  static constexpr int OFF_CA = 0;
-  static constexpr int OFF_CB = OFF_CA + S * CONV_A;
-  static constexpr int OFF_C = OFF_CB + S * CONV_B;
-  static constexpr int OFF_RB = OFF_C + 2 * kEpiChunkBytes;
-  static constexpr int OFF_CS = OFF_RB + S * RAW_B;          // column scales: 2 x BN floats
-  static constexpr int OFF_BAR = OFF_CS + 2 * BN * 4;
-  static constexpr int NBAR = 4 * S + 2 * 2 + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  static constexpr int XFORM_THREADS = 256;
-  static_assert(SMEM <= 232448, "shared memory budget");
-  // kind::i8 descriptor: D = S32 (2 at bit 4), A = B = signed int8 (1),
-  // K-major, N >> 3 at bit 17, M >> 4 at bit 24.
-  static constexpr uint32_t IDESC =
-      (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
-};
-
 // Eight two's-complement nibbles (byte j: elements 2j low, 2j+1 high) ->
-// eight int8 in element order.
+// eight int8 in element order (the int8 weight copy).
 __device__ __forceinline__ uint2 int4x8_to_int8(uint32_t w) {
   uint32_t lo = w & 0x0F0F0F0Fu;             // elements 0, 2, 4, 6
   uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;      // elements 1, 3, 5, 7
@@ -61,236 +29,12 @@ __device__ __forceinline__ uint2 int4x8_to_int8(uint32_t w) {
   return make_uint2(__byte_perm(lo, hi, 0x5140u), __byte_perm(lo, hi, 0x7362u));
 }
 
-__device__ __forceinline__ uint32_t sw128q(uint32_t r, uint32_t c) {
-  return r * 128u + ((c ^ (r & 7u)) << 4);
-}
-
 __device__ __forceinline__ bool warp_wait2q(uint64_t* a, uint32_t pa, uint64_t* b, uint32_t pb,
                                             long long limit, volatile int* abort_flag) {
   int ok = 0;
   if (lane_id() == 0)
     ok = (*abort_flag == 0) && mbar_wait(a, pa, limit) && mbar_wait(b, pb, limit);
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
-template <int S>
-__global__ void __launch_bounds__(512, 1)
-    k_gemm_qarvd(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                 const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
-  using C = QarvdCfg<S>;
-  constexpr int BN = C::BN;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align_1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);     // A (TMA) + raw B (TMA)
-  uint64_t* raw_empty = full + S;                                     // transform done with raw B
-  uint64_t* conv_full = raw_empty + S;                                // transform wrote B
-  uint64_t* empty = conv_full + S;                                    // MMA done with the stage
-  uint64_t* tfull = empty + S;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-
-  pdl_wait();   // before the first global access
-  // Class sizes (device-resident, written by the weight preparation).
-  const int k_norm_pad = p.kinfo[1];
-  const int k_out_pad = p.kinfo[3];
-  const int k_used = k_norm_pad + k_out_pad;
-  const int num_kst = (k_used + C::BK - 1) / C::BK;
-
-  const int warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) {
-    prefetch_tmap(&tm_a);
-    prefetch_tmap(&tm_b);
-    prefetch_tmap(&tm_y);
-    for (int i = 0; i < S; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&raw_empty[i], C::XFORM_THREADS / 32);
-      mbar_init(&conv_full[i], C::XFORM_THREADS / 32);
-      mbar_init(&empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 10) tmem_alloc(tmem_slot, 512);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp < 8) {
-    // ------------------------------------------------------------ transform
-    const uint32_t tid = threadIdx.x;
-    int it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-      for (int ks = 0; ks < num_kst; ++ks, ++it) {
-        const int s = it % S;
-        const uint32_t ph = (it / S) & 1;
-        // raw B landed (full) and the MMA is done with this stage's B (empty)
-        if (!warp_wait2q(&full[s], ph, &empty[s], ph ^ 1, p.wait_limit, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const uint8_t* rb = smem + C::OFF_RB + s * C::RAW_B;
-        uint8_t* cb = smem + C::OFF_CB + s * C::CONV_B;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {   // BN rows x 8 chunks of 16 int8 (8 raw bytes)
-          const uint32_t idx = tid + C::XFORM_THREADS * i;
-          const uint32_t r = idx >> 3, c = idx & 7u;
-          const uint2 q = *reinterpret_cast<const uint2*>(rb + idx * 8);
-          const uint2 a = int4x8_to_int8(q.x);
-          const uint2 b = int4x8_to_int8(q.y);
-          *reinterpret_cast<uint4*>(cb + sw128q(r, c)) = make_uint4(a.x, a.y, b.x, b.y);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane_id() == 0) {
-          mbar_arrive(&raw_empty[s]);
-          mbar_arrive(&conv_full[s]);
-        }
-      }
-    }
-    if (!ok && lane_id() == 0) fail_timeout(p.status, abort_flag);
-  } else if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    if (elect_one()) {
-      int it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        int mb, nb;
-        tile_coords(t, p, mb, nb);
-        for (int ks = 0; ks < num_kst; ++ks, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
-          // the MMA is done with A (empty) and the transform with raw B (raw_empty)
-          if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1, p.wait_limit) ||
-              !mbar_wait(&raw_empty[s], ph ^ 1, p.wait_limit)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[s], C::CONV_A + C::RAW_B);
-          tma_load_2d(smem + C::OFF_CA + s * C::CONV_A, &tm_a, &full[s], ks * C::BK, mb * C::BM);
-          tma_load_2d(smem + C::OFF_RB + s * C::RAW_B, &tm_b, &full[s], ks * (C::BK / 2), nb * BN);
-        }
-      }
-      if (!ok) fail_timeout(p.status, abort_flag);
-      drain_loads(full, it, S, p.status);
-    }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
-      int it = 0, local = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
-        const int acc = local & 1;
-        const uint32_t aph = (local >> 1) & 1;
-        if (*abort_flag || !mbar_wait(&tempty[acc], aph ^ 1, p.wait_limit)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_norm = tmem + acc * 2 * BN;
-        const uint32_t d_out = d_norm + BN;
-        bool started_norm = false, started_out = false;
-        for (int ks = 0; ks < num_kst; ++ks, ++it) {
-          const int s = it % S;
-          const uint32_t ph = (it / S) & 1;
-          if (*abort_flag || !mbar_wait(&conv_full[s], ph, p.wait_limit)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + C::OFF_CA + s * C::CONV_A);
-          const uint32_t b_base = smem_u32(smem + C::OFF_CB + s * C::CONV_B);
-#pragma unroll
-          for (int i = 0; i < C::BK / 32; ++i) {
-            const int kk = ks * C::BK + 32 * i;
-            if (kk >= k_used) break;
-            const bool normal = kk < k_norm_pad;
-            const uint64_t adesc = smem_desc(a_base + 32 * i, 0, 1024, kSwizzle128B);
-            const uint64_t bdesc = smem_desc(b_base + 32 * i, 0, 1024, kSwizzle128B);
-            tc_mma_i8(normal ? d_norm : d_out, adesc, bdesc, C::IDESC,
-                      (normal ? started_norm : started_out) ? 1u : 0u);
-            if (normal) started_norm = true; else started_out = true;
-          }
-          tc_commit(&empty[s]);
-        }
-        if (!ok) break;
-        tc_commit(&tfull[acc]);
-      }
-      if (!ok) fail_timeout(p.status, abort_flag);
-      drain_mma(drain, p.status);
-    }
-  } else if (warp >= 12) {
-    // ------------------------------------------------------------ epilogue
-    const float sx = ld_dep(p.g_a);
-    const int ew = warp & 3;
-    const int lane = lane_id();
-    const int row = threadIdx.x & 127;
-    float* cs = reinterpret_cast<float*>(smem + C::OFF_CS);
-    EpilogueState es{};
-    int local = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
-      int mb, nb;
-      tile_coords(t, p, mb, nb);
-      const int acc = local & 1;
-      const uint32_t aph = (local >> 1) & 1;
-      // column scales of this tile (columns past N read as 0)
-      const int n = nb * BN + row;
-      const float sn = (n < p.N) ? __ldg(p.col_scale0 + n) : 0.f;
-      const float so = (n < p.N) ? __ldg(p.col_scale1 + n) : 0.f;
-      if (!epilogue_wait_uniform(&tfull[acc], aph, p.wait_limit, abort_flag, p.status)) break;
-      cs[row] = sn;           // safe: the previous tile's readers passed the barrier above
-      cs[BN + row] = so;
-      named_bar_sync(1, 128);
-      tc_fence_after();
-      const uint32_t base = tmem + acc * 2 * BN + (static_cast<uint32_t>(ew * 32) << 16);
-#pragma unroll 1
-      for (int c = 0; c < BN / kEpiChunkCols; ++c) {
-        uint32_t packed[32];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t an[32], ao[32];
-          const uint32_t col = c * kEpiChunkCols + h * 32;
-          tmem_ld32(base + col, an);
-          tmem_ld32(base + BN + col, ao);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float y[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int jj = 2 * j + e;
-              const float fn = k_norm_pad ? static_cast<float>(static_cast<int32_t>(an[jj])) : 0.f;
-              const float fo = k_out_pad ? static_cast<float>(static_cast<int32_t>(ao[jj])) : 0.f;
-              const float v = __fadd_rn(__fmul_rn(cs[col + jj], fn), __fmul_rn(cs[BN + col + jj], fo));
-              y[e] = __fmul_rn(sx, v);
-            }
-            packed[16 * h + j] = pack_bf16x2(y[0], y[1]);
-          }
-        }
-        if (c == BN / kEpiChunkCols - 1) {
-          tc_fence_before();
-          if (lane == 0) mbar_arrive(&tempty[acc]);
-        }
-        if (nb * BN + c * kEpiChunkCols < p.N)
-          epilogue_store_chunk(packed, smem + C::OFF_C, &tm_y, nb * BN + c * kEpiChunkCols, mb * C::BM, es);
-      }
-    }
-    epilogue_finish(es);
-  }
-
-  pdl_release();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 10) tmem_dealloc(tmem, 512);
 }
 
 // --------------------------------------------------------------------------
@@ -661,6 +405,330 @@ ql_status launch_expand_int4_i8(const void* codes, int32_t N, int32_t Kp, void* 
   return cudaGetLastError() == cudaSuccess ? QL_OK : QL_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------------------
+// INT4 weights without the int8 copy, as the MMA's A operand in tensor
+// memory: the widened weights never pass through shared memory.  The tile is
+// transposed, D_c[n, m] = sum_{k in class c} 16 W[n, k] q[m, k]: 128 weight
+// rows on the TMEM lanes (the MMA's M), 128 tokens as the MMA's N.
+//
+// Widening: a nibble moved to the high half of its byte is the int8 value
+// 16 w (the nibble's sign bit lands on the byte's), so one mask, one shift
+// and two byte permutes widen eight codes; the accumulators hold 16 x the
+// integer sums (|16 acc| < 2^31 for K <= 16384), and the epilogue shifts the
+// factor out exactly before the oracle's rounding order
+// s_x (s_norm[n] acc_n + s_out[n] acc_o).
+//
+// Persistent, one CTA (512 to 768 threads) per SM, weight tiles fastest:
+//   warp 0      TMA producer: int8 activation tile (128 tokens x 128 K bytes,
+//               128-byte swizzle) and INT4 weight tile (128 rows x 64 bytes);
+//   warp 1      TMEM allocator and MMA issuer (kind::i8, 128 x 128 x 32, A
+//               from tensor memory; each 32-deep K step goes to its class);
+//   4 XG transform warps (from warp 4), XG groups of four: group g widens
+//               the stages it with it % XG == g; lane l of warp w owns weight
+//               row 32 (w % 4) + l and writes its 128 widened K bytes of a
+//               stage into one of four 32-column A slots with tcgen05.st;
+//   8 epilogue warps: a TMEM lane quarter and half of the 128 token columns
+//               each; y stored in 32 x 32 boxes (tokens x weight rows) by TMA.
+// Tensor memory: normal-class accumulators for two tiles (0-255), ONE
+// outlier-class accumulator (256-383) and the A slots (384-511).  The
+// outlier K steps come last in a tile, so the MMA waits for the previous
+// tile's epilogue to release the outlier accumulator only when it reaches
+// them, while that epilogue has had the whole normal class to run.
+// ---------------------------------------------------------------------------
+template <int RS, int XG>
+struct QarvdTsCfg {
+  static constexpr int BMT = 128;                  // tokens per tile (MMA N)
+  static constexpr int BK = 128;                   // K bytes (int8 elements) per stage
+  static constexpr int AS = 4;                     // A slots of 32 columns
+  static constexpr int ACC_OUT = 2 * BMT;          // outlier accumulator column
+  static constexpr int A_COL = 3 * BMT;            // first A slot column
+  static constexpr int B_BYTES = BMT * BK;         // int8 activations, 128-byte rows
+  static constexpr int W_BYTES = 128 * BK / 2;     // INT4 codes, 64 bytes per weight row
+  static constexpr int OFF_B = 0;
+  static constexpr int OFF_W = OFF_B + RS * B_BYTES;
+  static constexpr int OFF_C = OFF_W + RS * W_BYTES;       // 8 epilogue warps x 2 staging boxes
+  static constexpr int OFF_BAR = OFF_C + 8 * 2 * kWarpBoxBytes;
+  static constexpr int NBAR = 2 * RS + 2 * AS + 2 * 2 + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM = OFF_MISC + 16 + 1024;
+  static constexpr int EPI0 = 4 + 4 * XG;
+  static constexpr int THREADS = (EPI0 + 8) * 32;
+  static constexpr int EPI_CH = BMT / 2 / 32;
+  static_assert(XG >= 1 && XG <= 3, "transform warp groups");
+  static_assert(A_COL + 32 * AS <= 512, "tensor memory budget");
+  static_assert(SMEM <= 232448, "shared memory budget");
+  // kind::i8: D = S32 (2 at bit 4), A = B = signed int8, K-major, N = BMT, M = 128
+  static constexpr uint32_t IDESC =
+      (2u << 4) | (1u << 7) | (1u << 10) | (uint32_t(BMT >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+};
+
+// Eight two's-complement nibbles (byte j: elements 2j low, 2j+1 high) ->
+// eight int8 = 16 x the codes, in element order.
+__device__ __forceinline__ uint2 int4x8_to_int8_x16(uint32_t w) {
+  const uint32_t hi = w & 0xF0F0F0F0u;           // 16 e1, 16 e3, 16 e5, 16 e7
+  const uint32_t lo = (w << 4) & 0xF0F0F0F0u;    // 16 e0, 16 e2, 16 e4, 16 e6
+  return make_uint2(__byte_perm(lo, hi, 0x5140u), __byte_perm(lo, hi, 0x7362u));
+}
+
+template <int RS, int XG>
+__global__ void __launch_bounds__(QarvdTsCfg<RS, XG>::THREADS, 1)
+    k_gemm_qarvd_ts(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                    const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
+  using C = QarvdTsCfg<RS, XG>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* raw_empty = raw_full + RS;
+  uint64_t* xf_full = raw_empty + RS;
+  uint64_t* xf_empty = xf_full + C::AS;
+  uint64_t* tfull = xf_empty + C::AS;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* out_empty = tempty + 2;
+  uint64_t* drain = out_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane = lane_id();
+  if (threadIdx.x == 0) {
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_w);
+    prefetch_tmap(&tm_y);
+    for (int i = 0; i < RS; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_empty[i], 1);   // the stage's MMA commit (issued after the transform read it)
+    }
+    for (int i = 0; i < C::AS; ++i) {
+      mbar_init(&xf_full[i], 4);     // the four transform warps of the stage's group
+      mbar_init(&xf_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 8);
+    }
+    mbar_init(out_empty, 8);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t a_slots = tmem + C::A_COL;
+  pdl_wait();   // before the first global access
+  // class sizes (device-resident, written by the weight preparation)
+  const int k_norm_pad = p.kinfo[1];
+  const int k_out_pad = p.kinfo[3];
+  const int k_used = k_norm_pad + k_out_pad;
+  const int num_kst = (k_used + C::BK - 1) / C::BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (elect_one()) {
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        const int mb = t / p.tiles_n, nb = t - (t / p.tiles_n) * p.tiles_n;
+        for (int ks = 0; ks < num_kst; ++ks, ++it) {
+          const int s = it % RS;
+          if (*abort_flag || !mbar_wait(&raw_empty[s], ((it / RS) & 1) ^ 1, p.wait_limit)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&raw_full[s], C::B_BYTES + C::W_BYTES);
+          tma_load_2d(smem + C::OFF_B + s * C::B_BYTES, &tm_x, &raw_full[s], ks * C::BK, mb * C::BMT);
+          tma_load_2d(smem + C::OFF_W + s * C::W_BYTES, &tm_w, &raw_full[s], ks * (C::BK / 2), nb * 128);
+        }
+      }
+      if (!ok) fail_timeout(p.status, abort_flag);
+      drain_loads(raw_full, it, RS, p.status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      int it = 0, local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++local) {
+        const int acc = local & 1;
+        if (*abort_flag || !mbar_wait(&tempty[acc], ((local >> 1) & 1) ^ 1, p.wait_limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_norm = tmem + acc * C::BMT;
+        const uint32_t d_out = tmem + C::ACC_OUT;
+        bool started_norm = false, started_out = false;
+        for (int ks = 0; ks < num_kst && ok; ++ks, ++it) {
+          const int rs = it % RS, sl = it % C::AS;
+          if (*abort_flag || !mbar_wait(&raw_full[rs], (it / RS) & 1, p.wait_limit) ||
+              !mbar_wait(&xf_full[sl], (it / C::AS) & 1, p.wait_limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t b_base = smem_u32(smem + C::OFF_B + rs * C::B_BYTES);
+#pragma unroll
+          for (int i = 0; i < C::BK / 32; ++i) {
+            const int kk = ks * C::BK + 32 * i;
+            if (kk >= k_used) break;
+            const bool normal = kk < k_norm_pad;
+            if (!normal && !started_out && local > 0) {
+              // the previous tile's epilogue must have read the outlier accumulator
+              if (!mbar_wait(out_empty, (local - 1) & 1, p.wait_limit)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            tc_mma_i8_ts(normal ? d_norm : d_out, a_slots + 32 * sl + 8 * i,
+                         smem_desc(b_base + 32 * i, 0, 1024, kSwizzle128B), C::IDESC,
+                         (normal ? started_norm : started_out) ? 1u : 0u);
+            if (normal) started_norm = true; else started_out = true;
+          }
+          tc_commit(&raw_empty[rs]);
+          tc_commit(&xf_empty[sl]);
+        }
+        if (!ok) break;
+        tc_commit(&tfull[acc]);
+      }
+      if (!ok) fail_timeout(p.status, abort_flag);
+      drain_mma(drain, p.status);
+    }
+  } else if (warp >= 4 && warp < C::EPI0) {
+    // ------------------------------------------------------------ transform
+    const uint32_t q = static_cast<uint32_t>(warp & 3);
+    const uint32_t row = 32 * q + lane;
+    const int group = (warp - 4) >> 2;    // widens the stages it with it % XG == group
+    int it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      for (int ks = 0; ks < num_kst; ++ks, ++it) {
+        if (it % XG != group) continue;
+        const int rs = it % RS, sl = it % C::AS;
+        if (!warp_wait2q(&raw_full[rs], (it / RS) & 1, &xf_empty[sl], ((it / C::AS) & 1) ^ 1, p.wait_limit,
+                         abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint4* wr = reinterpret_cast<const uint4*>(smem + C::OFF_W + rs * C::W_BYTES + row * (C::BK / 2));
+        uint32_t v[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {   // 16 bytes = 32 codes -> 8 words
+          const uint4 r = wr[c];
+          const uint32_t cw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint2 o = int4x8_to_int8_x16(cw[j]);
+            v[8 * c + 2 * j] = o.x;
+            v[8 * c + 2 * j + 1] = o.y;
+          }
+        }
+        tmem_st32(a_slots + ((32 * q) << 16) + 32 * sl, v);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xf_full[sl]);
+      }
+    }
+    if (!ok && lane == 0) fail_timeout(p.status, abort_flag);
+  } else if (warp >= C::EPI0) {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t q = static_cast<uint32_t>(warp & 3);
+    const int half = (warp - C::EPI0) >> 2;
+    const float sx = ld_dep(p.g_a);
+    uint8_t* stage = smem + C::OFF_C + (warp - C::EPI0) * 2 * kWarpBoxBytes;
+    int next = 0, local = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++local) {
+      const int mb = t / p.tiles_n, nb = t - (t / p.tiles_n) * p.tiles_n;
+      const int acc = local & 1;
+      const int n0 = nb * 128 + 32 * static_cast<int>(q);   // this warp's weight rows = output columns
+      const int n = n0 + static_cast<int>(lane);
+      const float sn = (n < p.N) ? __ldg(p.col_scale0 + n) : 0.f;
+      const float so = (n < p.N) ? __ldg(p.col_scale1 + n) : 0.f;
+      if (!warp_wait_uniform(&tfull[acc], (local >> 1) & 1, p.wait_limit, abort_flag, p.status)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < C::EPI_CH; ++c) {
+        const int col = half * (C::BMT / 2) + 32 * c;
+        const int m0 = mb * C::BMT + col;
+        uint32_t an[32], ao[32];
+        tmem_ld32(tmem + ((32 * q) << 16) + acc * C::BMT + col, an);
+        if (k_out_pad) tmem_ld32(tmem + ((32 * q) << 16) + C::ACC_OUT + col, ao);
+        tmem_ld_wait();
+        if (c == C::EPI_CH - 1) {   // both accumulators read: release them
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&tempty[acc]);
+            mbar_arrive(out_empty);
+          }
+        }
+        if (m0 >= p.M || n0 >= p.N) continue;   // warp-uniform: the box is outside Y
+        uint8_t* buf = stage + next * kWarpBoxBytes;
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(buf) + lane;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          // 16 x the integer sums: the shift is exact
+          const float fn = k_norm_pad ? static_cast<float>(static_cast<int32_t>(an[j]) >> 4) : 0.f;
+          const float fo = k_out_pad ? static_cast<float>(static_cast<int32_t>(ao[j]) >> 4) : 0.f;
+          const float v = __fadd_rn(__fmul_rn(sn, fn), __fmul_rn(so, fo));
+          dst[32 * j] = __float2bfloat16_rn(__fmul_rn(sx, v));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, buf, n0, m0);
+          bulk_commit();
+        }
+        next ^= 1;
+      }
+    }
+    epilogue_warp_finish();
+  }
+
+  pdl_release();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+template <int RS, int XG>
+static ql_status launch_qarvd_ts(const void* a_codes, const float* s_x, int64_t M, const ql_weights* w, void* Y,
+                                 cudaStream_t st, int* status) {
+  using C = QarvdTsCfg<RS, XG>;
+  const int N = w->N, Kp = w->Kp;
+  CUtensorMap tx, tw, ty;
+  if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kp, M, Kp, C::BK, C::BMT,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, Kp / 2, N, Kp / 2, C::BK / 2, 128,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<int64_t>(N) * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_NONE))
+    return QL_ERR_CUDA;
+  GemmArgs p{};
+  fill_gemm_args(p, M, N, Kp, 128, status);
+  p.tiles_m = static_cast<int32_t>((M + C::BMT - 1) / C::BMT);
+  p.num_tiles = p.tiles_m * p.tiles_n;
+  p.g_a = s_x;
+  p.col_scale0 = w->s_norm;
+  p.col_scale1 = w->s_out;
+  p.kinfo = w->kinfo;
+  auto kern = k_gemm_qarvd_ts<RS, XG>;
+  if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
+  const int grid = std::min(p.num_tiles, num_sms());
+  if (launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, tx, tw, ty, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QL_ERR_CUDA;
+  }
+  return QL_OK;
+}
+
 ql_status launch_gemm_qarvd(const void* a_codes, const float* s_x, int64_t M, const ql_weights* w, void* Y,
                             cudaStream_t st, int* status) {
   if (M == 0) return QL_OK;
@@ -668,31 +736,7 @@ ql_status launch_gemm_qarvd(const void* a_codes, const float* s_x, int64_t M, co
     if (M > 128) return launch_qarvd_pre<true, 4, 128, 256>(a_codes, s_x, M, w, Y, st, status);
     return launch_qarvd_pre<false, 5, 128, 128>(a_codes, s_x, M, w, Y, st, status);
   }
-  constexpr int S = 4;
-  using C = QarvdCfg<S>;
-  const int N = w->N, Kp = w->Kp;
-  CUtensorMap ta, tb, ty;
-  if (!make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, Kp, M, Kp, C::BK, C::BM,
-                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes, Kp / 2, N, Kp / 2, C::BK / 2, C::BN,
-                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_tmap_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<int64_t>(N) * 2, 64, 128,
-                    CU_TENSOR_MAP_SWIZZLE_128B))
-    return QL_ERR_CUDA;
-  GemmArgs p{};
-  fill_gemm_args(p, M, N, Kp, C::BN, status);
-  p.g_a = s_x;
-  p.col_scale0 = w->s_norm;
-  p.col_scale1 = w->s_out;
-  p.kinfo = w->kinfo;
-  auto kern = k_gemm_qarvd<S>;
-  if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
-  const int grid = std::min(p.num_tiles, num_sms());
-  if (launch_pdl(kern, dim3(grid), dim3(512), C::SMEM, st, 1, ta, tb, ty, p) != cudaSuccess) {
-    (void)cudaGetLastError();
-    return QL_ERR_CUDA;
-  }
-  return QL_OK;
+  return launch_qarvd_ts<6, 2>(a_codes, s_x, M, w, Y, st, status);
 }
 
 }  // namespace ql

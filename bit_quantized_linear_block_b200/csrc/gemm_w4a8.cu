@@ -354,7 +354,7 @@ static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int
 // N) and writes Y[m, n] = bf16(RN(RN(g_w * alpha_mul) * s_m) * D[n, m]), the
 // rounding of the other forms.
 //
-// Persistent, one CTA (512 or 640 threads) per SM, tiles of 128 weight rows x BMT
+// Persistent, one CTA (512 to 768 threads) per SM, tiles of 128 weight rows x BMT
 // tokens, weight tiles fastest (the CTAs running at once share a few token
 // tiles and sweep the whole weight matrix, which stays in L2):
 //   warp 0      TMA producer: the f16-coded activation tile (BMT x 64,
@@ -362,12 +362,14 @@ static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int
 //               and its 512-byte scale column, into an RS-deep ring;
 //   warp 1      TMEM allocator and MMA issuer (kind::f16, 128 x BMT x 16,
 //               A from tensor memory);
-//   XW transform warps (4 or 8, from warp 4): lane l of warp w owns weight
-//               row 32 (w % 4) + l and 64 / (XW / 4) of the stage's 64 K
-//               elements; it widens the row's FP4 codes times their E4M3
-//               scales to f16 (hardware e2m1x2 -> f16x2 convert, f16
-//               multiply: exact) and writes the words into one of AS
-//               32-column A slots of its TMEM lane with tcgen05.st;
+//   4 XG transform warps (from warp 4), XG groups of four: group g widens
+//               the stages it with it % XG == g, so a stage's widening
+//               latency is spread over XG stages of MMA time.  Lane l of
+//               warp w owns weight row 32 (w % 4) + l; per 64-deep K stage it
+//               widens the row's 64 FP4 codes times their E4M3 scales to f16
+//               (hardware e2m1x2 -> f16x2 convert, f16 multiply: exact) and
+//               writes the 32 words into one of AS 32-column A slots of its
+//               TMEM lane with tcgen05.st;
 //   8 epilogue warps (after the transform warps): warp w reads TMEM lane
 //               quarter w % 4 and half of the BMT columns, scales column m
 //               by s_m, and stores 32 x 32 boxes of Y (tokens x weight rows)
@@ -375,7 +377,7 @@ static ql_status launch_w4a8_cfg(const void* a_codes, const float* a_scales, int
 // Tensor memory: two BMT-column accumulators (one for BMT = 256) and
 // AS = (512 - NACC BMT) / 32 A slots.  All waits are bounded (the W4A4 kernel's timeout protocol).
 // ---------------------------------------------------------------------------
-template <int BMT, int RS, int XW>
+template <int BMT, int RS, int XG>
 struct W4A8TsCfg {
   static constexpr int BK = 64;                    // K elements per stage
   // two accumulators where they leave room for four A slots, else one
@@ -392,11 +394,10 @@ struct W4A8TsCfg {
   static constexpr int NBAR = 2 * RS + 2 * AS + 2 * 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM = OFF_MISC + 16 + 1024;
-  static constexpr int EPI0 = 4 + XW;              // first epilogue warp
+  static constexpr int EPI0 = 4 + 4 * XG;          // first epilogue warp
   static constexpr int THREADS = (EPI0 + 8) * 32;
-  static constexpr int KPT = 64 / (XW / 4);         // K elements per transform thread and stage
   static constexpr int EPI_CH = BMT / 2 / 32;      // 32-column boxes per epilogue warp and tile
-  static_assert(XW == 4 || XW == 8, "transform warps");
+  static_assert(XG >= 1 && XG <= 3, "transform warp groups");
   static_assert(AS >= 2, "tensor memory budget");
   static_assert(B_BYTES % 1024 == 0 && BMT % 64 == 0, "swizzled tiles, whole epilogue boxes");
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -404,11 +405,11 @@ struct W4A8TsCfg {
   static constexpr uint32_t IDESC = (1u << 4) | (uint32_t(BMT >> 3) << 17) | (uint32_t(128 >> 4) << 24);
 };
 
-template <int BMT, int RS, int XW>
-__global__ void __launch_bounds__(W4A8TsCfg<BMT, RS, XW>::THREADS, 1)
+template <int BMT, int RS, int XG>
+__global__ void __launch_bounds__(W4A8TsCfg<BMT, RS, XG>::THREADS, 1)
     k_gemm_w4a8_ts(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                    const __grid_constant__ CUtensorMap tm_y, const GemmArgs p) {
-  using C = W4A8TsCfg<BMT, RS, XW>;
+  using C = W4A8TsCfg<BMT, RS, XG>;
   if (p.gate != nullptr) {   // device-routed forward
     pdl_wait();
     if (gated_off(p.gate, p.gate_value)) {
@@ -439,7 +440,7 @@ __global__ void __launch_bounds__(W4A8TsCfg<BMT, RS, XW>::THREADS, 1)
       mbar_init(&raw_empty[i], 1);   // the stage's MMA commit (issued after the transform read it)
     }
     for (int i = 0; i < C::AS; ++i) {
-      mbar_init(&xf_full[i], XW);    // the transform warps
+      mbar_init(&xf_full[i], 4);     // the four transform warps of the stage's group
       mbar_init(&xf_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -520,11 +521,12 @@ __global__ void __launch_bounds__(W4A8TsCfg<BMT, RS, XW>::THREADS, 1)
     // ------------------------------------------------------------ transform
     const uint32_t q = static_cast<uint32_t>(warp & 3);
     const uint32_t row = 32 * q + lane;   // weight row within the tile = TMEM lane
-    const uint32_t kh = static_cast<uint32_t>(warp - 4) >> 2;   // this warp's share of the stage's K
+    const int group = (warp - 4) >> 2;    // widens the stages it with it % XG == group
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
       for (int ks = 0; ks < p.num_kst; ++ks, ++it) {
+        if (it % XG != group) continue;
         const int rs = it % RS, sl = it % C::AS;
         if (!warp_wait2(&raw_full[rs], (it / RS) & 1, &xf_empty[sl], ((it / C::AS) & 1) ^ 1, p.wait_limit,
                         abort_flag)) {
@@ -534,35 +536,19 @@ __global__ void __launch_bounds__(W4A8TsCfg<BMT, RS, XW>::THREADS, 1)
         tc_fence_after();
         // scale atom: byte (row % 32) * 16 + (row / 32) * 4 + k16 holds the block scale of K block k16
         const uint32_t sb4 = *reinterpret_cast<const uint32_t*>(smem + C::OFF_SF + rs * C::SF_BYTES + lane * 16 + q * 4);
-        const uint4* wr = reinterpret_cast<const uint4*>(smem + C::OFF_W + rs * C::W_BYTES + row * 32 + kh * (C::KPT / 2));
-        const uint32_t col = a_slots + ((32 * q) << 16) + 32 * sl + kh * (C::KPT / 2);
-        if constexpr (XW == 4) {
-          const uint4 c0 = wr[0], c1 = wr[1];
-          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          uint32_t v[32];
+        const uint4* wr = reinterpret_cast<const uint4*>(smem + C::OFF_W + rs * C::W_BYTES + row * 32);
+        const uint4 c0 = wr[0], c1 = wr[1];
+        const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        uint32_t v[32];
 #pragma unroll
-          for (int w8 = 0; w8 < 8; ++w8) {   // codes 8 w8 .. 8 w8 + 7: half of block w8 / 2
-            const uint4 o = fp4x8_scaled_to_f16(cw[w8], (sb4 >> (8 * (w8 >> 1))) & 0xFFu);
-            v[4 * w8] = o.x;
-            v[4 * w8 + 1] = o.y;
-            v[4 * w8 + 2] = o.z;
-            v[4 * w8 + 3] = o.w;
-          }
-          tmem_st32(col, v);
-        } else {   // K elements 32 kh .. 32 kh + 31: blocks 2 kh, 2 kh + 1
-          const uint4 c0 = wr[0];
-          const uint32_t cw[4] = {c0.x, c0.y, c0.z, c0.w};
-          uint32_t v[16];
-#pragma unroll
-          for (int w8 = 0; w8 < 4; ++w8) {
-            const uint4 o = fp4x8_scaled_to_f16(cw[w8], (sb4 >> (8 * (2 * kh + (w8 >> 1)))) & 0xFFu);
-            v[4 * w8] = o.x;
-            v[4 * w8 + 1] = o.y;
-            v[4 * w8 + 2] = o.z;
-            v[4 * w8 + 3] = o.w;
-          }
-          tmem_st16(col, v);
+        for (int w8 = 0; w8 < 8; ++w8) {   // codes 8 w8 .. 8 w8 + 7: half of block w8 / 2
+          const uint4 o = fp4x8_scaled_to_f16(cw[w8], (sb4 >> (8 * (w8 >> 1))) & 0xFFu);
+          v[4 * w8] = o.x;
+          v[4 * w8 + 1] = o.y;
+          v[4 * w8 + 2] = o.z;
+          v[4 * w8 + 3] = o.w;
         }
+        tmem_st32(a_slots + ((32 * q) << 16) + 32 * sl, v);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -625,10 +611,10 @@ __global__ void __launch_bounds__(W4A8TsCfg<BMT, RS, XW>::THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-template <int BMT, int RS, int XW>
+template <int BMT, int RS, int XG>
 static ql_status launch_w4a8_ts_cfg(const void* a_codes, const float* a_scales, int64_t M, const ql_weights* w,
                                     void* Y, cudaStream_t st, int* status, Gate gate) {
-  using C = W4A8TsCfg<BMT, RS, XW>;
+  using C = W4A8TsCfg<BMT, RS, XG>;
   const int N = w->N, K = w->K;
   CUtensorMap tx, tw, ty;
   if (!make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, a_codes, K, M, static_cast<int64_t>(K) * 2, C::BK, BMT,
@@ -651,7 +637,7 @@ static ql_status launch_w4a8_ts_cfg(const void* a_codes, const float* a_scales, 
   p.alpha_mul = w->hadamard ? (1.0f / 128.0f) : 1.0f;
   p.gate = gate.route;
   p.gate_value = gate.value;
-  auto kern = k_gemm_w4a8_ts<BMT, RS, XW>;
+  auto kern = k_gemm_w4a8_ts<BMT, RS, XG>;
   if (!set_smem_attr(reinterpret_cast<const void*>(kern), C::SMEM)) return QL_ERR_CUDA;
   const int grid = std::min(p.num_tiles, num_sms());
   if (launch_pdl(kern, dim3(grid), dim3(C::THREADS), C::SMEM, st, 1, tx, tw, ty, p) != cudaSuccess) {
@@ -667,7 +653,7 @@ ql_status launch_gemm_w4a8(const void* a_codes, const float* a_scales, int64_t M
   const bool n192 = w->N % 192 == 0;
   if (a_f16) {
     // without the weight copy: the weights widened into tensor memory
-    if (w->w16 == nullptr) return launch_w4a8_ts_cfg<192, 6, 8>(a_codes, a_scales, M, w, Y, st, status, gate);
+    if (w->w16 == nullptr) return launch_w4a8_ts_cfg<192, 6, 2>(a_codes, a_scales, M, w, Y, st, status, gate);
     // f16 activations and pre-expanded weights: both operands by TMA
     if (n192) return launch_w4a8_cfg<192, 1, 4, true, true>(a_codes, a_scales, M, w, Y, st, status, gate);
     return launch_w4a8_cfg<128, 1, 5, true, true>(a_codes, a_scales, M, w, Y, st, status, gate);

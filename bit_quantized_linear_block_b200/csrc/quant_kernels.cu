@@ -456,6 +456,15 @@ __global__ void __launch_bounds__(kQuantThreads, 1)
 // converts two codes per instruction.  The rounding is a conversion of the
 // rounded product, never an addition after it: the compiler may fuse a
 // product and a following addition into one FMA, which rounds once.
+// rint(RN(x * inv)) in the low byte of the result, for |RN(x * inv)| < 2^22:
+// RN(y + 1.5 * 2^23) holds rint(y) (RN to even) in its low mantissa bits.
+// __fmul_rn and __fadd_rn are never contracted into one FMA (which would
+// round x * inv + 1.5 * 2^23 once and differ where RN(x * inv) is a
+// half-integer); the packed f32x2 forms gave exactly that difference.
+__device__ __forceinline__ int rint_low_byte(float x, float inv) {
+  return static_cast<int>(__float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.0f)));
+}
+
 __device__ __forceinline__ uint32_t pack4_s8(int a0, int a1, int a2, int a3) {
   const uint32_t t01 = __byte_perm(static_cast<uint32_t>(a0), static_cast<uint32_t>(a1), 0x0040);
   const uint32_t t23 = __byte_perm(static_cast<uint32_t>(a2), static_cast<uint32_t>(a3), 0x0040);
@@ -601,8 +610,9 @@ __global__ void __launch_bounds__(kThreadsHbm)
 // round-robin, so a group's ragged unit count does not load one warp more
 // than the others.
 //
-// Codes: rint(RN(x * RN(qmax / amax))), low bytes packed by byte permutes;
-// no clamp is needed, as in the per-token quantizer (|y| < qmax + 1/2).
+// Codes: rint(RN(x * RN(qmax / amax))) by rint_low_byte, low bytes packed
+// by byte permutes; no clamp is needed, as in the per-token quantizer
+// (|y| < qmax + 1/2).
 // ---------------------------------------------------------------------------
 constexpr int kPermMaxRing = 4;
 constexpr int kPermThreads = 256;
@@ -660,7 +670,6 @@ __global__ void __launch_bounds__(kPermThreads)
   const float fq = static_cast<float>(qmax);
   const float inv = (amax == 0.f) ? 0.f : __fdiv_rn(fq, amax);
   if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = (amax == 0.f) ? 0.f : __fdiv_rn(amax, fq);
-  const float2 inv2 = make_float2(inv, inv);
   __syncthreads();   // gather table complete
   const int32_t upr = (Kp + kPermUnit - 1) / kPermUnit;   // units per row
   int32_t deal = 0;                                       // units dealt before this group, mod kPermWarps
@@ -709,9 +718,9 @@ __global__ void __launch_bounds__(kPermThreads)
                                          __uint_as_float(static_cast<uint32_t>(xr[gi.x >> 16]) << 16));
           const float2 v23 = make_float2(__uint_as_float(static_cast<uint32_t>(xr[gi.y & 0xFFFFu]) << 16),
                                          __uint_as_float(static_cast<uint32_t>(xr[gi.y >> 16]) << 16));
-          const float2 y01 = __fmul2_rn(v01, inv2), y23 = __fmul2_rn(v23, inv2);
           *reinterpret_cast<uint32_t*>(dst + j) =
-              pack4_s8(__float2int_rn(y01.x), __float2int_rn(y01.y), __float2int_rn(y23.x), __float2int_rn(y23.y));
+              pack4_s8(rint_low_byte(v01.x, inv), rint_low_byte(v01.y, inv), rint_low_byte(v23.x, inv),
+                       rint_low_byte(v23.y, inv));
         }
       }
     }
