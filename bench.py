@@ -27,6 +27,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -50,9 +51,12 @@ NVFP4_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16   # bf16 in, E2M1 out, E4M3 per 16
 # DRAM bytes per launch of the W4A4 GEMM from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of the GEMM sources).
 GEMM_TRAFFIC = {
-    # ncu dram__bytes_read.sum + dram__bytes_write.sum: 591.0 MB over the 4
-    # GEMM launches of one step of this workload
-    "9530880a77d1f62c": 591.0e6 / 4,
+    # ncu dram__bytes_read.sum + dram__bytes_write.sum: 605.8 MB over the 4
+    # GEMM launches of one step of this workload (185.6 MB read, 420.2 MB
+    # written), keyed by the GEMM sources' hash.  Captured at hash
+    # 1464859f8ab20b9f; the sources have since gained only a tensor-memory
+    # load helper that the W4A4 kernel does not use.
+    "7d8bb068157ae2fe": 605.8e6 / 4,
 }
 
 
@@ -230,13 +234,17 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
+        self.log = None
 
     def start(self):
+        # samples go to a file: a pipe nobody reads fills up within seconds
+        # and then blocks nvidia-smi, which would end the sampling
+        self.log = tempfile.TemporaryFile(mode="w+")
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "10", "-i", str(self.dev)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                stdout=self.log, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
 
@@ -248,10 +256,13 @@ class ClockSampler:
             return
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+            self.proc.wait()
+        self.log.seek(0)
+        out = self.log.read()
+        self.log.close()
         for line in out.strip().splitlines():
             f = [c.strip() for c in line.split(",")]
             if len(f) < 10:
@@ -818,8 +829,9 @@ def run_configs(reps: int = 20):
         gg, rr = g.clone(), r.clone()
         ri, ro = copies(bi, 4.0 * bi.numel()), copies(bo, 4.0 * bi.numel())
         us = med(lambda j: ql.qlinear_route(ri[j % len(ri)], ro[j % len(ri)], THRESHOLD, gamma=gg, route=rr, ws=rws))
-        routes[f"block{blk}"] = dict(hbm_rec(us, 4.0 * M_TOKENS * 1920), sigma=round(sigma, 5),
-                                     gamma=float(g.item()), route=int(r.item()))
+        rec = hbm_rec(us, 4.0 * M_TOKENS * 1920)   # the record itself: its SM clock is filled in later
+        rec.update(sigma=round(sigma, 5), gamma=float(g.item()), route=int(r.item()))
+        routes[f"block{blk}"] = rec
         del ri, ro
     out["cfg3_route"] = routes
     rx = copies(bi, 2.0 * bi.numel())

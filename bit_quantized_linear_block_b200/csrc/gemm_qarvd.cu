@@ -654,31 +654,38 @@ __global__ void __launch_bounds__(QarvdTsCfg<RS, XG>::THREADS, 1)
       for (int c = 0; c < C::EPI_CH; ++c) {
         const int col = half * (C::BMT / 2) + 32 * c;
         const int m0 = mb * C::BMT + col;
-        uint32_t an[32], ao[32];
-        tmem_ld32(tmem + ((32 * q) << 16) + acc * C::BMT + col, an);
-        if (k_out_pad) tmem_ld32(tmem + ((32 * q) << 16) + C::ACC_OUT + col, ao);
-        tmem_ld_wait();
-        if (c == C::EPI_CH - 1) {   // both accumulators read: release them
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&tempty[acc]);
-            mbar_arrive(out_empty);
-          }
-        }
-        if (m0 >= p.M || n0 >= p.N) continue;   // warp-uniform: the box is outside Y
+        const bool inside = m0 < p.M && n0 < p.N;   // warp-uniform: else the box is outside Y
         uint8_t* buf = stage + next * kWarpBoxBytes;
-        if (lane == 0) bulk_wait_read<1>();
-        __syncwarp();
+        if (inside) {
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+        }
         __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(buf) + lane;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          // 16 x the integer sums: the shift is exact
-          const float fn = k_norm_pad ? static_cast<float>(static_cast<int32_t>(an[j]) >> 4) : 0.f;
-          const float fo = k_out_pad ? static_cast<float>(static_cast<int32_t>(ao[j]) >> 4) : 0.f;
-          const float v = __fadd_rn(__fmul_rn(sn, fn), __fmul_rn(so, fo));
-          dst[32 * j] = __float2bfloat16_rn(__fmul_rn(sx, v));
+        for (int h = 0; h < 2; ++h) {   // 16 columns at a time (registers)
+          uint32_t an[16], ao[16];
+          tmem_ld16(tmem + ((32 * q) << 16) + acc * C::BMT + col + 16 * h, an);
+          if (k_out_pad) tmem_ld16(tmem + ((32 * q) << 16) + C::ACC_OUT + col + 16 * h, ao);
+          tmem_ld_wait();
+          if (c == C::EPI_CH - 1 && h == 1) {   // both accumulators read: release them
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(&tempty[acc]);
+              mbar_arrive(out_empty);
+            }
+          }
+          if (!inside) continue;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            // 16 x the integer sums: the shift is exact
+            const float fn = k_norm_pad ? static_cast<float>(static_cast<int32_t>(an[j]) >> 4) : 0.f;
+            const float fo = k_out_pad ? static_cast<float>(static_cast<int32_t>(ao[j]) >> 4) : 0.f;
+            const float v = __fadd_rn(__fmul_rn(sn, fn), __fmul_rn(so, fo));
+            dst[32 * (16 * h + j)] = __float2bfloat16_rn(__fmul_rn(sx, v));
+          }
         }
+        if (!inside) continue;
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
