@@ -54,9 +54,9 @@ GEMM_TRAFFIC = {
     # ncu dram__bytes_read.sum + dram__bytes_write.sum: 605.8 MB over the 4
     # GEMM launches of one step of this workload (185.6 MB read, 420.2 MB
     # written), keyed by the GEMM sources' hash.  Captured at hash
-    # 1464859f8ab20b9f; the sources have since gained only a tensor-memory
-    # load helper that the W4A4 kernel does not use.
-    "7d8bb068157ae2fe": 605.8e6 / 4,
+    # 1464859f8ab20b9f; the sources have since changed only in tensor-memory
+    # load/store helpers that the W4A4 kernel does not use.
+    "c71c5df16e5feb64": 605.8e6 / 4,
 }
 
 
