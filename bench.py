@@ -253,6 +253,9 @@ class ClockSampler:
         active throttle reasons)."""
         self.samples = []
         if self.proc is None:
+            if self.log is not None:
+                self.log.close()
+                self.log = None
             return
         self.proc.terminate()
         try:
